@@ -1,0 +1,136 @@
+/*
+ * dilattn -- LongNet dilated attention, forward and backward, on one B200
+ * (sm_100a). C ABI: plain pointers and sizes, nothing from PyTorch.
+ *
+ * The operation (from the LongNet pages: the gptget.net summary of arXiv
+ * 2307.02486, sections "方法论" and "方法详解"; its abstract, printed on every
+ * page; and the DarcStar commentary on the darcstar.tech page):
+ *
+ *   For each pattern i = (w_i, r_i) and head h, the length-N sequence is cut
+ *   into segments [s*w_i, min((s+1)*w_i, N)); segment s keeps rows
+ *   s*w_i + (h mod r_i) + k*r_i below its end ("方法详解": equal segments,
+ *   several dilation rates, a different offset per head). Softmax attention
+ *   with scale 1/sqrt(d) runs on the kept rows of each segment, causal in
+ *   position order when causal = 1 (abstract: a drop-in replacement for
+ *   standard attention). The per-pattern results of a row are merged as
+ *   O = sum_i Z_i O_i / sum_j Z_j, Z_i being pattern i's softmax
+ *   denominator, carried as a log-sum-exp (DarcStar commentary: the shared
+ *   denominator must stay exact). Rows no pattern keeps get O = 0 and
+ *   lse = -inf. The merged result equals one softmax over the multiset
+ *   union of the keys the patterns give the row.
+ *
+ * Layouts (all row-major, last index fastest):
+ *   q, k, v, out, dout, dq, dk, dv : [B][N][H][d]
+ *   lse                            : [B][H][N] float32, natural log
+ * Element types: the unsuffixed entry points take bfloat16 tensors (stored as
+ * 16-bit words) and compute in fp32 with bf16 tensor-core products; the _f32
+ * entry points take float32 tensors and compute in plain fp32.
+ *
+ * Ownership: every tensor pointer is a DEVICE pointer owned by the caller;
+ * the library keeps no reference after the call returns. w and r are HOST
+ * arrays of npat ints, read before the call returns. Workspaces are
+ * caller-owned device memory of at least the size the matching
+ * *_workspace_size function returns, 256-byte aligned; their contents on
+ * entry do not matter and are garbage on return.
+ *
+ * Asynchrony: every compute entry point validates its arguments, enqueues
+ * its kernels on `stream` and returns; faults during execution surface at the
+ * caller's next synchronisation (ordinary CUDA semantics). Nothing throws
+ * across the ABI. A status of DILATTN_ERR_CUDA leaves the CUDA error message
+ * in dilattn_last_error().
+ *
+ * Constraints checked on every call (violations return
+ * DILATTN_ERR_INVALID_ARG or DILATTN_ERR_UNSUPPORTED and launch nothing):
+ *   B, N, H >= 1; 1 <= npat <= DILATTN_MAX_PATTERNS; w_i >= 1; r_i >= 1;
+ *   causal in {0, 1}; B*N*H*d < 2^40; tensor pointers non-NULL and 16-byte
+ *   aligned; outputs do not alias inputs; d in {64, 128}; the current device
+ *   has compute capability 10.x.
+ */
+#ifndef DILATTN_H
+#define DILATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define DILATTN_MAX_PATTERNS 16
+
+enum dilattn_status {
+  DILATTN_OK = 0,
+  DILATTN_ERR_INVALID_ARG = 1,  /* bad shape, pointer, alignment or pattern */
+  DILATTN_ERR_UNSUPPORTED = 2,  /* d not in {64, 128}, or device not CC 10.x */
+  DILATTN_ERR_CUDA = 3,         /* a CUDA call or launch failed */
+  DILATTN_ERR_WORKSPACE = 4,    /* workspace NULL, misaligned or too small */
+  DILATTN_ERR_INTERNAL = 5      /* a kernel reported an internal failure */
+};
+
+/* Human-readable name of a status code (static string). */
+const char* dilattn_status_string(int status);
+
+/* Message of the last CUDA error this thread saw inside the library ("" if none). */
+const char* dilattn_last_error(void);
+
+/*
+ * Forward. Writes out [B][N][H][d] bf16 and, unless lse is NULL,
+ * lse [B][H][N] fp32. Workspace: fp32 per-pattern partial results
+ * (one row of d + 1 floats per kept row of every pattern), at least
+ * dilattn_fwd_workspace_size(...) bytes.
+ */
+size_t dilattn_fwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
+                                  int npat);
+int dilattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                int B, int N, int H, int d, const int* w, const int* r, int npat, int causal,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Backward of dilattn_fwd: given out and lse from the forward and the
+ * output gradient dout (all device), writes dq, dk, dv [B][N][H][d] bf16, the
+ * full derivative of sum(out * dout). The probabilities are recomputed from
+ * the saved lse. Workspace: fp32 accumulators for dq, dk, dv and the row
+ * term D = rowsum(dout * out), at least dilattn_bwd_workspace_size(...) bytes.
+ */
+size_t dilattn_bwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
+                                  int npat);
+int dilattn_bwd(const void* q, const void* k, const void* v, const void* out,
+                const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                int B, int N, int H, int d, const int* w, const int* r, int npat, int causal,
+                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * fp32 forward and backward (same semantics, float32 tensors, no workspace,
+ * full fp32 FMA arithmetic without TF32). Meant for small problems: each
+ * output row is computed by one thread.
+ */
+int dilattn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse,
+                    int B, int N, int H, int d, const int* w, const int* r, int npat,
+                    int causal, cudaStream_t stream);
+int dilattn_bwd_f32(const float* q, const float* k, const float* v, const float* out,
+                    const float* lse, const float* dout, float* dq, float* dk, float* dv,
+                    int B, int N, int H, int d, const int* w, const int* r, int npat,
+                    int causal, cudaStream_t stream);
+
+/*
+ * Row selection, as the attention kernels see it: sig [H][N] (device,
+ * uint32) receives bit i at (h, n) when pattern i keeps row n for head h.
+ * It enumerates kept rows with the same segment/offset code the attention
+ * kernels use to address their tiles, so it checks that code bit for bit.
+ */
+int dilattn_selection(uint32_t* sig, int N, int H, const int* w, const int* r, int npat,
+                      cudaStream_t stream);
+
+/*
+ * Reads and clears the library's device-side error word on the current
+ * device after synchronising `stream`. *code receives 0 when no kernel
+ * reported a failure (a bounded wait that ran out sets a nonzero code).
+ */
+int dilattn_device_error(cudaStream_t stream, int* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DILATTN_H */

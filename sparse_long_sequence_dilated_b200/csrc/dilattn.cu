@@ -1,0 +1,460 @@
+// libdilattn: C-ABI entry points (validation, TMA descriptor set-up, launches).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+#include <vector>
+
+#include "dilattn.h"
+#include "common.cuh"
+#include "fwd_tc.cuh"
+#include "simt.cuh"
+
+namespace dil {
+
+__device__ int g_dev_error;  // device-side error word (bounded waits that ran out)
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+int cuda_fail(cudaError_t e, const char* what) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", what, cudaGetErrorString(e),
+           (int)e);
+  return DILATTN_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ device state
+struct DeviceState {
+  bool init = false;
+  bool arch_ok = false;
+  int* err_word = nullptr;
+  int num_sms = 0;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceState> g_devices;
+
+int device_state(DeviceState** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& st = g_devices[dev];
+  if (!st.init) {
+    int major = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+    st.arch_ok = (major == 10);
+    if (st.arch_ok) {
+      e = cudaDeviceGetAttribute(&st.num_sms, cudaDevAttrMultiProcessorCount, dev);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+      e = cudaGetSymbolAddress(reinterpret_cast<void**>(&st.err_word), g_dev_error);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+      e = cudaFuncSetAttribute(fwd_tile_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<64>::SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      e = cudaFuncSetAttribute(fwd_tile_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<128>::SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+    }
+    st.init = true;
+  }
+  if (!st.arch_ok) return DILATTN_ERR_UNSUPPORTED;
+  *out = &st;
+  return DILATTN_OK;
+}
+
+// ------------------------------------------------------------------ TMA descriptors
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+int get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+    return DILATTN_ERR_CUDA;
+  }
+  return DILATTN_OK;
+}
+
+// Strided view of a [B][N][H][d] bf16 tensor that gathers every r-th row:
+// dims {d, H, r, ceil(N / r), B}, byte strides {2d, 2Hd, 2Hdr, 2HdN}, base
+// shifted back by `shift` rows so that row p sits at phase (p + shift) mod r,
+// index (p + shift) / r. Rows at or past N fall outside the view and read as
+// zeros; rows before 0 are never addressed because every tile starts at a
+// kept row >= 0. Box: 64 columns (128 bytes, 128-byte swizzle) x 128 rows.
+using MapKey = std::tuple<const void*, int, int, int, int, int, int, int>;
+std::mutex g_map_mu;
+std::map<MapKey, CUtensorMap> g_maps;
+
+int strided_map(const void* ptr, int B, int N, int H, int d, int r, int shift, CUtensorMap* out) {
+  MapKey key{ptr, B, N, H, d, r, shift, 0};
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *out = it->second;
+      return DILATTN_OK;
+    }
+  }
+  int rc = get_encoder();
+  if (rc != DILATTN_OK) return rc;
+  const long long rowb = (long long)H * d * 2;
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)r,
+                        (cuuint64_t)(((long long)N + shift) / r), (cuuint64_t)B};
+  cuuint64_t strides[4] = {(cuuint64_t)d * 2, (cuuint64_t)rowb, (cuuint64_t)(rowb * r),
+                           (cuuint64_t)(rowb * N)};
+  cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)BM, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  void* base = (void*)((const char*)ptr - (long long)shift * rowb);
+  CUtensorMap m;
+  CUresult cr = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)cr);
+    return DILATTN_ERR_CUDA;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    if (g_maps.size() > 4096) g_maps.clear();
+    g_maps[key] = m;
+  }
+  *out = m;
+  return DILATTN_OK;
+}
+
+// ------------------------------------------------------------------ validation
+int check_shape(int B, int N, int H, int d, const int* w, const int* r, int npat, int causal) {
+  if (B < 1 || N < 1 || H < 1 || d < 1) return DILATTN_ERR_INVALID_ARG;
+  if (npat < 1 || npat > DILATTN_MAX_PATTERNS || w == nullptr || r == nullptr)
+    return DILATTN_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return DILATTN_ERR_INVALID_ARG;
+  const double elems = (double)B * N * H * d;
+  if (elems >= 1099511627776.0) return DILATTN_ERR_INVALID_ARG;
+  for (int i = 0; i < npat; ++i) {
+    if (w[i] < 1 || r[i] < 1) return DILATTN_ERR_INVALID_ARG;
+    if ((double)r[i] * H * d * 4 >= 1099511627776.0) return DILATTN_ERR_INVALID_ARG;
+  }
+  return DILATTN_OK;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
+  const char* x = (const char*)a;
+  const char* y = (const char*)b;
+  return x < y + bn && y < x + an;
+}
+
+long long make_geoms(int B, int N, int H, const int* w, const int* r, int npat,
+                     PatternGeom* geo) {
+  long long rows = 0;
+  for (int i = 0; i < npat; ++i) {
+    PatternGeom& g = geo[i];
+    g.w = w[i];
+    g.r = r[i];
+    g.nseg = (int)(((long long)N + w[i] - 1) / w[i]);
+    const long long span = std::min<long long>(w[i], N);
+    g.nmax = (int)((span + r[i] - 1) / r[i]);
+    g.ntiles = (g.nmax + BM - 1) / BM;
+    g.shift = (int)((r[i] - N % r[i]) % r[i]);
+    g.part_base = rows;
+    rows += (long long)B * H * g.nseg * g.nmax;
+  }
+  return rows;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Longest-first unit order for the tile kernel (see FwdParams).
+long long make_schedule(FwdParams& p) {
+  std::vector<int> order(p.npat);
+  for (int i = 0; i < p.npat; ++i) order[i] = i;
+  std::stable_sort(order.begin(), order.end(),
+                   [&](int a, int b) { return p.pat[a].ntiles > p.pat[b].ntiles; });
+  std::vector<int> vals;
+  for (int i : order)
+    if (vals.empty() || vals.back() != p.pat[i].ntiles) vals.push_back(p.pat[i].ntiles);
+  for (int i = 0; i < p.npat; ++i) p.order[i] = order[i];
+  p.nband = (int)vals.size();
+  p.band_start[0] = 0;
+  for (int j = 0; j < p.nband; ++j) {
+    const int lo = j + 1 < p.nband ? vals[j + 1] : 0;
+    p.band_nt[j] = vals[j];
+    int act = 0;
+    long long per = 0;
+    for (int a = 0; a < p.npat; ++a) {
+      if (p.pat[order[a]].ntiles >= vals[j]) {
+        ++act;
+        per += (long long)p.pat[order[a]].nseg * p.B * p.H;
+      }
+    }
+    p.band_npat[j] = act;
+    p.band_per_level[j] = per;
+    p.band_start[j + 1] = p.band_start[j] + (long long)(vals[j] - lo) * per;
+  }
+  p.band_nt[p.nband] = 0;
+  return p.band_start[p.nband];
+}
+
+template <int D>
+int launch_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N,
+               int H, const int* w, const int* r, int npat, int causal, void* ws,
+               DeviceState* st, cudaStream_t stream) {
+  static_assert(sizeof(FwdParams) < 32000, "kernel parameter block too large");
+  FwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.npat = npat;
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  p.causal = causal;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  const long long rows = make_geoms(B, N, H, w, r, npat, p.pat);
+  p.part_o = reinterpret_cast<float*>(ws);
+  p.part_lse = reinterpret_cast<float*>((char*)ws + align256((size_t)rows * D * 4));
+  p.err = st->err_word;
+  for (int i = 0; i < npat; ++i) {
+    int rc = strided_map(q, B, N, H, D, r[i], p.pat[i].shift, &p.tmq[i]);
+    if (rc == DILATTN_OK) rc = strided_map(k, B, N, H, D, r[i], p.pat[i].shift, &p.tmk[i]);
+    if (rc == DILATTN_OK) rc = strided_map(v, B, N, H, D, r[i], p.pat[i].shift, &p.tmv[i]);
+    if (rc != DILATTN_OK) return rc;
+  }
+  const long long units = make_schedule(p);
+  if (units > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
+  fwd_tile_kernel<D><<<(unsigned)units, 192, FwdCfg<D>::SMEM_BYTES, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fwd_tile_kernel launch");
+
+  MergeParams mp;
+  memset(&mp, 0, sizeof(mp));
+  memcpy(mp.pat, p.pat, sizeof(mp.pat));
+  mp.npat = npat;
+  mp.B = B;
+  mp.N = N;
+  mp.H = H;
+  mp.part_o = p.part_o;
+  mp.part_lse = p.part_lse;
+  mp.out = reinterpret_cast<__nv_bfloat16*>(out);
+  mp.lse = lse;
+  const long long total_rows = (long long)B * N * H;
+  const long long blocks = (total_rows + 7) / 8;
+  merge_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(mp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "merge_kernel launch");
+  return DILATTN_OK;
+}
+
+RowParams make_row_params(int B, int N, int H, int d, const int* w, const int* r, int npat,
+                          int causal) {
+  RowParams p;
+  memset(&p, 0, sizeof(p));
+  make_geoms(B, N, H, w, r, npat, p.pat);
+  p.npat = npat;
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  p.causal = causal;
+  p.tau = (float)(1.0 / std::sqrt((double)d));
+  return p;
+}
+
+}  // namespace
+}  // namespace dil
+
+using namespace dil;
+
+extern "C" {
+
+const char* dilattn_status_string(int status) {
+  switch (status) {
+    case DILATTN_OK: return "DILATTN_OK";
+    case DILATTN_ERR_INVALID_ARG: return "DILATTN_ERR_INVALID_ARG";
+    case DILATTN_ERR_UNSUPPORTED: return "DILATTN_ERR_UNSUPPORTED";
+    case DILATTN_ERR_CUDA: return "DILATTN_ERR_CUDA";
+    case DILATTN_ERR_WORKSPACE: return "DILATTN_ERR_WORKSPACE";
+    case DILATTN_ERR_INTERNAL: return "DILATTN_ERR_INTERNAL";
+    default: return "DILATTN_UNKNOWN_STATUS";
+  }
+}
+
+const char* dilattn_last_error(void) { return g_last_error; }
+
+size_t dilattn_fwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
+                                  int npat) {
+  if (check_shape(B, N, H, d, w, r, npat, 1) != DILATTN_OK) return 0;
+  PatternGeom geo[kMaxPat];
+  const long long rows = make_geoms(B, N, H, w, r, npat, geo);
+  return align256((size_t)rows * d * 4) + align256((size_t)rows * 4);
+}
+
+int dilattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N,
+                int H, int d, const int* w, const int* r, int npat, int causal, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream) {
+  int rc = check_shape(B, N, H, d, w, r, npat, causal);
+  if (rc != DILATTN_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return DILATTN_ERR_INVALID_ARG;
+  if (lse != nullptr && !aligned16(lse)) return DILATTN_ERR_INVALID_ARG;
+  const size_t tb = (size_t)B * N * H * d * 2;
+  if (overlaps(out, tb, q, tb) || overlaps(out, tb, k, tb) || overlaps(out, tb, v, tb))
+    return DILATTN_ERR_INVALID_ARG;
+  if (lse != nullptr) {
+    const size_t lb = (size_t)B * H * N * 4;
+    if (overlaps(lse, lb, q, tb) || overlaps(lse, lb, k, tb) || overlaps(lse, lb, v, tb) ||
+        overlaps(lse, lb, out, tb))
+      return DILATTN_ERR_INVALID_ARG;
+  }
+  if (d != 64 && d != 128) return DILATTN_ERR_UNSUPPORTED;
+  const size_t need = dilattn_fwd_workspace_size(B, N, H, d, w, r, npat);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0 ||
+      workspace_bytes < need)
+    return DILATTN_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  if (d == 64)
+    return launch_fwd<64>(q, k, v, out, lse, B, N, H, w, r, npat, causal, workspace, st, stream);
+  return launch_fwd<128>(q, k, v, out, lse, B, N, H, w, r, npat, causal, workspace, st, stream);
+}
+
+size_t dilattn_bwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
+                                  int npat) {
+  if (check_shape(B, N, H, d, w, r, npat, 1) != DILATTN_OK) return 0;
+  const size_t t = (size_t)B * N * H * d * 4;
+  return 3 * align256(t) + align256((size_t)B * H * N * 4);
+}
+
+int dilattn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                const void* dout, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+                const int* w, const int* r, int npat, int causal, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream) {
+  (void)q; (void)k; (void)v; (void)out; (void)lse; (void)dout; (void)dq; (void)dk; (void)dv;
+  (void)B; (void)N; (void)H; (void)d; (void)w; (void)r; (void)npat; (void)causal;
+  (void)workspace; (void)workspace_bytes; (void)stream;
+  snprintf(g_last_error, sizeof(g_last_error), "bf16 backward not built yet");
+  return DILATTN_ERR_UNSUPPORTED;
+}
+
+int dilattn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B,
+                    int N, int H, int d, const int* w, const int* r, int npat, int causal,
+                    cudaStream_t stream) {
+  int rc = check_shape(B, N, H, d, w, r, npat, causal);
+  if (rc != DILATTN_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return DILATTN_ERR_INVALID_ARG;
+  if (lse != nullptr && !aligned16(lse)) return DILATTN_ERR_INVALID_ARG;
+  const size_t tb = (size_t)B * N * H * d * 4;
+  if (overlaps(out, tb, q, tb) || overlaps(out, tb, k, tb) || overlaps(out, tb, v, tb))
+    return DILATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return DILATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  RowParams p = make_row_params(B, N, H, d, w, r, npat, causal);
+  const long long rows = (long long)B * N * H;
+  const unsigned blocks = (unsigned)((rows + 127) / 128);
+  if (d == 64)
+    fwd_f32_kernel<64><<<blocks, 128, 0, stream>>>(p, q, k, v, out, lse);
+  else
+    fwd_f32_kernel<128><<<blocks, 128, 0, stream>>>(p, q, k, v, out, lse);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "fwd_f32_kernel launch");
+  return DILATTN_OK;
+}
+
+int dilattn_bwd_f32(const float* q, const float* k, const float* v, const float* out,
+                    const float* lse, const float* dout, float* dq, float* dk, float* dv, int B,
+                    int N, int H, int d, const int* w, const int* r, int npat, int causal,
+                    cudaStream_t stream) {
+  int rc = check_shape(B, N, H, d, w, r, npat, causal);
+  if (rc != DILATTN_OK) return rc;
+  const void* ins[6] = {q, k, v, out, lse, dout};
+  for (const void* x : ins)
+    if (!aligned16(x)) return DILATTN_ERR_INVALID_ARG;
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return DILATTN_ERR_INVALID_ARG;
+  const size_t tb = (size_t)B * N * H * d * 4;
+  const size_t lb = (size_t)B * H * N * 4;
+  void* outs[3] = {dq, dk, dv};
+  for (void* o : outs) {
+    for (int j = 0; j < 6; ++j)
+      if (overlaps(o, tb, ins[j], j == 4 ? lb : tb)) return DILATTN_ERR_INVALID_ARG;
+  }
+  if (overlaps(dq, tb, dk, tb) || overlaps(dq, tb, dv, tb) || overlaps(dk, tb, dv, tb))
+    return DILATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return DILATTN_ERR_UNSUPPORTED;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  RowParams p = make_row_params(B, N, H, d, w, r, npat, causal);
+  const long long rows = (long long)B * N * H;
+  const unsigned blocks = (unsigned)((rows + 127) / 128);
+  if (d == 64) {
+    bwd_dq_f32_kernel<64><<<blocks, 128, 0, stream>>>(p, q, k, v, out, lse, dout, dq);
+    bwd_dkdv_f32_kernel<64><<<blocks, 128, 0, stream>>>(p, q, k, v, out, lse, dout, dk, dv);
+  } else {
+    bwd_dq_f32_kernel<128><<<blocks, 128, 0, stream>>>(p, q, k, v, out, lse, dout, dq);
+    bwd_dkdv_f32_kernel<128><<<blocks, 128, 0, stream>>>(p, q, k, v, out, lse, dout, dk, dv);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bwd_f32 launch");
+  return DILATTN_OK;
+}
+
+int dilattn_selection(uint32_t* sig, int N, int H, const int* w, const int* r, int npat,
+                      cudaStream_t stream) {
+  int rc = check_shape(1, N, H, 1, w, r, npat, 1);
+  if (rc != DILATTN_OK) return rc;
+  if (!aligned16(sig)) return DILATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  PatternGeom geo[kMaxPat];
+  make_geoms(1, N, H, w, r, npat, geo);
+  cudaError_t e = cudaMemsetAsync(sig, 0, (size_t)H * N * 4, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  for (int i = 0; i < npat; ++i) {
+    const long long gx = (long long)geo[i].nseg * H;
+    if (gx > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
+    const int gy = std::min(64, (geo[i].nmax + 255) / 256);
+    selection_kernel<<<dim3((unsigned)gx, gy), 256, 0, stream>>>(geo[i], i, N, H, sig);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selection_kernel launch");
+  return DILATTN_OK;
+}
+
+int dilattn_device_error(cudaStream_t stream, int* code) {
+  if (code == nullptr) return DILATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  e = cudaMemcpy(&v, st->err_word, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  const int zero = 0;
+  e = cudaMemcpy(st->err_word, &zero, sizeof(int), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
+  *code = v;
+  return DILATTN_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,375 @@
+// Forward tile kernel: tcgen05 tensor cores, TMA-gathered dilated rows,
+// fp32 online softmax; one CTA per (pattern, segment, batch, head, query tile).
+//
+// Each CTA runs causal softmax attention between 128 kept query rows of one
+// pattern segment and the segment's kept key rows (the dilated, per-head
+// offset rows of the LongNet method description: gptget.net summary of arXiv
+// 2307.02486, "方法详解"). Kept rows are addressed by a 5-D TMA view of the
+// [B][N][H][d] tensor, {d, H, r (phase), N/r, B}, so the stride-r gather
+// happens inside the copy engine with no materialised copy. The CTA writes
+// the pattern's normalised output O_i and its log-sum-exp for those rows to
+// an fp32 partial buffer; the merge kernel combines patterns.
+//
+// Warp roles (192 threads):
+//   warp 0      TMA producer: Q tile once, then a ring of K/V tiles.
+//   warp 1      TMEM allocator and single-thread MMA issuer:
+//               S = Q K^T (SMEM x SMEM -> TMEM), O += P V (TMEM x SMEM -> TMEM).
+//   warps 2..5  softmax: one thread per query row (TMEM lane), fp32 running
+//               max / sum, P = exp2(S*scale - m) stored to TMEM as bf16,
+//               O rescaled in TMEM when the max rises, epilogue.
+// TMEM columns: S [0,128), P [128,192) (bf16 pairs), O [192, 192+D).
+#pragma once
+
+#include "common.cuh"
+
+namespace dil {
+
+struct FwdParams {
+  CUtensorMap tmq[kMaxPat];
+  CUtensorMap tmk[kMaxPat];
+  CUtensorMap tmv[kMaxPat];
+  PatternGeom pat[kMaxPat];
+  int npat, B, N, H, causal;
+  float scale_log2;  // log2(e) / sqrt(d)
+  // Longest-first schedule: units are ordered by query-tile index t
+  // descending; band j covers t in [band_nt[j+1], band_nt[j]) with the first
+  // band_npat[j] patterns of order[] active, band_per_level[j] units per t.
+  int nband;
+  int band_nt[kMaxPat + 1];
+  int band_npat[kMaxPat];
+  int order[kMaxPat];
+  long long band_per_level[kMaxPat];
+  long long band_start[kMaxPat + 1];
+  float* part_o;    // [rows][D]
+  float* part_lse;  // [rows] natural-log lse of each pattern's partial
+  int* err;
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int KCH = D / 64;                 // 128-byte column chunks per row
+  static constexpr int STAGES = 2;                   // K/V ring depth
+  static constexpr int CHUNK_BYTES = BM * 128;       // 128 rows x 64 bf16
+  static constexpr int Q_BYTES = KCH * CHUNK_BYTES;
+  static constexpr int KV_BYTES = KCH * CHUNK_BYTES;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
+  static constexpr int TM_S = 0, TM_P = 128, TM_O = 192;
+  static constexpr int TMEM_COLS = (TM_O + D <= 256) ? 256 : 512;
+  static constexpr int MIN_BLOCKS = (D == 64) ? 2 : 1;
+};
+
+struct FwdUnit {
+  int pat, seg, b, h, t;
+};
+
+__device__ __forceinline__ FwdUnit decode_fwd_unit(const FwdParams& p, long long u) {
+  int j = 0;
+  while (j + 1 < p.nband && u >= p.band_start[j + 1]) ++j;
+  long long u2 = u - p.band_start[j];
+  FwdUnit w;
+  w.t = p.band_nt[j] - 1 - (int)(u2 / p.band_per_level[j]);
+  long long rem = u2 % p.band_per_level[j];
+  w.pat = p.order[0];
+  for (int a = 0; a < p.band_npat[j]; ++a) {
+    int i = p.order[a];
+    long long cnt = (long long)p.pat[i].nseg * p.B * p.H;
+    if (rem < cnt) {
+      w.pat = i;
+      break;
+    }
+    rem -= cnt;
+  }
+  w.h = (int)(rem % p.H);
+  rem /= p.H;
+  w.b = (int)(rem % p.B);
+  w.seg = (int)(rem / p.B);
+  return w;
+}
+
+// Coordinates of kept row v of a segment in the strided TMA view.
+__device__ __forceinline__ void view_coords(const PatternGeom& g, const SegInfo& si, int v,
+                                            int& phase, int& m) {
+  long long pos = si.start + si.off + (long long)v * g.r + g.shift;
+  phase = (int)(pos % g.r);
+  m = (int)(pos / g.r);
+}
+
+// Bounded wait taken by all 32 lanes of a warp, with a warp-uniform result.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          int* err) {
+  const bool ok = mbar_wait(bar, parity, abort, err);
+  return __all_sync(0xffffffffu, ok);
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, FwdCfg<D>::MIN_BLOCKS)
+    fwd_tile_kernel(const __grid_constant__ FwdParams p) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t base = (raw_s + 1023u) & ~1023u;
+  uint8_t* base_g = smem_raw + (base - raw_s);
+
+  const FwdUnit wu = decode_fwd_unit(p, blockIdx.x);
+  const PatternGeom g = p.pat[wu.pat];
+  const SegInfo si = seg_info(g, p.N, wu.h, wu.seg);
+  if (wu.t * BM >= si.n) return;  // tile past the segment's kept rows (uniform exit)
+  const int nkv = p.causal ? (wu.t + 1) : (si.n + BN - 1) / BN;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const uint32_t sQ = base + C::OFF_Q;
+  const uint32_t sK = base + C::OFF_K;
+  const uint32_t sV = base + C::OFF_V;
+  const uint32_t bars = base + C::OFF_BAR;
+  const uint32_t b_qfull = bars;
+  auto b_kfull = [&](int s) { return bars + 8u + 8u * s; };
+  auto b_vfull = [&](int s) { return bars + 8u + 8u * C::STAGES + 8u * s; };
+  auto b_empty = [&](int s) { return bars + 8u + 16u * C::STAGES + 8u * s; };
+  const uint32_t b_sfull = bars + 8u + 24u * C::STAGES;
+  const uint32_t b_sfree = b_sfull + 8u;
+  const uint32_t b_pfull = b_sfull + 16u;
+  const uint32_t b_odone = b_sfull + 24u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_qfull, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(b_kfull(s), 1);
+      mbar_init(b_vfull(s), 1);
+      mbar_init(b_empty(s), 1);
+    }
+    mbar_init(b_sfull, 1);
+    mbar_init(b_sfree, 4);
+    mbar_init(b_pfull, 4);
+    mbar_init(b_odone, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&p.tmq[wu.pat]);
+    prefetch_tmap(&p.tmk[wu.pat]);
+    prefetch_tmap(&p.tmv[wu.pat]);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const CUtensorMap* mq = &p.tmq[wu.pat];
+      const CUtensorMap* mk = &p.tmk[wu.pat];
+      const CUtensorMap* mv = &p.tmv[wu.pat];
+      int ph, m;
+      view_coords(g, si, wu.t * BM, ph, m);
+      mbar_arrive_expect_tx(b_qfull, C::Q_BYTES);
+      for (int c = 0; c < C::KCH; ++c)
+        tma_load_5d(sQ + c * C::CHUNK_BYTES, mq, b_qfull, c * 64, wu.h, ph, m, wu.b);
+      int issued = 0;
+      for (int it = 0; it < nkv; ++it) {
+        const int s = it % C::STAGES;
+        if (!mbar_wait(b_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, p.err)) break;
+        view_coords(g, si, it * BN, ph, m);
+        mbar_arrive_expect_tx(b_kfull(s), C::KV_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_5d(sK + s * C::KV_BYTES + c * C::CHUNK_BYTES, mk, b_kfull(s), c * 64, wu.h, ph,
+                      m, wu.b);
+        mbar_arrive_expect_tx(b_vfull(s), C::KV_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_5d(sV + s * C::KV_BYTES + c * C::CHUNK_BYTES, mv, b_vfull(s), c * 64, wu.h, ph,
+                      m, wu.b);
+        ++issued;
+      }
+      if (*abort_flag) {
+        // Drain copies still in flight before the CTA's shared memory goes away.
+        volatile int no_abort = 0;
+        mbar_wait(b_qfull, 0, &no_abort, nullptr, 200000000ull);
+        for (int it = issued - C::STAGES; it < issued; ++it) {
+          if (it < 0) continue;
+          const int s = it % C::STAGES;
+          const uint32_t par = (it / C::STAGES) & 1;
+          mbar_wait(b_kfull(s), par, &no_abort, nullptr, 200000000ull);
+          mbar_wait(b_vfull(s), par, &no_abort, nullptr, 200000000ull);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16(BM, BN, 0, 0);  // Q (K-major) x K (K-major)
+      constexpr uint32_t kIdO = idesc_bf16(BM, D, 0, 1);   // P (TMEM) x V (MN-major)
+      auto issue_s = [&](int s) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+          const uint64_t a = sw128_desc(sQ + off, 16, 1024);
+          const uint64_t bd = sw128_desc(sK + s * C::KV_BYTES + off, 16, 1024);
+          mma_ss(tmem + C::TM_S, a, bd, kIdS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int s, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bd = sw128_desc(sV + s * C::KV_BYTES + kk * 2048, C::CHUNK_BYTES, 1024);
+          mma_ts(tmem + C::TM_O, tmem + C::TM_P + kk * 8, bd, kIdO, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(b_qfull, 0, abort_flag, p.err) &&
+                mbar_wait(b_kfull(0), 0, abort_flag, p.err);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        mma_commit(b_sfull);
+      }
+      for (int it = 0; ok && it < nkv; ++it) {
+        if (it + 1 < nkv) {
+          const int s1 = (it + 1) % C::STAGES;
+          if (!mbar_wait(b_kfull(s1), ((it + 1) / C::STAGES) & 1, abort_flag, p.err)) break;
+          if (!mbar_wait(b_sfree, it & 1, abort_flag, p.err)) break;
+          tc_fence_after();
+          issue_s(s1);
+          mma_commit(b_sfull);
+        }
+        if (!mbar_wait(b_pfull, it & 1, abort_flag, p.err)) break;
+        const int s = it % C::STAGES;
+        if (!mbar_wait(b_vfull(s), (it / C::STAGES) & 1, abort_flag, p.err)) break;
+        tc_fence_after();
+        issue_pv(s, it > 0);
+        mma_commit(b_empty(s));
+        mma_commit(b_odone);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const int vq = wu.t * BM + row;
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+    const float sc = p.scale_log2;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int it = 0; it < nkv; ++it) {
+      if (!warp_wait(b_sfull, it & 1, abort_flag, p.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float s[BN];
+#pragma unroll
+      for (int c4 = 0; c4 < BN / 32; ++c4) {
+        uint32_t r[32];
+        tmem_ld32_sync(tl + C::TM_S + c4 * 32, r);
+#pragma unroll
+        for (int c = 0; c < 32; ++c) s[c4 * 32 + c] = __uint_as_float(r[c]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_sfree);
+
+      if (p.causal) {
+        if (it == wu.t) {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            if (c > row) s[c] = -INFINITY;
+        }
+      } else if (it == nkv - 1) {
+        const int lim = si.n - it * BN;
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if (c >= lim) s[c] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
+      const float m_new = fmaxf(m_run, mx * sc);
+      const float alpha = ex2(m_run - m_new);
+      uint32_t pk[BN / 2];
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < BN / 2; ++c) {
+        const float p0 = ex2(fmaf(s[2 * c], sc, -m_new));
+        const float p1 = ex2(fmaf(s[2 * c + 1], sc, -m_new));
+        sum += p0 + p1;
+        pk[c] = pack_bf16(p0, p1);
+      }
+      l_run = l_run * alpha + sum;
+      m_run = m_new;
+
+      if (it > 0) {
+        // PV of the previous tile must be complete before O is rescaled and P overwritten.
+        if (!warp_wait(b_odone, (it - 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha < 1.f)) {
+#pragma unroll
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t r[32];
+            tmem_ld32_sync(tl + C::TM_O + c4 * 32, r);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
+            tmem_st32_sync(tl + C::TM_O + c4 * 32, r);
+          }
+        }
+      }
+#pragma unroll
+      for (int c4 = 0; c4 < BN / 64; ++c4) {
+        uint32_t r[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) r[c] = pk[c4 * 32 + c];
+        tmem_st32_sync(tl + C::TM_P + c4 * 32, r);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_pfull);
+    }
+    if (ok && warp_wait(b_odone, (nkv - 1) & 1, abort_flag, p.err)) {
+      tc_fence_after();
+      const bool valid = vq < si.n;
+      const long long prow =
+          g.part_base + ((long long)(wu.b * p.H + wu.h) * g.nseg + wu.seg) * g.nmax + vq;
+      const float inv = 1.f / l_run;
+      float* dst = p.part_o + prow * D;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t r[32];
+        tmem_ld32_sync(tl + C::TM_O + c4 * 32, r);
+        if (valid) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            float4 o4 = make_float4(__uint_as_float(r[c]) * inv, __uint_as_float(r[c + 1]) * inv,
+                                    __uint_as_float(r[c + 2]) * inv,
+                                    __uint_as_float(r[c + 3]) * inv);
+            *reinterpret_cast<float4*>(dst + c4 * 32 + c) = o4;
+          }
+        }
+      }
+      if (valid) p.part_lse[prow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace dil

@@ -1,0 +1,212 @@
+"""Thin ctypes binding of libdilattn (include/dilattn.h).
+
+The ``dilattn_*`` functions mirror the C entry points one to one (integer
+device pointers and sizes). ``fwd`` / ``bwd`` / ``selection`` add only
+argument marshalling for torch tensors: shape checks, output and workspace
+allocation with torch, and the current CUDA stream. Every step of the
+computation runs in the library's CUDA kernels; there is no other code path,
+and a missing or unloadable library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libdilattn.so")
+
+DILATTN_OK = 0
+MAX_PATTERNS = 16
+
+_c = ctypes
+_vp = _c.c_void_p
+_i = _c.c_int
+_sz = _c.c_size_t
+_ip = _c.POINTER(_c.c_int)
+
+# name -> (restype, argtypes); exactly the functions include/dilattn.h declares
+SIGNATURES = {
+    "dilattn_status_string": (_c.c_char_p, [_i]),
+    "dilattn_last_error": (_c.c_char_p, []),
+    "dilattn_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _ip, _ip, _i]),
+    "dilattn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp, _sz, _vp]),
+    "dilattn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _ip, _ip, _i]),
+    "dilattn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i,
+                         _i, _vp, _sz, _vp]),
+    "dilattn_fwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
+    "dilattn_bwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip,
+                             _i, _i, _vp]),
+    "dilattn_selection": (_i, [_vp, _i, _i, _ip, _ip, _i, _vp]),
+    "dilattn_device_error": (_i, [_vp, _ip]),
+}
+
+_lib = None
+
+
+class DilattnError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(msg)
+        self.status = status
+
+
+def load(path: str = LIB_PATH):
+    """Load libdilattn.so (raises if it is missing or lacks a declared symbol)."""
+    global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m sparse_long_sequence_dilated_b200.build`")
+    lib = _c.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path == LIB_PATH:
+        _lib = lib
+    return lib
+
+
+def __getattr__(name):
+    if name in SIGNATURES:
+        return getattr(load(), name)
+    raise AttributeError(name)
+
+
+def status_string(status: int) -> str:
+    return load().dilattn_status_string(status).decode()
+
+
+def last_error() -> str:
+    return load().dilattn_last_error().decode()
+
+
+def _check(rc: int, what: str):
+    if rc != DILATTN_OK:
+        raise DilattnError(rc, f"{what}: {status_string(rc)} {last_error()}".strip())
+
+
+def _patterns(patterns: Sequence[Tuple[int, int]]):
+    n = len(patterns)
+    w = (_c.c_int * max(n, 1))(*[int(p[0]) for p in patterns])
+    r = (_c.c_int * max(n, 1))(*[int(p[1]) for p in patterns])
+    return w, r, n
+
+
+# ---------------------------------------------------------------------------
+# torch-tensor convenience wrappers (marshalling only)
+# ---------------------------------------------------------------------------
+def _torch():
+    import torch
+    return torch
+
+
+def _stream_handle(stream) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return int(s.cuda_stream)
+
+
+def _shape(q):
+    if q.dim() != 4:
+        raise ValueError("expected a [B, N, H, d] tensor")
+    return tuple(int(x) for x in q.shape)
+
+
+def fwd_workspace_size(B, N, H, d, patterns) -> int:
+    w, r, n = _patterns(patterns)
+    return int(load().dilattn_fwd_workspace_size(B, N, H, d, w, r, n))
+
+
+def bwd_workspace_size(B, N, H, d, patterns) -> int:
+    w, r, n = _patterns(patterns)
+    return int(load().dilattn_bwd_workspace_size(B, N, H, d, w, r, n))
+
+
+def fwd(q, k, v, patterns, causal: bool = True, out=None, lse=None, workspace=None,
+        stream=None):
+    """Merged dilated attention. bf16 tensors go to dilattn_fwd, float32 to dilattn_fwd_f32.
+
+    Returns (out [B, N, H, d] in q's dtype, lse [B, H, N] float32).
+    """
+    torch = _torch()
+    B, N, H, d = _shape(q)
+    for t in (k, v):
+        if tuple(t.shape) != (B, N, H, d) or t.dtype != q.dtype:
+            raise ValueError("q, k, v must share shape and dtype")
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    w, r, n = _patterns(patterns)
+    s = _stream_handle(stream)
+    lib = load()
+    if q.dtype == torch.bfloat16:
+        need = int(lib.dilattn_fwd_workspace_size(B, N, H, d, w, r, n))
+        if workspace is None:
+            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+        rc = lib.dilattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), B, N, H, d, w, r, n, int(causal),
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(), s)
+        _check(rc, "dilattn_fwd")
+    elif q.dtype == torch.float32:
+        rc = lib.dilattn_fwd_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr(), B, N, H, d, w, r, n, int(causal), s)
+        _check(rc, "dilattn_fwd_f32")
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    return out, lse
+
+
+def bwd(q, k, v, out, lse, dout, patterns, causal: bool = True, dq=None, dk=None, dv=None,
+        workspace=None, stream=None):
+    """Gradients (dq, dk, dv) of sum(out * dout) for the forward that produced out, lse."""
+    torch = _torch()
+    B, N, H, d = _shape(q)
+    for t in (k, v, out, dout):
+        if tuple(t.shape) != (B, N, H, d) or t.dtype != q.dtype:
+            raise ValueError("q, k, v, out, dout must share shape and dtype")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    w, r, n = _patterns(patterns)
+    s = _stream_handle(stream)
+    lib = load()
+    if q.dtype == torch.bfloat16:
+        need = int(lib.dilattn_bwd_workspace_size(B, N, H, d, w, r, n))
+        if workspace is None:
+            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+        rc = lib.dilattn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                             dv.data_ptr(), B, N, H, d, w, r, n, int(causal),
+                             workspace.data_ptr(), workspace.numel() * workspace.element_size(), s)
+        _check(rc, "dilattn_bwd")
+    elif q.dtype == torch.float32:
+        rc = lib.dilattn_bwd_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                 dv.data_ptr(), B, N, H, d, w, r, n, int(causal), s)
+        _check(rc, "dilattn_bwd_f32")
+    else:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    return dq, dk, dv
+
+
+def selection(N: int, H: int, patterns, device="cuda", stream=None):
+    """uint32-bit selection map [H, N] (returned as int32 tensor bits) from dilattn_selection."""
+    torch = _torch()
+    sig = torch.empty((H, N), dtype=torch.int32, device=device)
+    w, r, n = _patterns(patterns)
+    rc = load().dilattn_selection(sig.data_ptr(), N, H, w, r, n, _stream_handle(stream))
+    _check(rc, "dilattn_selection")
+    return sig
+
+
+def device_error(stream=None) -> int:
+    code = _c.c_int(0)
+    rc = load().dilattn_device_error(_stream_handle(stream), _c.byref(code))
+    _check(rc, "dilattn_device_error")
+    return int(code.value)

@@ -1,0 +1,109 @@
+"""GPU parity of the forward pass against the float64 oracle (same seeded inputs).
+
+Sizes the oracle finishes in seconds cover several tiles and ragged tails in
+full; the full-size workloads are checked on sampled rows the oracle computes
+one by one, with the same launch configuration the benchmark times.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_long_sequence_dilated_b200 import dilattn
+from sparse_long_sequence_dilated_b200.workloads import WORKLOADS, make_inputs
+from tests.gpu_util import check_close, check_lse, to_device, to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_full(B, N, H, d, pats, causal, dtype, seed=0):
+    inp = make_inputs(B, N, H, d, seed, dtype)
+    q, k, v = to_device(inp, dtype=dtype)
+    out, lse = dilattn.fwd(q, k, v, pats, causal)
+    torch.cuda.synchronize()
+    assert dilattn.device_error() == 0
+    want_o, want_l = oracle.fwd(inp["q"], inp["k"], inp["v"], pats, causal)
+    check_close(to_f64(out), want_o, dtype, "out")
+    check_lse(to_f64(lse), want_l, 2e-2 if dtype == "bf16" else 1e-4)
+
+
+def test_tiny_f32_workload():
+    wl = WORKLOADS["tiny_f32"]
+    _run_full(wl.B, wl.N, wl.H, wl.d, wl.patterns, wl.causal, "f32", wl.seed)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("pats", [
+    [(256, 1), (512, 2), (1024, 4)],
+    [(384, 1), (700, 3), (1000, 6), (1100, 12)],     # ragged: w and r do not divide N
+    [(1100, 1)],                                      # one long segment, ragged tail tile
+    [(64, 5), (96, 200), (1100, 7)],                  # r > w: empty segments; tiny tiles
+])
+def test_bf16_small(pats, causal):
+    _run_full(2, 1100, 3, 64, pats, causal, "bf16", seed=1)
+
+
+def test_bf16_d128_small():
+    _run_full(1, 1536, 4, 128, [(256, 1), (512, 2), (1536, 4)], True, "bf16", seed=2)
+
+
+def test_f32_ragged():
+    _run_full(1, 700, 3, 64, [(256, 1), (300, 3), (700, 5)], False, "f32", seed=3)
+
+
+def test_unselected_rows_zero():
+    # (w, r) = (40, 16): only every 16th row of a segment is kept; the rest get O = 0, lse = -inf
+    inp = make_inputs(1, 300, 16, 64, 5, "bf16")
+    q, k, v = to_device(inp)
+    pats = [(40, 16)]
+    out, lse = dilattn.fwd(q, k, v, pats, True)
+    want_o, want_l = oracle.fwd(inp["q"], inp["k"], inp["v"], pats, True)
+    check_close(to_f64(out), want_o, "bf16", "out")
+    check_lse(to_f64(lse), want_l, 2e-2)
+
+
+@pytest.mark.parametrize("name", ["longnet_base_32k", "train_check_2k"])
+def test_workload_full(name):
+    wl = WORKLOADS[name]
+    _run_full(wl.B, wl.N, wl.H, wl.d, wl.patterns, wl.causal, wl.dtype, wl.seed)
+
+
+@pytest.mark.parametrize("N,H,pats", [
+    (32768, 12, WORKLOADS["longnet_base_32k"].patterns),
+    (1100, 3, [(384, 1), (700, 3), (1000, 6), (1100, 12)]),
+    (300, 16, [(40, 16), (7, 3), (300, 1)]),
+])
+def test_selection_bit_exact(N, H, pats):
+    sig = dilattn.selection(N, H, pats).cpu().numpy().view(np.uint32)
+    want = oracle.selection_signature(N, H, pats)
+    assert np.array_equal(sig, want)
+
+
+def _sampled_rows(B, N, H, n_rows, seed):
+    rng = np.random.default_rng(seed)
+    rows = set()
+    for n in (0, 1, N - 1, N - 2, N // 2):
+        for h in (0, H - 1):
+            rows.add((0, h, n))
+    while len(rows) < n_rows:
+        rows.add((int(rng.integers(0, B)), int(rng.integers(0, H)), int(rng.integers(0, N))))
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("name", ["sweep_131072", "sweep_1048576", "wide_128k"])
+def test_workload_sampled(name):
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl.B, wl.N, wl.H, wl.d, wl.seed, wl.dtype)
+    q, k, v = to_device(inp)
+    out, lse = dilattn.fwd(q, k, v, wl.patterns, wl.causal)
+    torch.cuda.synchronize()
+    assert dilattn.device_error() == 0
+    rows = _sampled_rows(wl.B, wl.N, wl.H, 48, 7)
+    want_o, want_l = oracle.fwd_rows(inp["q"], inp["k"], inp["v"], wl.patterns, rows, wl.causal)
+    idx_b = torch.tensor([r[0] for r in rows])
+    idx_h = torch.tensor([r[1] for r in rows])
+    idx_n = torch.tensor([r[2] for r in rows])
+    got_o = to_f64(out.cpu()[idx_b, idx_n, idx_h])
+    got_l = to_f64(lse.cpu()[idx_b, idx_h, idx_n])
+    check_close(got_o, want_o, "bf16", name)
+    check_lse(got_l, want_l, 2e-2, name)

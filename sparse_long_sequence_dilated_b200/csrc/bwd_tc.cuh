@@ -1,0 +1,406 @@
+// Backward kernels: preprocess (D = rowsum(dO * O), zero the fp32
+// accumulators), the tcgen05 key-tile kernel, and the fp32 -> bf16 convert.
+//
+// The merged forward is one softmax over the multiset union of the keys the
+// patterns give a row (LongNet pages: segments, dilation and per-head
+// offsets from the gptget.net summary of arXiv 2307.02486, "方法详解"; the
+// shared-denominator merge from the DarcStar commentary). So with the merged
+// lse L and D = rowsum(dO * O) every (pattern, segment) contributes the
+// ordinary attention-backward terms with P = exp(tau S - L), and the
+// contributions of different patterns simply add up.
+//
+// Key-tile kernel: one CTA per (pattern, segment, batch, head, key tile u),
+// looping over the segment's query tiles t (t >= u when causal). Per pair:
+//   S^T  = K Q^T,  dP^T = V dO^T                     (SMEM x SMEM -> TMEM)
+//   P^T  = exp2(S^T tau log2e - L log2e), dS^T = P^T (dP^T - D)   (threads)
+//   dV  += P^T dO,  dK += dS^T Q                     (TMEM x SMEM -> TMEM)
+//   dQ   = dS K                                      (SMEM x SMEM -> TMEM)
+// dQ is added to an fp32 accumulator with vector atomics after every pair;
+// dK, dV are added once at the end (other patterns reach the same key rows).
+//
+// Warp roles (192 threads): warp 0 TMA producer (+ per-tile L and D rows),
+// warp 1 TMEM allocator and MMA issuer, warps 2..5 one thread per TMEM lane.
+// TMEM columns: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256,320),
+// dK [320,384), dQ [384,448).
+#pragma once
+
+#include "common.cuh"
+
+namespace dil {
+
+struct BwdParams {
+  CUtensorMap tmq[kMaxPat], tmk[kMaxPat], tmv[kMaxPat], tmdo[kMaxPat];
+  CUtensorMap tmq_t[kMaxPat], tmk_t[kMaxPat], tmv_t[kMaxPat], tmdo_t[kMaxPat];
+  PatternGeom pat[kMaxPat];
+  int npat, B, N, H, causal;
+  float scale_log2;  // log2(e) / sqrt(d)
+  float tau;         // 1 / sqrt(d)
+  Sched sched;
+  const float* lse;   // [B][H][N] natural log
+  const float* drow;  // [B][H][N]
+  float* dq_acc;      // [B][N][H][64]
+  float* dk_acc;
+  float* dv_acc;
+  int* err;
+};
+
+struct BwdCfg {
+  static constexpr int D = 64;
+  static constexpr int STAGES = 2;
+  static constexpr int TILE = BM * 128;  // 128 rows x 64 bf16
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;                 // STAGES tiles
+  static constexpr int OFF_DO = OFF_Q + STAGES * TILE;       // STAGES tiles
+  static constexpr int OFF_DS = OFF_DO + STAGES * TILE;      // 2 chunks of [128 kv][64 q]
+  static constexpr int OFF_L = OFF_DS + 2 * TILE;            // STAGES x 128 floats
+  static constexpr int OFF_D = OFF_L + STAGES * BM * 4;      // STAGES x 128 floats
+  static constexpr int OFF_BAR = OFF_D + STAGES * BM * 4;
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
+  static constexpr int TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 320, TM_DQ = 384;
+  static constexpr int TMEM_COLS = 512;
+};
+
+__device__ __forceinline__ void red_add4(float* dst, float a, float b, float c, float d) {
+  atomicAdd(reinterpret_cast<float4*>(dst), make_float4(a, b, c, d));
+}
+
+__global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant__ BwdParams p) {
+  using C = BwdCfg;
+  constexpr int D = C::D;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_s = smem_u32(smem_raw);
+  const uint32_t base = (raw_s + 1023u) & ~1023u;
+  uint8_t* base_g = smem_raw + (base - raw_s);
+
+  const TileUnit wu = decode_unit(p.sched, p.pat, p.B, p.H, blockIdx.x);
+  const PatternGeom g = p.pat[wu.pat];
+  const SegInfo si = seg_info(g, p.N, wu.h, wu.seg);
+  const int nq = (si.n + BM - 1) / BM;
+  const int u = g.ntiles - 1 - wu.t;  // key tile; long (small u) tiles come first
+  if (u >= nq) return;                // uniform exit: no key rows here
+  const int t0 = p.causal ? u : 0;
+  const int npairs = nq - t0;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
+  const uint32_t sQ = base + C::OFF_Q, sDO = base + C::OFF_DO, sDS = base + C::OFF_DS;
+  float* sL = reinterpret_cast<float*>(base_g + C::OFF_L);
+  float* sD = reinterpret_cast<float*>(base_g + C::OFF_D);
+  const uint32_t bars = base + C::OFF_BAR;
+  const uint32_t b_kvfull = bars;
+  auto b_qfull = [&](int s) { return bars + 8u + 8u * s; };
+  auto b_qempty = [&](int s) { return bars + 8u + 8u * C::STAGES + 8u * s; };
+  const uint32_t b_sdp = bars + 8u + 16u * C::STAGES;
+  const uint32_t b_ds = b_sdp + 8u;
+  const uint32_t b_dq = b_sdp + 16u;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
+
+  int phase0, m0;
+  view_coords(g, si, 0, phase0, m0);
+  const bool tail_view = phase0 < g.nmod;
+  const CUtensorMap* mq = tail_view ? &p.tmq_t[wu.pat] : &p.tmq[wu.pat];
+  const CUtensorMap* mk = tail_view ? &p.tmk_t[wu.pat] : &p.tmk[wu.pat];
+  const CUtensorMap* mv = tail_view ? &p.tmv_t[wu.pat] : &p.tmv[wu.pat];
+  const CUtensorMap* mdo = tail_view ? &p.tmdo_t[wu.pat] : &p.tmdo[wu.pat];
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_kvfull, 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(b_qfull(s), 1);
+      mbar_init(b_qempty(s), 1);
+    }
+    mbar_init(b_sdp, 1);
+    mbar_init(b_ds, 4);
+    mbar_init(b_dq, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(mq);
+    prefetch_tmap(mk);
+    prefetch_tmap(mv);
+    prefetch_tmap(mdo);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  const long long lrow0 = ((long long)wu.b * p.H + wu.h) * p.N;  // lse / D row base
+  const float log2e = 1.4426950408889634f;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int ph, m;
+    if (lane == 0) {
+      view_coords(g, si, u * BN, ph, m);
+      mbar_arrive_expect_tx(b_kvfull, 2 * C::TILE);
+      tma_load_5d(sK, mk, b_kvfull, 0, wu.h, ph, m, wu.b);
+      tma_load_5d(sV, mv, b_kvfull, 0, wu.h, ph, m, wu.b);
+    }
+    int issued = 0;
+    for (int it = 0; it < npairs; ++it) {
+      const int s = it % C::STAGES;
+      const int t = t0 + it;
+      if (!warp_wait(b_qempty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, p.err)) break;
+      // merged lse (log2 units) and D for the tile's query rows; rows past the
+      // segment get L = +inf, so their probabilities are exactly zero
+#pragma unroll
+      for (int jj = 0; jj < BM / 32; ++jj) {
+        const int j = lane + 32 * jj;
+        const int vq = t * BM + j;
+        float L = INFINITY, Dv = 0.f;
+        if (vq < si.n) {
+          const long long pos = si.start + si.off + (long long)vq * g.r;
+          L = p.lse[lrow0 + pos] * log2e;
+          Dv = p.drow[lrow0 + pos];
+        }
+        sL[s * BM + j] = L;
+        sD[s * BM + j] = Dv;
+      }
+      __syncwarp();
+      if (lane == 0) {
+        view_coords(g, si, t * BM, ph, m);
+        mbar_arrive_expect_tx(b_qfull(s), 2 * C::TILE);
+        tma_load_5d(sQ + s * C::TILE, mq, b_qfull(s), 0, wu.h, ph, m, wu.b);
+        tma_load_5d(sDO + s * C::TILE, mdo, b_qfull(s), 0, wu.h, ph, m, wu.b);
+      }
+      ++issued;
+    }
+    if (lane == 0 && *abort_flag) {
+      volatile int no_abort = 0;
+      mbar_wait(b_kvfull, 0, &no_abort, nullptr, 200000000ull);
+      for (int it = issued - C::STAGES; it < issued; ++it) {
+        if (it < 0) continue;
+        mbar_wait(b_qfull(it % C::STAGES), (it / C::STAGES) & 1, &no_abort, nullptr, 200000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16(BM, BM, 0, 0);   // K x Q^T, V x dO^T
+      constexpr uint32_t kIdKV = idesc_bf16(BM, D, 0, 1);   // P^T (TMEM) x dO, dS^T (TMEM) x Q
+      constexpr uint32_t kIdQ = idesc_bf16(BM, D, 1, 1);    // dS (MN-major SMEM) x K
+      bool ok = mbar_wait(b_kvfull, 0, abort_flag, p.err);
+      for (int it = 0; ok && it < npairs; ++it) {
+        const int s = it % C::STAGES;
+        if (!mbar_wait(b_qfull(s), (it / C::STAGES) & 1, abort_flag, p.err)) break;
+        // every MMA of the previous pair (readers of TMEM P^T / dS^T) is complete
+        if (it > 0 && !mbar_wait(b_dq, (it - 1) & 1, abort_flag, p.err)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = sw128_desc(sK + kk * 32, 16, 1024);
+          const uint64_t b = sw128_desc(sQ + s * C::TILE + kk * 32, 16, 1024);
+          mma_ss(tmem + C::TM_S, a, b, kIdS, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = sw128_desc(sV + kk * 32, 16, 1024);
+          const uint64_t b = sw128_desc(sDO + s * C::TILE + kk * 32, 16, 1024);
+          mma_ss(tmem + C::TM_DP, a, b, kIdS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(b_sdp);
+        if (!mbar_wait(b_ds, it & 1, abort_flag, p.err)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint64_t bdo = sw128_desc(sDO + s * C::TILE + kk * 2048, C::TILE, 1024);
+          mma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, bdo, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint64_t bq = sw128_desc(sQ + s * C::TILE + kk * 2048, C::TILE, 1024);
+          mma_ts(tmem + C::TM_DK, tmem + C::TM_DP + kk * 8, bq, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t a = sw128_desc(sDS + kk * 2048, C::TILE, 1024);
+          const uint64_t b = sw128_desc(sK + kk * 2048, C::TILE, 1024);
+          mma_ss(tmem + C::TM_DQ, a, b, kIdQ, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(b_qempty(s));
+        mma_commit(b_dq);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ lanes = rows
+    const int q4 = warp & 3;
+    const int c = q4 * 32 + lane;            // key row of S^T / dP^T / dV / dK, query row of dQ
+    const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+    const bool key_valid = u * BN + c < si.n;
+    const float sc = p.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < npairs; ++it) {
+      const int s = it % C::STAGES;
+      const int t = t0 + it;
+      if (!warp_wait(b_qfull(s), (it / C::STAGES) & 1, abort_flag, p.err) ||
+          !warp_wait(b_sdp, it & 1, abort_flag, p.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float* Ls = sL + s * BM;
+      const float* Ds = sD + s * BM;
+      const bool diag = p.causal && t == u;
+#pragma unroll 1
+      for (int c4 = 0; c4 < BM / 32; ++c4) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32_sync(tl + C::TM_S + c4 * 32, sv);
+        tmem_ld32_sync(tl + C::TM_DP + c4 * 32, dv);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pr[2], ds[2];
+#pragma unroll
+          for (int f = 0; f < 2; ++f) {
+            const int j = c4 * 32 + e + f;
+            float pv = ex2(fmaf(__uint_as_float(sv[e + f]), sc, -Ls[j]));
+            if (!key_valid || (diag && j < c)) pv = 0.f;
+            pr[f] = pv;
+            ds[f] = pv * (__uint_as_float(dv[e + f]) - Ds[j]);
+          }
+          pk[e / 2] = pack_bf16(pr[0], pr[1]);
+          dk[e / 2] = pack_bf16(ds[0], ds[1]);
+        }
+        // P^T and dS^T go over the already-read columns of S^T and dP^T
+        tmem_st16_sync(tl + C::TM_S + c4 * 16, pk);
+        tmem_st16_sync(tl + C::TM_DP + c4 * 16, dk);
+        // dS (query-major) into SMEM for dQ = dS K: row c of chunk (j / 64)
+        // holds dS[j][c] for 64 consecutive j, 16-byte pieces XOR-swizzled by c % 8
+        {
+          const int chunk = c4 >> 1;
+          const int piece0 = (c4 & 1) * 4;
+          uint8_t* rowp = base_g + C::OFF_DS + chunk * C::TILE + c * 128;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int piece = (piece0 + k) ^ (c & 7);
+            *reinterpret_cast<uint4*>(rowp + piece * 16) =
+                make_uint4(dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_ds);
+
+      // dQ rows of this query tile: lane c of TMEM is query row t*128 + c
+      if (!warp_wait(b_dq, it & 1, abort_flag, p.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int vq = t * BM + c;
+      const bool q_valid = vq < si.n;
+      float* dst = p.dq_acc;
+      if (q_valid) {
+        const long long pos = si.start + si.off + (long long)vq * g.r;
+        dst += (((long long)wu.b * p.N + pos) * p.H + wu.h) * D;
+      }
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t r[32];
+        tmem_ld32_sync(tl + C::TM_DQ + c4 * 32, r);
+        if (q_valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            red_add4(dst + c4 * 32 + e, __uint_as_float(r[e]) * p.tau,
+                     __uint_as_float(r[e + 1]) * p.tau, __uint_as_float(r[e + 2]) * p.tau,
+                     __uint_as_float(r[e + 3]) * p.tau);
+        }
+      }
+      tc_fence_before();
+    }
+    // dK, dV of the key tile (all pairs are complete after the last dQ wait);
+    // every lane takes the collective TMEM loads, only valid rows store
+    if (ok) {
+      const long long pos = si.start + si.off + (long long)(u * BN + c) * g.r;
+      const long long off = key_valid ? (((long long)wu.b * p.N + pos) * p.H + wu.h) * D : 0;
+#pragma unroll
+      for (int c4 = 0; c4 < D / 32; ++c4) {
+        uint32_t r[32];
+        tmem_ld32_sync(tl + C::TM_DV + c4 * 32, r);
+        if (key_valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            red_add4(p.dv_acc + off + c4 * 32 + e, __uint_as_float(r[e]),
+                     __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
+                     __uint_as_float(r[e + 3]));
+        }
+        tmem_ld32_sync(tl + C::TM_DK + c4 * 32, r);
+        if (key_valid) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            red_add4(p.dk_acc + off + c4 * 32 + e, __uint_as_float(r[e]) * p.tau,
+                     __uint_as_float(r[e + 1]) * p.tau, __uint_as_float(r[e + 2]) * p.tau,
+                     __uint_as_float(r[e + 3]) * p.tau);
+        }
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// D = rowsum(dO * O) per (b, h, n) and zeroed fp32 accumulators; one warp per row.
+struct PrepParams {
+  int B, N, H;
+  const __nv_bfloat16* out;
+  const __nv_bfloat16* dout;
+  float* drow;
+  float* dq_acc;
+  float* dk_acc;
+  float* dv_acc;
+};
+
+__global__ void __launch_bounds__(256) bwd_prep_kernel(PrepParams p) {
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= (long long)p.B * p.N * p.H) return;
+  const __nv_bfloat162 o = reinterpret_cast<const __nv_bfloat162*>(p.out + row * 64)[lane];
+  const __nv_bfloat162 d = reinterpret_cast<const __nv_bfloat162*>(p.dout + row * 64)[lane];
+  float acc = __low2float(o) * __low2float(d) + __high2float(o) * __high2float(d);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  const float2 z = make_float2(0.f, 0.f);
+  reinterpret_cast<float2*>(p.dq_acc + row * 64)[lane] = z;
+  reinterpret_cast<float2*>(p.dk_acc + row * 64)[lane] = z;
+  reinterpret_cast<float2*>(p.dv_acc + row * 64)[lane] = z;
+  if (lane == 0) {
+    const int h = (int)(row % p.H);
+    const long long bn = row / p.H;
+    const int n = (int)(bn % p.N);
+    const int b = (int)(bn / p.N);
+    p.drow[((long long)b * p.H + h) * p.N + n] = acc;
+  }
+}
+
+// fp32 accumulators -> bf16 gradients (round to nearest even).
+__global__ void __launch_bounds__(256) bwd_convert_kernel(long long n4, const float4* dq,
+                                                          const float4* dk, const float4* dv,
+                                                          uint2* gq, uint2* gk, uint2* gv) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (long long)gridDim.x * blockDim.x) {
+    const float4 a = dq[i], b = dk[i], c = dv[i];
+    gq[i] = make_uint2(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w));
+    gk[i] = make_uint2(pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
+    gv[i] = make_uint2(pack_bf16(c.x, c.y), pack_bf16(c.z, c.w));
+  }
+}
+
+}  // namespace dil

@@ -22,7 +22,7 @@ struct PatternGeom {
   int nseg;            // ceil(N / w): number of segments
   int nmax;            // ceil(min(w, N) / r): row capacity of one segment
   int ntiles;          // ceil(nmax / BM)
-  int shift;           // (r - N % r) % r: row shift of the strided TMA view
+  int nmod;            // N mod r: phases below it have one row more in the strided view
   long long part_base; // first row of this pattern in the partial-result buffer
 };
 
@@ -278,6 +278,77 @@ __device__ __forceinline__ void tmem_st32_sync(uint32_t taddr, const uint32_t (&
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
       "tcgen05.wait::st.sync.aligned;"
       :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+      : "memory");
+}
+}  // namespace dil
+
+namespace dil {
+// Longest-first order of tile units (pattern, segment, batch, head, level t):
+// units are ordered by level t descending; band j covers t in
+// [nt[j+1], nt[j]) with the first npat_active[j] patterns of order[]
+// active and per_level[j] units per level.
+struct Sched {
+  int nband;
+  int nt[kMaxPat + 1];
+  int npat_active[kMaxPat];
+  int order[kMaxPat];
+  long long per_level[kMaxPat];
+  long long start[kMaxPat + 1];
+};
+
+struct TileUnit {
+  int pat, seg, b, h, t;
+};
+
+__device__ __forceinline__ TileUnit decode_unit(const Sched& sc, const PatternGeom* pat, int B,
+                                                int H, long long u) {
+  int j = 0;
+  while (j + 1 < sc.nband && u >= sc.start[j + 1]) ++j;
+  const long long u2 = u - sc.start[j];
+  TileUnit w;
+  w.t = sc.nt[j] - 1 - (int)(u2 / sc.per_level[j]);
+  long long rem = u2 % sc.per_level[j];
+  w.pat = sc.order[0];
+  for (int a = 0; a < sc.npat_active[j]; ++a) {
+    const int i = sc.order[a];
+    const long long cnt = (long long)pat[i].nseg * B * H;
+    if (rem < cnt) {
+      w.pat = i;
+      break;
+    }
+    rem -= cnt;
+  }
+  w.h = (int)(rem % H);
+  rem /= H;
+  w.b = (int)(rem % B);
+  w.seg = (int)(rem / B);
+  return w;
+}
+
+// Coordinates of kept row v of a segment in the strided TMA view: the row's
+// position is phase + m * r.
+__device__ __forceinline__ void view_coords(const PatternGeom& g, const SegInfo& si, int v,
+                                            int& phase, int& m) {
+  const long long pos = si.start + si.off + (long long)v * g.r;
+  phase = (int)(pos % g.r);
+  m = (int)(pos / g.r);
+}
+
+// Bounded wait taken by all 32 lanes of a warp, with a warp-uniform result.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
+                                          int* err) {
+  const bool ok = mbar_wait(bar, parity, abort, err);
+  return __all_sync(0xffffffffu, ok);
+}
+}  // namespace dil
+
+namespace dil {
+// tcgen05.st of 16 columns followed by tcgen05.wait::st.
+__device__ __forceinline__ void tmem_st16_sync(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};\n\t"
+      "tcgen05.wait::st.sync.aligned;"
+      :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
       : "memory");
 }
 }  // namespace dil

@@ -15,6 +15,7 @@
 #include "dilattn.h"
 #include "common.cuh"
 #include "fwd_tc.cuh"
+#include "bwd_tc.cuh"
 #include "simt.cuh"
 
 namespace dil {
@@ -64,6 +65,9 @@ int device_state(DeviceState** out) {
       e = cudaFuncSetAttribute(fwd_tile_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                FwdCfg<128>::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      e = cudaFuncSetAttribute(bwd_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               BwdCfg::SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
     }
     st.init = true;
   }
@@ -92,18 +96,25 @@ int get_encoder() {
   return DILATTN_OK;
 }
 
-// Strided view of a [B][N][H][d] bf16 tensor that gathers every r-th row:
-// dims {d, H, r, ceil(N / r), B}, byte strides {2d, 2Hd, 2Hdr, 2HdN}, base
-// shifted back by `shift` rows so that row p sits at phase (p + shift) mod r,
-// index (p + shift) / r. Rows at or past N fall outside the view and read as
-// zeros; rows before 0 are never addressed because every tile starts at a
-// kept row >= 0. Box: 64 columns (128 bytes, 128-byte swizzle) x 128 rows.
-using MapKey = std::tuple<const void*, int, int, int, int, int, int, int>;
+// Strided view of a [B][N][H][d] bf16 tensor that gathers every r-th row,
+// with the tensor's own base address: dims {d, H, P, M, B}, byte strides
+// {2d, 2Hd, 2Hdr, 2HdN}, so element (c, h, ph, m, b) is row ph + m*r of
+// batch b. The main view has P = r phases and M = floor(N/r) rows; the tail
+// view has P = N mod r and M = floor(N/r) + 1. Either way every in-bounds
+// coordinate is a row below N, and rows past it read as zeros. Box: 64
+// columns (128 bytes, 128-byte swizzle) x 128 rows.
+using MapKey = std::tuple<const void*, int, int, int, int, int, int>;
 std::mutex g_map_mu;
 std::map<MapKey, CUtensorMap> g_maps;
 
-int strided_map(const void* ptr, int B, int N, int H, int d, int r, int shift, CUtensorMap* out) {
-  MapKey key{ptr, B, N, H, d, r, shift, 0};
+int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CUtensorMap* out) {
+  const long long nfloor = N / r;
+  const int nmod = N % r;
+  if ((tail && nmod == 0) || (!tail && nfloor == 0)) {
+    memset(out, 0, sizeof(*out));  // a view no tile of this problem can address
+    return DILATTN_OK;
+  }
+  MapKey key{ptr, B, N, H, d, r, tail};
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -115,17 +126,17 @@ int strided_map(const void* ptr, int B, int N, int H, int d, int r, int shift, C
   int rc = get_encoder();
   if (rc != DILATTN_OK) return rc;
   const long long rowb = (long long)H * d * 2;
-  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)r,
-                        (cuuint64_t)(((long long)N + shift) / r), (cuuint64_t)B};
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)(tail ? nmod : r),
+                        (cuuint64_t)(tail ? nfloor + 1 : nfloor), (cuuint64_t)B};
   cuuint64_t strides[4] = {(cuuint64_t)d * 2, (cuuint64_t)rowb, (cuuint64_t)(rowb * r),
                            (cuuint64_t)(rowb * N)};
   cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)BM, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-  void* base = (void*)((const char*)ptr - (long long)shift * rowb);
   CUtensorMap m;
-  CUresult cr = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, base, dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult cr = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) {
     snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)cr);
     return DILATTN_ERR_CUDA;
@@ -173,7 +184,7 @@ long long make_geoms(int B, int N, int H, const int* w, const int* r, int npat,
     const long long span = std::min<long long>(w[i], N);
     g.nmax = (int)((span + r[i] - 1) / r[i]);
     g.ntiles = (g.nmax + BM - 1) / BM;
-    g.shift = (int)((r[i] - N % r[i]) % r[i]);
+    g.nmod = N % r[i];
     g.part_base = rows;
     rows += (long long)B * H * g.nseg * g.nmax;
   }
@@ -182,35 +193,35 @@ long long make_geoms(int B, int N, int H, const int* w, const int* r, int npat,
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Longest-first unit order for the tile kernel (see FwdParams).
-long long make_schedule(FwdParams& p) {
-  std::vector<int> order(p.npat);
-  for (int i = 0; i < p.npat; ++i) order[i] = i;
+// Longest-first unit order for the tile kernels (see Sched).
+long long make_schedule(const PatternGeom* pat, int npat, int B, int H, Sched& sc) {
+  std::vector<int> order(npat);
+  for (int i = 0; i < npat; ++i) order[i] = i;
   std::stable_sort(order.begin(), order.end(),
-                   [&](int a, int b) { return p.pat[a].ntiles > p.pat[b].ntiles; });
+                   [&](int a, int b) { return pat[a].ntiles > pat[b].ntiles; });
   std::vector<int> vals;
   for (int i : order)
-    if (vals.empty() || vals.back() != p.pat[i].ntiles) vals.push_back(p.pat[i].ntiles);
-  for (int i = 0; i < p.npat; ++i) p.order[i] = order[i];
-  p.nband = (int)vals.size();
-  p.band_start[0] = 0;
-  for (int j = 0; j < p.nband; ++j) {
-    const int lo = j + 1 < p.nband ? vals[j + 1] : 0;
-    p.band_nt[j] = vals[j];
+    if (vals.empty() || vals.back() != pat[i].ntiles) vals.push_back(pat[i].ntiles);
+  for (int i = 0; i < npat; ++i) sc.order[i] = order[i];
+  sc.nband = (int)vals.size();
+  sc.start[0] = 0;
+  for (int j = 0; j < sc.nband; ++j) {
+    const int lo = j + 1 < sc.nband ? vals[j + 1] : 0;
+    sc.nt[j] = vals[j];
     int act = 0;
     long long per = 0;
-    for (int a = 0; a < p.npat; ++a) {
-      if (p.pat[order[a]].ntiles >= vals[j]) {
+    for (int a = 0; a < npat; ++a) {
+      if (pat[order[a]].ntiles >= vals[j]) {
         ++act;
-        per += (long long)p.pat[order[a]].nseg * p.B * p.H;
+        per += (long long)pat[order[a]].nseg * B * H;
       }
     }
-    p.band_npat[j] = act;
-    p.band_per_level[j] = per;
-    p.band_start[j + 1] = p.band_start[j] + (long long)(vals[j] - lo) * per;
+    sc.npat_active[j] = act;
+    sc.per_level[j] = per;
+    sc.start[j + 1] = sc.start[j] + (long long)(vals[j] - lo) * per;
   }
-  p.band_nt[p.nband] = 0;
-  return p.band_start[p.nband];
+  sc.nt[sc.nband] = 0;
+  return sc.start[sc.nband];
 }
 
 template <int D>
@@ -231,12 +242,16 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   p.part_lse = reinterpret_cast<float*>((char*)ws + align256((size_t)rows * D * 4));
   p.err = st->err_word;
   for (int i = 0; i < npat; ++i) {
-    int rc = strided_map(q, B, N, H, D, r[i], p.pat[i].shift, &p.tmq[i]);
-    if (rc == DILATTN_OK) rc = strided_map(k, B, N, H, D, r[i], p.pat[i].shift, &p.tmk[i]);
-    if (rc == DILATTN_OK) rc = strided_map(v, B, N, H, D, r[i], p.pat[i].shift, &p.tmv[i]);
-    if (rc != DILATTN_OK) return rc;
+    const void* src[3] = {q, k, v};
+    CUtensorMap* dst[3] = {&p.tmq[i], &p.tmk[i], &p.tmv[i]};
+    CUtensorMap* dst_t[3] = {&p.tmq_t[i], &p.tmk_t[i], &p.tmv_t[i]};
+    for (int j = 0; j < 3; ++j) {
+      int rc = strided_map(src[j], B, N, H, D, r[i], 0, dst[j]);
+      if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j]);
+      if (rc != DILATTN_OK) return rc;
+    }
   }
-  const long long units = make_schedule(p);
+  const long long units = make_schedule(p.pat, npat, B, H, p.sched);
   if (units > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
   fwd_tile_kernel<D><<<(unsigned)units, 192, FwdCfg<D>::SMEM_BYTES, stream>>>(p);
   cudaError_t e = cudaGetLastError();
@@ -258,6 +273,72 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   merge_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(mp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "merge_kernel launch");
+  return DILATTN_OK;
+}
+
+int launch_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
+               const void* dout, void* dq, void* dk, void* dv, int B, int N, int H,
+               const int* w, const int* r, int npat, int causal, void* ws, DeviceState* st,
+               cudaStream_t stream) {
+  constexpr int D = 64;
+  static_assert(sizeof(BwdParams) < 32000, "kernel parameter block too large");
+  BwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.npat = npat;
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  p.causal = causal;
+  p.tau = (float)(1.0 / std::sqrt((double)D));
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  make_geoms(B, N, H, w, r, npat, p.pat);
+  const size_t tbytes = align256((size_t)B * N * H * D * 4);
+  char* wsb = reinterpret_cast<char*>(ws);
+  p.dq_acc = reinterpret_cast<float*>(wsb);
+  p.dk_acc = reinterpret_cast<float*>(wsb + tbytes);
+  p.dv_acc = reinterpret_cast<float*>(wsb + 2 * tbytes);
+  float* drow = reinterpret_cast<float*>(wsb + 3 * tbytes);
+  p.drow = drow;
+  p.lse = lse;
+  p.err = st->err_word;
+  for (int i = 0; i < npat; ++i) {
+    const void* src[4] = {q, k, v, dout};
+    CUtensorMap* dst[4] = {&p.tmq[i], &p.tmk[i], &p.tmv[i], &p.tmdo[i]};
+    CUtensorMap* dst_t[4] = {&p.tmq_t[i], &p.tmk_t[i], &p.tmv_t[i], &p.tmdo_t[i]};
+    for (int j = 0; j < 4; ++j) {
+      int rc = strided_map(src[j], B, N, H, D, r[i], 0, dst[j]);
+      if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j]);
+      if (rc != DILATTN_OK) return rc;
+    }
+  }
+  const long long units = make_schedule(p.pat, npat, B, H, p.sched);
+  if (units > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
+  const long long rows = (long long)B * N * H;
+
+  PrepParams pp;
+  pp.B = B;
+  pp.N = N;
+  pp.H = H;
+  pp.out = reinterpret_cast<const __nv_bfloat16*>(out);
+  pp.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
+  pp.drow = drow;
+  pp.dq_acc = p.dq_acc;
+  pp.dk_acc = p.dk_acc;
+  pp.dv_acc = p.dv_acc;
+  bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(pp);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bwd_prep_kernel launch");
+  bwd_tile_kernel<<<(unsigned)units, 192, BwdCfg::SMEM_BYTES, stream>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bwd_tile_kernel launch");
+  const long long n4 = rows * D / 4;
+  const long long cblocks = std::min<long long>((n4 + 255) / 256, (long long)st->num_sms * 16);
+  bwd_convert_kernel<<<(unsigned)cblocks, 256, 0, stream>>>(
+      n4, reinterpret_cast<const float4*>(p.dq_acc), reinterpret_cast<const float4*>(p.dk_acc),
+      reinterpret_cast<const float4*>(p.dv_acc), reinterpret_cast<uint2*>(dq),
+      reinterpret_cast<uint2*>(dk), reinterpret_cast<uint2*>(dv));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "bwd_convert_kernel launch");
   return DILATTN_OK;
 }
 
@@ -345,11 +426,33 @@ int dilattn_bwd(const void* q, const void* k, const void* v, const void* out, co
                 const void* dout, void* dq, void* dk, void* dv, int B, int N, int H, int d,
                 const int* w, const int* r, int npat, int causal, void* workspace,
                 size_t workspace_bytes, cudaStream_t stream) {
-  (void)q; (void)k; (void)v; (void)out; (void)lse; (void)dout; (void)dq; (void)dk; (void)dv;
-  (void)B; (void)N; (void)H; (void)d; (void)w; (void)r; (void)npat; (void)causal;
-  (void)workspace; (void)workspace_bytes; (void)stream;
-  snprintf(g_last_error, sizeof(g_last_error), "bf16 backward not built yet");
-  return DILATTN_ERR_UNSUPPORTED;
+  int rc = check_shape(B, N, H, d, w, r, npat, causal);
+  if (rc != DILATTN_OK) return rc;
+  const void* ins[6] = {q, k, v, out, lse, dout};
+  for (const void* x : ins)
+    if (!aligned16(x)) return DILATTN_ERR_INVALID_ARG;
+  if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return DILATTN_ERR_INVALID_ARG;
+  const size_t tb = (size_t)B * N * H * d * 2;
+  const size_t lb = (size_t)B * H * N * 4;
+  void* outs[3] = {dq, dk, dv};
+  for (void* o : outs)
+    for (int j = 0; j < 6; ++j)
+      if (overlaps(o, tb, ins[j], j == 4 ? lb : tb)) return DILATTN_ERR_INVALID_ARG;
+  if (overlaps(dq, tb, dk, tb) || overlaps(dq, tb, dv, tb) || overlaps(dk, tb, dv, tb))
+    return DILATTN_ERR_INVALID_ARG;
+  if (d != 64) {
+    snprintf(g_last_error, sizeof(g_last_error), "bf16 backward is built for d = 64");
+    return DILATTN_ERR_UNSUPPORTED;
+  }
+  const size_t need = dilattn_bwd_workspace_size(B, N, H, d, w, r, npat);
+  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0 ||
+      workspace_bytes < need)
+    return DILATTN_ERR_WORKSPACE;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, N, H, w, r, npat, causal, workspace,
+                    st, stream);
 }
 
 int dilattn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B,

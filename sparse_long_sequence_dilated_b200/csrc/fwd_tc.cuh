@@ -6,7 +6,11 @@
 // offset rows of the LongNet method description: gptget.net summary of arXiv
 // 2307.02486, "方法详解"). Kept rows are addressed by a 5-D TMA view of the
 // [B][N][H][d] tensor, {d, H, r (phase), N/r, B}, so the stride-r gather
-// happens inside the copy engine with no materialised copy. The CTA writes
+// happens inside the copy engine with no materialised copy. Each stride r
+// has two views with the tensor's own base address: phases [0, r) over
+// floor(N/r) rows, and phases [0, N mod r) over floor(N/r) + 1 rows; a tile
+// at phase ph uses the second when ph < N mod r, so the view's bounds are
+// exactly the rows below N and rows past N read as zeros. The CTA writes
 // the pattern's normalised output O_i and its log-sum-exp for those rows to
 // an fp32 partial buffer; the merge kernel combines patterns.
 //
@@ -25,21 +29,16 @@
 namespace dil {
 
 struct FwdParams {
-  CUtensorMap tmq[kMaxPat];
+  CUtensorMap tmq[kMaxPat];   // phases [0, r), floor(N/r) rows
   CUtensorMap tmk[kMaxPat];
   CUtensorMap tmv[kMaxPat];
+  CUtensorMap tmq_t[kMaxPat]; // phases [0, N mod r), floor(N/r) + 1 rows
+  CUtensorMap tmk_t[kMaxPat];
+  CUtensorMap tmv_t[kMaxPat];
   PatternGeom pat[kMaxPat];
   int npat, B, N, H, causal;
   float scale_log2;  // log2(e) / sqrt(d)
-  // Longest-first schedule: units are ordered by query-tile index t
-  // descending; band j covers t in [band_nt[j+1], band_nt[j]) with the first
-  // band_npat[j] patterns of order[] active, band_per_level[j] units per t.
-  int nband;
-  int band_nt[kMaxPat + 1];
-  int band_npat[kMaxPat];
-  int order[kMaxPat];
-  long long band_per_level[kMaxPat];
-  long long band_start[kMaxPat + 1];
+  Sched sched;
   float* part_o;    // [rows][D]
   float* part_lse;  // [rows] natural-log lse of each pattern's partial
   int* err;
@@ -62,49 +61,6 @@ struct FwdCfg {
   static constexpr int MIN_BLOCKS = (D == 64) ? 2 : 1;
 };
 
-struct FwdUnit {
-  int pat, seg, b, h, t;
-};
-
-__device__ __forceinline__ FwdUnit decode_fwd_unit(const FwdParams& p, long long u) {
-  int j = 0;
-  while (j + 1 < p.nband && u >= p.band_start[j + 1]) ++j;
-  long long u2 = u - p.band_start[j];
-  FwdUnit w;
-  w.t = p.band_nt[j] - 1 - (int)(u2 / p.band_per_level[j]);
-  long long rem = u2 % p.band_per_level[j];
-  w.pat = p.order[0];
-  for (int a = 0; a < p.band_npat[j]; ++a) {
-    int i = p.order[a];
-    long long cnt = (long long)p.pat[i].nseg * p.B * p.H;
-    if (rem < cnt) {
-      w.pat = i;
-      break;
-    }
-    rem -= cnt;
-  }
-  w.h = (int)(rem % p.H);
-  rem /= p.H;
-  w.b = (int)(rem % p.B);
-  w.seg = (int)(rem / p.B);
-  return w;
-}
-
-// Coordinates of kept row v of a segment in the strided TMA view.
-__device__ __forceinline__ void view_coords(const PatternGeom& g, const SegInfo& si, int v,
-                                            int& phase, int& m) {
-  long long pos = si.start + si.off + (long long)v * g.r + g.shift;
-  phase = (int)(pos % g.r);
-  m = (int)(pos / g.r);
-}
-
-// Bounded wait taken by all 32 lanes of a warp, with a warp-uniform result.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* err) {
-  const bool ok = mbar_wait(bar, parity, abort, err);
-  return __all_sync(0xffffffffu, ok);
-}
-
 template <int D>
 __global__ void __launch_bounds__(192, FwdCfg<D>::MIN_BLOCKS)
     fwd_tile_kernel(const __grid_constant__ FwdParams p) {
@@ -114,7 +70,7 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::MIN_BLOCKS)
   const uint32_t base = (raw_s + 1023u) & ~1023u;
   uint8_t* base_g = smem_raw + (base - raw_s);
 
-  const FwdUnit wu = decode_fwd_unit(p, blockIdx.x);
+  const TileUnit wu = decode_unit(p.sched, p.pat, p.B, p.H, blockIdx.x);
   const PatternGeom g = p.pat[wu.pat];
   const SegInfo si = seg_info(g, p.N, wu.h, wu.seg);
   if (wu.t * BM >= si.n) return;  // tile past the segment's kept rows (uniform exit)
@@ -153,10 +109,17 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::MIN_BLOCKS)
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  // All tiles of a (pattern, segment, head) share one phase, hence one view.
+  int phase0, m0;
+  view_coords(g, si, 0, phase0, m0);
+  const bool tail_view = phase0 < g.nmod;
+  const CUtensorMap* mq = tail_view ? &p.tmq_t[wu.pat] : &p.tmq[wu.pat];
+  const CUtensorMap* mk = tail_view ? &p.tmk_t[wu.pat] : &p.tmk[wu.pat];
+  const CUtensorMap* mv = tail_view ? &p.tmv_t[wu.pat] : &p.tmv[wu.pat];
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&p.tmq[wu.pat]);
-    prefetch_tmap(&p.tmk[wu.pat]);
-    prefetch_tmap(&p.tmv[wu.pat]);
+    prefetch_tmap(mq);
+    prefetch_tmap(mk);
+    prefetch_tmap(mv);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -170,9 +133,6 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::MIN_BLOCKS)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const CUtensorMap* mq = &p.tmq[wu.pat];
-      const CUtensorMap* mk = &p.tmk[wu.pat];
-      const CUtensorMap* mv = &p.tmv[wu.pat];
       int ph, m;
       view_coords(g, si, wu.t * BM, ph, m);
       mbar_arrive_expect_tx(b_qfull, C::Q_BYTES);

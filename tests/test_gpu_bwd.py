@@ -1,0 +1,98 @@
+"""GPU parity of the backward pass against the float64 oracle.
+
+Full comparisons at sizes the oracle finishes in seconds; at full workload
+sizes, sampled dq rows and dk/dv rows computed one by one by the oracle, plus
+two identities that hold at any size: per (batch, head) the dk rows sum to 0
+(every query's dS row sums to 0) and the dv rows sum to the dO rows of the
+selected queries (every query's probabilities sum to 1).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from sparse_long_sequence_dilated_b200 import dilattn
+from sparse_long_sequence_dilated_b200.workloads import WORKLOADS, make_inputs
+from tests.gpu_util import check_close, to_device, to_f64
+
+pytestmark = pytest.mark.gpu
+NAMES = ("q", "k", "v", "dout")
+
+
+def _run_full(B, N, H, d, pats, causal, dtype, seed=0):
+    inp = make_inputs(B, N, H, d, seed, dtype, NAMES)
+    q, k, v, do = to_device(inp, NAMES, dtype)
+    out, lse = dilattn.fwd(q, k, v, pats, causal)
+    dq, dk, dv = dilattn.bwd(q, k, v, out, lse, do, pats, causal)
+    torch.cuda.synchronize()
+    assert dilattn.device_error() == 0
+    # the oracle differentiates its own float64 forward
+    gq, gk, gv = oracle.bwd(inp["q"], inp["k"], inp["v"], inp["dout"], pats, causal)
+    check_close(to_f64(dq), gq, dtype, "dq")
+    check_close(to_f64(dk), gk, dtype, "dk")
+    check_close(to_f64(dv), gv, dtype, "dv")
+
+
+def test_train_check_workload():
+    wl = WORKLOADS["train_check_2k"]
+    _run_full(wl.B, wl.N, wl.H, wl.d, wl.patterns, wl.causal, wl.dtype, wl.seed)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("pats", [
+    [(384, 1), (700, 3), (1000, 6), (1100, 12)],
+    [(64, 5), (96, 200), (1100, 7)],
+    [(1100, 1)],
+])
+def test_bf16_small(pats, causal):
+    _run_full(2, 1100, 3, 64, pats, causal, "bf16", seed=11)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_f32_small(causal):
+    _run_full(1, 600, 3, 64, [(128, 1), (300, 3), (600, 4)], causal, "f32", seed=12)
+
+
+def test_f32_d128():
+    _run_full(1, 300, 2, 128, [(100, 1), (300, 2)], True, "f32", seed=13)
+
+
+def _identities(inp_do, sig, dk, dv):
+    """sum_n dk[b, n, h] = 0 and sum_n dv[b, n, h] = sum of dO over the rows some pattern keeps.
+
+    Each stored element carries at most ~2^-8 relative error (bf16 rounding
+    plus fp32 arithmetic), independent across rows, so the sums may deviate
+    by a few times 2^-8 * sqrt(sum of squares)."""
+    sel = (sig.T[None, :, :, None] != 0)          # [1, N, H, 1]
+    want_v = (inp_do * sel).sum(axis=1)
+    tol_k = 6 * 2.0 ** -8 * np.sqrt((dk ** 2).sum(axis=1)) + 1e-3
+    tol_v = 6 * 2.0 ** -8 * np.sqrt((dv ** 2).sum(axis=1)) + 1e-3
+    err_k = np.abs(dk.sum(axis=1))
+    err_v = np.abs(dv.sum(axis=1) - want_v)
+    assert (err_k <= tol_k).all(), float((err_k / tol_k).max())
+    assert (err_v <= tol_v).all(), float((err_v / tol_v).max())
+
+
+@pytest.mark.parametrize("name", ["longnet_base_32k", "train_b4_32k", "sweep_262144"])
+def test_workload_sampled_and_identities(name):
+    wl = WORKLOADS[name]
+    inp = make_inputs(wl.B, wl.N, wl.H, wl.d, wl.seed, wl.dtype, NAMES)
+    q, k, v, do = to_device(inp, NAMES)
+    out, lse = dilattn.fwd(q, k, v, wl.patterns, wl.causal)
+    dq, dk, dv = dilattn.bwd(q, k, v, out, lse, do, wl.patterns, wl.causal)
+    torch.cuda.synchronize()
+    assert dilattn.device_error() == 0
+    rng = np.random.default_rng(3)
+    qrows = [(int(rng.integers(0, wl.B)), int(rng.integers(0, wl.H)), int(rng.integers(0, wl.N)))
+             for _ in range(24)] + [(0, 0, 0), (0, wl.H - 1, wl.N - 1)]
+    # key rows near the end keep the causal query sets small enough for the row oracle
+    krows = [(0, h, wl.N - 1 - int(x)) for h, x in zip(range(wl.H), rng.integers(0, 300, wl.H))]
+    gq, gk, gv = oracle.bwd_rows(inp["q"], inp["k"], inp["v"], inp["dout"], wl.patterns,
+                                 qrows, krows, wl.causal)
+    dq_c, dk_c, dv_c = dq.cpu(), dk.cpu(), dv.cpu()
+    sel = lambda t, rows: to_f64(t[[r[0] for r in rows], [r[2] for r in rows], [r[1] for r in rows]])
+    check_close(sel(dq_c, qrows), gq, "bf16", name + " dq rows")
+    check_close(sel(dk_c, krows), gk, "bf16", name + " dk rows")
+    check_close(sel(dv_c, krows), gv, "bf16", name + " dv rows")
+    sig = oracle.selection_signature(wl.N, wl.H, wl.patterns)
+    _identities(inp["dout"], sig, to_f64(dk_c), to_f64(dv_c))

@@ -123,6 +123,16 @@ int dilattn_selection(uint32_t* sig, int N, int H, const int* w, const int* r, i
                       cudaStream_t stream);
 
 /*
+ * Tracing hook. When both events are non-NULL, every later dilattn_fwd and
+ * dilattn_bwd call made by the calling host thread records tile_begin on its
+ * stream right before it launches its main tile kernel and tile_end right
+ * after, so the caller can time that one kernel with cudaEventElapsedTime.
+ * Passing NULL, NULL turns tracing off. The events stay owned by the caller
+ * and must outlive the calls that record them.
+ */
+int dilattn_set_trace_events(cudaEvent_t tile_begin, cudaEvent_t tile_end);
+
+/*
  * Reads and clears the library's device-side error word on the current
  * device after synchronising `stream`. *code receives 0 when no kernel
  * reported a failure (a bounded wait that ran out sets a nonzero code).

@@ -14,6 +14,7 @@
 //   S^T  = K Q^T,  dP^T = V dO^T                     (SMEM x SMEM -> TMEM)
 //   P^T  = exp2(S^T tau log2e - L log2e), dS^T = P^T (dP^T - D)   (threads)
 //   dV  += P^T dO,  dK += dS^T Q                     (TMEM x SMEM -> TMEM)
+//          (P^T enters dV as two bf16 halves, hi + lo, for an fp32-grade product)
 //   dQ   = dS K                                      (SMEM x SMEM -> TMEM)
 // dQ is added to an fp32 accumulator with vector atomics after every pair;
 // dK, dV are added once at the end (other patterns reach the same key rows).
@@ -214,7 +215,9 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint64_t bdo = sw128_desc(sDO + s * C::TILE + kk * 2048, C::TILE, 1024);
-          mma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, bdo, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t a_hi = tmem + C::TM_S + (kk >> 2) * 64 + (kk & 3) * 8;
+          mma_ts(tmem + C::TM_DV, a_hi, bdo, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + C::TM_DV, a_hi + 32, bdo, kIdKV, 1u);
         }
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
@@ -252,12 +255,13 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
       const float* Ls = sL + s * BM;
       const float* Ds = sD + s * BM;
       const bool diag = p.causal && t == u;
+      uint32_t plo_prev[16];
 #pragma unroll 1
       for (int c4 = 0; c4 < BM / 32; ++c4) {
         uint32_t sv[32], dv[32];
         tmem_ld32_sync(tl + C::TM_S + c4 * 32, sv);
         tmem_ld32_sync(tl + C::TM_DP + c4 * 32, dv);
-        uint32_t pk[16], dk[16];
+        uint32_t pk[16], plo[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float pr[2], ds[2];
@@ -269,11 +273,27 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
             pr[f] = pv;
             ds[f] = pv * (__uint_as_float(dv[e + f]) - Ds[j]);
           }
-          pk[e / 2] = pack_bf16(pr[0], pr[1]);
+          // P = hi + lo, both bf16: dV takes both halves, so P's own rounding
+          // (2^-9 relative) does not reach dV on top of dV's final bf16 rounding
+          const __nv_bfloat162 hi = __floats2bfloat162_rn(pr[0], pr[1]);
+          const float2 hf = __bfloat1622float2(hi);
+          pk[e / 2] = *reinterpret_cast<const uint32_t*>(&hi);
+          plo[e / 2] = pack_bf16(pr[0] - hf.x, pr[1] - hf.y);
           dk[e / 2] = pack_bf16(ds[0], ds[1]);
         }
-        // P^T and dS^T go over the already-read columns of S^T and dP^T
-        tmem_st16_sync(tl + C::TM_S + c4 * 16, pk);
+        // P^T (hi, lo) and dS^T go over already-read columns of S^T and dP^T.
+        // Query columns [64h, 64h + 64) of P^T: hi at TM_S + 64h + [0, 32),
+        // lo at TM_S + 64h + [32, 64); dS^T is packed densely at TM_DP.
+        const int half = c4 >> 1;
+        if ((c4 & 1) == 0) {
+          tmem_st16_sync(tl + C::TM_S + half * 64, pk);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) plo_prev[e] = plo[e];
+        } else {
+          tmem_st16_sync(tl + C::TM_S + half * 64 + 16, pk);
+          tmem_st16_sync(tl + C::TM_S + half * 64 + 32, plo_prev);
+          tmem_st16_sync(tl + C::TM_S + half * 64 + 48, plo);
+        }
         tmem_st16_sync(tl + C::TM_DP + c4 * 16, dk);
         // dS (query-major) into SMEM for dQ = dS K: row c of chunk (j / 64)
         // holds dS[j][c] for 64 consecutive j, 16-byte pieces XOR-swizzled by c % 8

@@ -26,10 +26,20 @@ namespace {
 
 thread_local char g_last_error[512] = "";
 
+
 int cuda_fail(cudaError_t e, const char* what) {
   snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", what, cudaGetErrorString(e),
            (int)e);
   return DILATTN_ERR_CUDA;
+}
+
+thread_local cudaEvent_t g_trace_begin = nullptr;
+thread_local cudaEvent_t g_trace_end = nullptr;
+
+int trace_mark(cudaEvent_t ev, cudaStream_t stream) {
+  if (ev == nullptr) return DILATTN_OK;
+  cudaError_t e = cudaEventRecord(ev, stream);
+  return e == cudaSuccess ? DILATTN_OK : cuda_fail(e, "cudaEventRecord");
 }
 
 // ------------------------------------------------------------------ device state
@@ -253,9 +263,13 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   }
   const long long units = make_schedule(p.pat, npat, B, H, p.sched);
   if (units > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
+  int rc = trace_mark(g_trace_begin, stream);
+  if (rc != DILATTN_OK) return rc;
   fwd_tile_kernel<D><<<(unsigned)units, 192, FwdCfg<D>::SMEM_BYTES, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd_tile_kernel launch");
+  rc = trace_mark(g_trace_end, stream);
+  if (rc != DILATTN_OK) return rc;
 
   MergeParams mp;
   memset(&mp, 0, sizeof(mp));
@@ -328,9 +342,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(pp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd_prep_kernel launch");
+  int rc = trace_mark(g_trace_begin, stream);
+  if (rc != DILATTN_OK) return rc;
   bwd_tile_kernel<<<(unsigned)units, 192, BwdCfg::SMEM_BYTES, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd_tile_kernel launch");
+  rc = trace_mark(g_trace_end, stream);
+  if (rc != DILATTN_OK) return rc;
   const long long n4 = rows * D / 4;
   const long long cblocks = std::min<long long>((n4 + 255) / 256, (long long)st->num_sms * 16);
   bwd_convert_kernel<<<(unsigned)cblocks, 256, 0, stream>>>(
@@ -540,6 +558,13 @@ int dilattn_selection(uint32_t* sig, int N, int H, const int* w, const int* r, i
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "selection_kernel launch");
+  return DILATTN_OK;
+}
+
+int dilattn_set_trace_events(cudaEvent_t tile_begin, cudaEvent_t tile_end) {
+  if ((tile_begin == nullptr) != (tile_end == nullptr)) return DILATTN_ERR_INVALID_ARG;
+  g_trace_begin = tile_begin;
+  g_trace_end = tile_end;
   return DILATTN_OK;
 }
 

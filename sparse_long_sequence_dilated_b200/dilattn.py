@@ -38,6 +38,7 @@ SIGNATURES = {
     "dilattn_bwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip,
                              _i, _i, _vp]),
     "dilattn_selection": (_i, [_vp, _i, _i, _ip, _ip, _i, _vp]),
+    "dilattn_set_trace_events": (_i, [_vp, _vp]),
     "dilattn_device_error": (_i, [_vp, _ip]),
 }
 
@@ -210,3 +211,12 @@ def device_error(stream=None) -> int:
     rc = load().dilattn_device_error(_stream_handle(stream), _c.byref(code))
     _check(rc, "dilattn_device_error")
     return int(code.value)
+
+
+def set_trace_events(begin=None, end=None):
+    """Record two torch.cuda.Event objects around the next calls' tile kernel (None, None: off).
+
+    The events must already exist on the device (record each once first)."""
+    b = int(begin.cuda_event) if begin is not None else None
+    e = int(end.cuda_event) if end is not None else None
+    _check(load().dilattn_set_trace_events(b, e), "dilattn_set_trace_events")

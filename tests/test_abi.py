@@ -91,3 +91,17 @@ def test_valid_call_without_gpu_reports_cuda_error():
                              None)
     assert rc in (CUDA, UNSUPPORTED)
     assert isinstance(dilattn.last_error(), str)
+
+
+# ---------------------------------------------------------------------------
+# host-side work counts against the oracle's brute-force multiplicity count
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("pats", [[(8, 1), (16, 2), (32, 4)], [(8, 1), (12, 2), (20, 3), (30, 6)],
+                                  [(5, 1), (7, 7), (3, 5)], [(9, 4)]])
+@pytest.mark.parametrize("causal", [True, False])
+def test_effective_pairs_matches_oracle(pats, causal):
+    import oracle
+    from sparse_long_sequence_dilated_b200 import flops
+    assert flops.effective_pairs(2, 30, 5, pats, causal) == oracle.effective_pairs(2, 30, 5, pats, causal)
+    want = sum(int(oracle.multiplicity(30, pats, h, causal).sum()) for h in range(5))
+    assert flops.effective_pairs(1, 30, 5, pats, causal) == want

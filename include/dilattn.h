@@ -87,6 +87,37 @@ int dilattn_fwd(const void* q, const void* k, const void* v, void* out, float* l
                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Forward for callers that cannot allocate device memory: same arguments and
+ * results as dilattn_fwd minus the workspace. Some callers have no way to
+ * get scratch memory: a plugin handed only its input and output pointers by a
+ * host framework, a server that reserves all device memory up front and
+ * forbids later cudaMalloc calls, or code that must not risk the implicit
+ * device synchronisation a cudaMalloc/cudaFree can bring. This entry point
+ * allocates nothing, neither itself nor through any library: the forward's
+ * per-pattern partial results go to a fixed array compiled into the library,
+ * DILATTN_NOALLOC_SCRATCH_BYTES (64 MiB) large, which every device that
+ * loads the library keeps reserved until the process exits. There is no
+ * counterpart in the LongNet pages; it only changes where scratch lives.
+ *
+ * Limits and rules:
+ *   - Problems whose dilattn_fwd_workspace_size(...) exceeds the array are
+ *     rejected with DILATTN_ERR_WORKSPACE (dilattn_last_error() gives the two
+ *     sizes); nothing is launched.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the one array, and it keeps whatever the
+ *     last call left there (this forward writes every scratch entry it later
+ *     reads, so nothing needs to start at zero). Calls that can overlap on the
+ *     GPU -- on different streams, or from different host threads -- race on
+ *     the array; the caller must order them, e.g. on one stream.
+ */
+#define DILATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int B, int N, int H, int d, const int* w, const int* r, int npat,
+                        int causal, cudaStream_t stream);
+
+/*
  * Backward of dilattn_fwd: given out and lse from the forward and the
  * output gradient dout (all device), writes dq, dk, dv [B][N][H][d] bf16, the
  * full derivative of sum(out * dout). The probabilities are recomputed from

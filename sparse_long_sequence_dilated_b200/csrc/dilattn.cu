@@ -586,3 +586,72 @@ int dilattn_device_error(cudaStream_t stream, int* code) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward with a scratch array compiled into the library (no allocation)
+// ---------------------------------------------------------------------------
+namespace dil {
+
+// Scratch of dilattn_fwd_noalloc. In host code this name is only a stand-in
+// for the device array: kernels get the address cudaGetSymbolAddress returns.
+__device__ __align__(256) unsigned char g_noalloc_scratch[DILATTN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+std::map<int, void*> g_noalloc_addr;  // device ordinal -> device address of the scratch
+
+// Device address of the scratch on the current device, looked up once per device.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  auto it = g_noalloc_addr.find(dev);
+  if (it == g_noalloc_addr.end()) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+    it = g_noalloc_addr.emplace(dev, ptr).first;
+  }
+  *out = it->second;
+  return DILATTN_OK;
+}
+}  // namespace
+}  // namespace dil
+
+extern "C" int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                   float* lse, int B, int N, int H, int d, const int* w,
+                                   const int* r, int npat, int causal, cudaStream_t stream) {
+  int rc = check_shape(B, N, H, d, w, r, npat, causal);
+  if (rc != DILATTN_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return DILATTN_ERR_INVALID_ARG;
+  if (lse != nullptr && !aligned16(lse)) return DILATTN_ERR_INVALID_ARG;
+  const size_t tb = (size_t)B * N * H * d * 2;
+  if (overlaps(out, tb, q, tb) || overlaps(out, tb, k, tb) || overlaps(out, tb, v, tb))
+    return DILATTN_ERR_INVALID_ARG;
+  if (lse != nullptr) {
+    const size_t lb = (size_t)B * H * N * 4;
+    if (overlaps(lse, lb, q, tb) || overlaps(lse, lb, k, tb) || overlaps(lse, lb, v, tb) ||
+        overlaps(lse, lb, out, tb))
+      return DILATTN_ERR_INVALID_ARG;
+  }
+  if (d != 64 && d != 128) return DILATTN_ERR_UNSUPPORTED;
+  const size_t need = dilattn_fwd_workspace_size(B, N, H, d, w, r, npat);
+  if (need > (size_t)DILATTN_NOALLOC_SCRATCH_BYTES) {
+    snprintf(g_last_error, sizeof(g_last_error),
+             "dilattn_fwd_noalloc: this problem needs %zu bytes of scratch; the built-in "
+             "scratch holds %zu bytes (use dilattn_fwd with a workspace)",
+             need, (size_t)DILATTN_NOALLOC_SCRATCH_BYTES);
+    return DILATTN_ERR_WORKSPACE;
+  }
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc != DILATTN_OK) return rc;
+  if (d == 64)
+    return launch_fwd<64>(q, k, v, out, lse, B, N, H, w, r, npat, causal, scratch, st, stream);
+  return launch_fwd<128>(q, k, v, out, lse, B, N, H, w, r, npat, causal, scratch, st, stream);
+}

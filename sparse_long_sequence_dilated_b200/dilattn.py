@@ -31,6 +31,7 @@ SIGNATURES = {
     "dilattn_last_error": (_c.c_char_p, []),
     "dilattn_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _ip, _ip, _i]),
     "dilattn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp, _sz, _vp]),
+    "dilattn_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
     "dilattn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _ip, _ip, _i]),
     "dilattn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i,
                          _i, _vp, _sz, _vp]),
@@ -220,3 +221,25 @@ def set_trace_events(begin=None, end=None):
     b = int(begin.cuda_event) if begin is not None else None
     e = int(end.cuda_event) if end is not None else None
     _check(load().dilattn_set_trace_events(b, e), "dilattn_set_trace_events")
+
+
+NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def fwd_noalloc(q, k, v, patterns, causal: bool = True, out=None, lse=None, stream=None):
+    """dilattn_fwd_noalloc on bf16 tensors: the forward with the library's built-in
+    scratch instead of a workspace, for callers that cannot allocate device memory.
+    (This wrapper itself still lets torch allocate ``out``/``lse`` when they are not
+    given; pass them in to allocate nothing.)"""
+    torch = _torch()
+    B, N, H, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    w, r, n = _patterns(patterns)
+    rc = load().dilattn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    lse.data_ptr(), B, N, H, d, w, r, n, int(causal),
+                                    _stream_handle(stream))
+    _check(rc, "dilattn_fwd_noalloc")
+    return out, lse

@@ -42,7 +42,7 @@ METRIC = "dilated-attn fwd/bwd effective TFLOP/s & tokens/s at N=32K–1M; % of 
 UNIT = "TFLOP/s"
 DEFAULT_WORKLOAD = "longnet_base_32k"
 PEAK_FALLBACK = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
-KERNEL_SOURCES = ("common.cuh", "fwd_tc.cuh", "bwd_tc.cuh", "simt.cuh", "dilattn.cu")
+KERNEL_SOURCES = ("common.cuh", "fwd_tc.cuh", "bwd_tc.cuh", "simt.cuh")  # device code only
 NAMES = ("q", "k", "v", "dout")
 
 

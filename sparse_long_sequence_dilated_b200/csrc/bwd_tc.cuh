@@ -16,8 +16,10 @@
 //   dV  += P^T dO,  dK += dS^T Q                     (TMEM x SMEM -> TMEM)
 //          (P^T enters dV as two bf16 halves, hi + lo, for an fp32-grade product)
 //   dQ   = dS K                                      (SMEM x SMEM -> TMEM)
-// dQ is added to an fp32 accumulator with vector atomics after every pair;
-// dK, dV are added once at the end (other patterns reach the same key rows).
+// dQ is staged in shared memory after every pair and added to an fp32
+// accumulator by a TMA reduce-add; dK, dV are added the same way once at the
+// end (other patterns and tiles reach the same rows). The three accumulators
+// form one [3B][N][H][64] fp32 tensor read through the same strided views.
 //
 // Warp roles (192 threads): warp 0 TMA producer (+ per-tile L and D rows),
 // warp 1 TMEM allocator and MMA issuer, warps 2..5 one thread per TMEM lane.
@@ -37,11 +39,9 @@ struct BwdParams {
   float scale_log2;  // log2(e) / sqrt(d)
   float tau;         // 1 / sqrt(d)
   Sched sched;
+  CUtensorMap tmacc[kMaxPat], tmacc_t[kMaxPat];  // fp32 [3B][N][H][64]: dq, dk, dv
   const float* lse;   // [B][H][N] natural log
   const float* drow;  // [B][H][N]
-  float* dq_acc;      // [B][N][H][64]
-  float* dk_acc;
-  float* dv_acc;
   int* err;
 };
 
@@ -54,7 +54,9 @@ struct BwdCfg {
   static constexpr int OFF_Q = OFF_V + TILE;                 // STAGES tiles
   static constexpr int OFF_DO = OFF_Q + STAGES * TILE;       // STAGES tiles
   static constexpr int OFF_DS = OFF_DO + STAGES * TILE;      // 2 chunks of [128 kv][64 q]
-  static constexpr int OFF_L = OFF_DS + 2 * TILE;            // STAGES x 128 floats
+  static constexpr int OFF_STG = OFF_DS + 2 * TILE;          // 2 x fp32 [2][128][32] staging
+  static constexpr int STG_BYTES = 2 * BM * 128;             // one 128 x 64 fp32 tile
+  static constexpr int OFF_L = OFF_STG + 2 * STG_BYTES;      // STAGES x 128 floats
   static constexpr int OFF_D = OFF_L + STAGES * BM * 4;      // STAGES x 128 floats
   static constexpr int OFF_BAR = OFF_D + STAGES * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
@@ -62,8 +64,19 @@ struct BwdCfg {
   static constexpr int TMEM_COLS = 512;
 };
 
-__device__ __forceinline__ void red_add4(float* dst, float a, float b, float c, float d) {
-  atomicAdd(reinterpret_cast<float4*>(dst), make_float4(a, b, c, d));
+// Thread `row` writes 32 fp32 (one 128-byte row of a [128][32] chunk with
+// 128-byte swizzle: 16-byte piece k lands at k ^ (row % 8)), scaled by `scale`.
+__device__ __forceinline__ void stage_row32(uint8_t* chunk, int row, const uint32_t (&r)[32],
+                                            float scale) {
+  uint8_t* rowp = chunk + row * 128;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float4 v = make_float4(__uint_as_float(r[4 * k]) * scale,
+                                 __uint_as_float(r[4 * k + 1]) * scale,
+                                 __uint_as_float(r[4 * k + 2]) * scale,
+                                 __uint_as_float(r[4 * k + 3]) * scale);
+    *reinterpret_cast<float4*>(rowp + ((k ^ (row & 7)) * 16)) = v;
+  }
 }
 
 __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant__ BwdParams p) {
@@ -96,6 +109,9 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
   const uint32_t b_sdp = bars + 8u + 16u * C::STAGES;
   const uint32_t b_ds = b_sdp + 8u;
   const uint32_t b_dq = b_sdp + 16u;
+  const uint32_t b_kv2 = b_sdp + 24u;
+  const uint32_t b_grp = b_sdp + 32u;  // sync point of the four row warps (bounded, unlike bar.sync)
+  const uint32_t sSTG = base + C::OFF_STG;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
 
@@ -106,6 +122,7 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
   const CUtensorMap* mk = tail_view ? &p.tmk_t[wu.pat] : &p.tmk[wu.pat];
   const CUtensorMap* mv = tail_view ? &p.tmv_t[wu.pat] : &p.tmv[wu.pat];
   const CUtensorMap* mdo = tail_view ? &p.tmdo_t[wu.pat] : &p.tmdo[wu.pat];
+  const CUtensorMap* macc = tail_view ? &p.tmacc_t[wu.pat] : &p.tmacc[wu.pat];
 
   if (threadIdx.x == 0) {
     mbar_init(b_kvfull, 1);
@@ -116,6 +133,8 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
     mbar_init(b_sdp, 1);
     mbar_init(b_ds, 4);
     mbar_init(b_dq, 1);
+    mbar_init(b_kv2, 1);
+    mbar_init(b_grp, 4);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -125,6 +144,7 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
     prefetch_tmap(mk);
     prefetch_tmap(mv);
     prefetch_tmap(mdo);
+    prefetch_tmap(macc);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -194,8 +214,9 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
       for (int it = 0; ok && it < npairs; ++it) {
         const int s = it % C::STAGES;
         if (!mbar_wait(b_qfull(s), (it / C::STAGES) & 1, abort_flag, p.err)) break;
-        // every MMA of the previous pair (readers of TMEM P^T / dS^T) is complete
-        if (it > 0 && !mbar_wait(b_dq, (it - 1) & 1, abort_flag, p.err)) break;
+        // the dV / dK MMAs of the previous pair (readers of TMEM P^T / dS^T) are
+        // complete; its dQ MMA (SMEM dS, TMEM dQ) may still run
+        if (it > 0 && !mbar_wait(b_kv2, (it - 1) & 1, abort_flag, p.err)) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -224,6 +245,7 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
           const uint64_t bq = sw128_desc(sQ + s * C::TILE + kk * 2048, C::TILE, 1024);
           mma_ts(tmem + C::TM_DK, tmem + C::TM_DP + kk * 8, bq, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
         }
+        mma_commit(b_kv2);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t a = sw128_desc(sDS + kk * 2048, C::TILE, 1024);
@@ -243,6 +265,15 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
     const bool key_valid = u * BN + c < si.n;
     const float sc = p.scale_log2;
     bool ok = true;
+    uint32_t gphase = 0;
+    // all four row warps meet here; every wait is bounded
+    auto group_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_grp);
+      const bool r = warp_wait(b_grp, gphase & 1, abort_flag, p.err);
+      ++gphase;
+      return r;
+    };
     for (int it = 0; it < npairs; ++it) {
       const int s = it % C::STAGES;
       const int t = t0 + it;
@@ -314,59 +345,76 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
       __syncwarp();
       if (lane == 0) mbar_arrive(b_ds);
 
-      // dQ rows of this query tile: lane c of TMEM is query row t*128 + c
+      // dQ of this query tile (TMEM lane c = query row t*128 + c) -> staging
+      // buffer (it & 1) -> TMA reduce-add into the fp32 dq accumulator. Rows
+      // past the segment hold exact zeros (their P is 0); rows past N are
+      // clipped by the view.
       if (!warp_wait(b_dq, it & 1, abort_flag, p.err)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int vq = t * BM + c;
-      const bool q_valid = vq < si.n;
-      float* dst = p.dq_acc;
-      if (q_valid) {
-        const long long pos = si.start + si.off + (long long)vq * g.r;
-        dst += (((long long)wu.b * p.N + pos) * p.H + wu.h) * D;
+      if (threadIdx.x == 64) bulk_wait_read<1>();  // the reduce that last read this buffer is done
+      if (!group_sync()) {
+        ok = false;
+        break;
       }
+      uint8_t* stg = base_g + C::OFF_STG + (it & 1) * C::STG_BYTES;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t r[32];
         tmem_ld32_sync(tl + C::TM_DQ + c4 * 32, r);
-        if (q_valid) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            red_add4(dst + c4 * 32 + e, __uint_as_float(r[e]) * p.tau,
-                     __uint_as_float(r[e + 1]) * p.tau, __uint_as_float(r[e + 2]) * p.tau,
-                     __uint_as_float(r[e + 3]) * p.tau);
-        }
+        stage_row32(stg + c4 * (C::STG_BYTES / 2), c, r, p.tau);
+      }
+      fence_proxy_async_smem();
+      if (!group_sync()) {
+        ok = false;
+        break;
+      }
+      if (threadIdx.x == 64) {
+        int ph, m;
+        view_coords(g, si, t * BM, ph, m);
+        const uint32_t src = sSTG + (it & 1) * C::STG_BYTES;
+        tma_reduce_add_5d(macc, src, 0, wu.h, ph, m, wu.b);
+        tma_reduce_add_5d(macc, src + C::STG_BYTES / 2, 32, wu.h, ph, m, wu.b);
+        bulk_commit();
       }
       tc_fence_before();
     }
-    // dK, dV of the key tile (all pairs are complete after the last dQ wait);
-    // every lane takes the collective TMEM loads, only valid rows store
+    // dK, dV of the key tile (all pairs are complete after the last dQ wait):
+    // dV -> buffer 0, tau * dK -> buffer 1, TMA reduce-add into the dv and dk
+    // accumulators (batch slots 2B + b and B + b). Rows past the segment are
+    // exact zeros (their P was forced to 0).
     if (ok) {
-      const long long pos = si.start + si.off + (long long)(u * BN + c) * g.r;
-      const long long off = key_valid ? (((long long)wu.b * p.N + pos) * p.H + wu.h) * D : 0;
+      if (threadIdx.x == 64) bulk_wait_read<0>();
+      ok = group_sync();
+    }
+    if (ok) {
+      uint8_t* stg = base_g + C::OFF_STG;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t r[32];
         tmem_ld32_sync(tl + C::TM_DV + c4 * 32, r);
-        if (key_valid) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            red_add4(p.dv_acc + off + c4 * 32 + e, __uint_as_float(r[e]),
-                     __uint_as_float(r[e + 1]), __uint_as_float(r[e + 2]),
-                     __uint_as_float(r[e + 3]));
-        }
+        stage_row32(stg + c4 * (C::STG_BYTES / 2), c, r, 1.f);
         tmem_ld32_sync(tl + C::TM_DK + c4 * 32, r);
-        if (key_valid) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            red_add4(p.dk_acc + off + c4 * 32 + e, __uint_as_float(r[e]) * p.tau,
-                     __uint_as_float(r[e + 1]) * p.tau, __uint_as_float(r[e + 2]) * p.tau,
-                     __uint_as_float(r[e + 3]) * p.tau);
-        }
+        stage_row32(stg + C::STG_BYTES + c4 * (C::STG_BYTES / 2), c, r, p.tau);
+      }
+      fence_proxy_async_smem();
+      ok = group_sync();
+    }
+    if (ok) {
+      if (threadIdx.x == 64) {
+        int ph, m;
+        view_coords(g, si, u * BN, ph, m);
+        tma_reduce_add_5d(macc, sSTG, 0, wu.h, ph, m, 2 * p.B + wu.b);
+        tma_reduce_add_5d(macc, sSTG + C::STG_BYTES / 2, 32, wu.h, ph, m, 2 * p.B + wu.b);
+        tma_reduce_add_5d(macc, sSTG + C::STG_BYTES, 0, wu.h, ph, m, p.B + wu.b);
+        tma_reduce_add_5d(macc, sSTG + C::STG_BYTES + C::STG_BYTES / 2, 32, wu.h, ph, m,
+                          p.B + wu.b);
+        bulk_commit();
       }
     }
+    if (threadIdx.x == 64) bulk_wait_all();  // shared memory stays until the reduces finish
     tc_fence_before();
   }
 

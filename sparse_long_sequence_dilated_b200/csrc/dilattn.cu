@@ -106,25 +106,27 @@ int get_encoder() {
   return DILATTN_OK;
 }
 
-// Strided view of a [B][N][H][d] bf16 tensor that gathers every r-th row,
-// with the tensor's own base address: dims {d, H, P, M, B}, byte strides
-// {2d, 2Hd, 2Hdr, 2HdN}, so element (c, h, ph, m, b) is row ph + m*r of
-// batch b. The main view has P = r phases and M = floor(N/r) rows; the tail
-// view has P = N mod r and M = floor(N/r) + 1. Either way every in-bounds
-// coordinate is a row below N, and rows past it read as zeros. Box: 64
-// columns (128 bytes, 128-byte swizzle) x 128 rows.
-using MapKey = std::tuple<const void*, int, int, int, int, int, int>;
+// Strided view of a [B][N][H][d] tensor (bf16, or fp32 when f32 is set) that
+// gathers every r-th row, with the tensor's own base address: dims
+// {d, H, P, M, B}, byte strides {e d, e H d, e H d r, e H d N} for element
+// size e, so element (c, h, ph, m, b) is row ph + m*r of batch b. The main
+// view has P = r phases and M = floor(N/r) rows; the tail view has
+// P = N mod r and M = floor(N/r) + 1. Either way every in-bounds coordinate is
+// a row below N; loads read zeros and stores/reduces skip rows past it. Box:
+// 128 bytes of columns (128-byte swizzle) x 128 rows.
+using MapKey = std::tuple<const void*, int, int, int, int, int, int, int>;
 std::mutex g_map_mu;
 std::map<MapKey, CUtensorMap> g_maps;
 
-int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CUtensorMap* out) {
+int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CUtensorMap* out,
+                int f32 = 0) {
   const long long nfloor = N / r;
   const int nmod = N % r;
   if ((tail && nmod == 0) || (!tail && nfloor == 0)) {
     memset(out, 0, sizeof(*out));  // a view no tile of this problem can address
     return DILATTN_OK;
   }
-  MapKey key{ptr, B, N, H, d, r, tail};
+  MapKey key{ptr, B, N, H, d, r, tail, f32};
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -135,15 +137,17 @@ int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CU
   }
   int rc = get_encoder();
   if (rc != DILATTN_OK) return rc;
-  const long long rowb = (long long)H * d * 2;
+  const int esz = f32 ? 4 : 2;
+  const long long rowb = (long long)H * d * esz;
   cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)(tail ? nmod : r),
                         (cuuint64_t)(tail ? nfloor + 1 : nfloor), (cuuint64_t)B};
-  cuuint64_t strides[4] = {(cuuint64_t)d * 2, (cuuint64_t)rowb, (cuuint64_t)(rowb * r),
+  cuuint64_t strides[4] = {(cuuint64_t)d * esz, (cuuint64_t)rowb, (cuuint64_t)(rowb * r),
                            (cuuint64_t)(rowb * N)};
-  cuuint32_t box[5] = {64, 1, 1, (cuuint32_t)BM, 1};
+  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, 1, (cuuint32_t)BM, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap m;
-  CUresult cr = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims,
+  CUresult cr = g_encode(&m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                         5, const_cast<void*>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -283,7 +287,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   mp.out = reinterpret_cast<__nv_bfloat16*>(out);
   mp.lse = lse;
   const long long total_rows = (long long)B * N * H;
-  const long long blocks = (total_rows + 7) / 8;
+  const long long blocks = (total_rows + 31) / 32;
   merge_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(mp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "merge_kernel launch");
@@ -306,11 +310,13 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   p.tau = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   make_geoms(B, N, H, w, r, npat, p.pat);
+  // [3B][N][H][64] fp32: dq for batches 0..B-1, then dk, then dv (B*N*H*64*4
+  // is a multiple of 256, so the three align256 blocks are adjacent)
   const size_t tbytes = align256((size_t)B * N * H * D * 4);
   char* wsb = reinterpret_cast<char*>(ws);
-  p.dq_acc = reinterpret_cast<float*>(wsb);
-  p.dk_acc = reinterpret_cast<float*>(wsb + tbytes);
-  p.dv_acc = reinterpret_cast<float*>(wsb + 2 * tbytes);
+  float* dq_acc = reinterpret_cast<float*>(wsb);
+  float* dk_acc = reinterpret_cast<float*>(wsb + tbytes);
+  float* dv_acc = reinterpret_cast<float*>(wsb + 2 * tbytes);
   float* drow = reinterpret_cast<float*>(wsb + 3 * tbytes);
   p.drow = drow;
   p.lse = lse;
@@ -324,6 +330,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
       if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j]);
       if (rc != DILATTN_OK) return rc;
     }
+    int rc = strided_map(dq_acc, 3 * B, N, H, D, r[i], 0, &p.tmacc[i], 1);
+    if (rc == DILATTN_OK) rc = strided_map(dq_acc, 3 * B, N, H, D, r[i], 1, &p.tmacc_t[i], 1);
+    if (rc != DILATTN_OK) return rc;
   }
   const long long units = make_schedule(p.pat, npat, B, H, p.sched);
   if (units > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
@@ -336,9 +345,9 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   pp.out = reinterpret_cast<const __nv_bfloat16*>(out);
   pp.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
   pp.drow = drow;
-  pp.dq_acc = p.dq_acc;
-  pp.dk_acc = p.dk_acc;
-  pp.dv_acc = p.dv_acc;
+  pp.dq_acc = dq_acc;
+  pp.dk_acc = dk_acc;
+  pp.dv_acc = dv_acc;
   bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(pp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd_prep_kernel launch");
@@ -352,8 +361,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   const long long n4 = rows * D / 4;
   const long long cblocks = std::min<long long>((n4 + 255) / 256, (long long)st->num_sms * 16);
   bwd_convert_kernel<<<(unsigned)cblocks, 256, 0, stream>>>(
-      n4, reinterpret_cast<const float4*>(p.dq_acc), reinterpret_cast<const float4*>(p.dk_acc),
-      reinterpret_cast<const float4*>(p.dv_acc), reinterpret_cast<uint2*>(dq),
+      n4, reinterpret_cast<const float4*>(dq_acc), reinterpret_cast<const float4*>(dk_acc),
+      reinterpret_cast<const float4*>(dv_acc), reinterpret_cast<uint2*>(dq),
       reinterpret_cast<uint2*>(dk), reinterpret_cast<uint2*>(dv));
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd_convert_kernel launch");

@@ -38,7 +38,7 @@ __device__ __forceinline__ RowPos row_pos(const PatternGeom& g, int N, int h, in
 
 // ---------------------------------------------------------------------------
 // Merge of per-pattern partials: L = log sum_i exp(lse_i),
-// O = sum_i exp(lse_i - L) O_i, one warp per output row.
+// O = sum_i exp(lse_i - L) O_i.
 // ---------------------------------------------------------------------------
 struct MergeParams {
   PatternGeom pat[kMaxPat];
@@ -49,66 +49,68 @@ struct MergeParams {
   float* lse;  // may be null
 };
 
+// 8 threads per output row, each owning D/8 consecutive columns; 32 rows per
+// 256-thread block. Single pass with a running max, so every partial load is
+// independent of the previous pattern's result.
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ MergeParams p) {
-  constexpr int PER = D / 32;
-  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
+  constexpr int PER = D / 8;  // floats per thread: 8 (d = 64) or 16 (d = 128)
+  const long long row = (long long)blockIdx.x * 32 + (threadIdx.x >> 3);
+  const int sub = threadIdx.x & 7;
   const long long total = (long long)p.B * p.N * p.H;
   if (row >= total) return;
   const int h = (int)(row % p.H);
   const long long bn = row / p.H;
   const int n = (int)(bn % p.N);
   const int b = (int)(bn / p.N);
+  const int bh = b * p.H + h;
 
-  long long prow[kMaxPat];
-  float li[kMaxPat];
-  int cnt = 0;
-  float mx = -INFINITY;
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float m = -INFINITY, l = 0.f;
 #pragma unroll
   for (int i = 0; i < kMaxPat; ++i) {
     if (i >= p.npat) break;
     const PatternGeom& g = p.pat[i];
-    const RowPos rp = row_pos(g, p.N, h, n);
-    if (!rp.kept) continue;
-    const long long pr = g.part_base + ((long long)(b * p.H + h) * g.nseg + rp.seg) * g.nmax + rp.v;
-    prow[cnt] = pr;
-    li[cnt] = p.part_lse[pr];
-    mx = fmaxf(mx, li[cnt]);
-    ++cnt;
-  }
-  float acc[PER];
+    const int seg = n / g.w;
+    const int rel = n - seg * g.w - h % g.r;
+    if (rel < 0 || rel % g.r != 0) continue;
+    const long long pr = g.part_base + ((long long)bh * g.nseg + seg) * g.nmax + rel / g.r;
+    const float li = __ldg(p.part_lse + pr);
+    const float4* src = reinterpret_cast<const float4*>(p.part_o + pr * D + sub * PER);
+    float4 x[PER / 4];
 #pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  float L = -INFINITY;
-  if (cnt > 0) {
-    float tot = 0.f;
-    for (int j = 0; j < cnt; ++j) tot += expf(li[j] - mx);
-    L = mx + logf(tot);
-    for (int j = 0; j < cnt; ++j) {
-      const float a = expf(li[j] - L);
-      const float* src = p.part_o + prow[j] * D + lane * PER;
-      if (PER == 2) {
-        const float2 x = *reinterpret_cast<const float2*>(src);
-        acc[0] += a * x.x;
-        acc[1] += a * x.y;
-      } else {
+    for (int e = 0; e < PER / 4; ++e) x[e] = __ldg(src + e);
+    // running merge of normalised partials: weights exp(li - m) relative to the running max
+    const float m_new = fmaxf(m, li);
+    const float c_old = expf(m - m_new);  // 0 on the first kept pattern
+    const float c_new = expf(li - m_new);
+    l = l * c_old + c_new;
 #pragma unroll
-        for (int e = 0; e < PER; e += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(src + e);
-          acc[e] += a * x.x;
-          acc[e + 1] += a * x.y;
-          acc[e + 2] += a * x.z;
-          acc[e + 3] += a * x.w;
-        }
-      }
+    for (int e = 0; e < PER / 4; ++e) {
+      acc[4 * e] = acc[4 * e] * c_old + c_new * x[e].x;
+      acc[4 * e + 1] = acc[4 * e + 1] * c_old + c_new * x[e].y;
+      acc[4 * e + 2] = acc[4 * e + 2] * c_old + c_new * x[e].z;
+      acc[4 * e + 3] = acc[4 * e + 3] * c_old + c_new * x[e].w;
     }
+    m = m_new;
   }
-  __nv_bfloat16* dst = p.out + row * D + lane * PER;
+  float L = -INFINITY;
+  if (l > 0.f) {
+    const float inv = 1.f / l;
 #pragma unroll
-  for (int e = 0; e < PER; e += 2)
-    *reinterpret_cast<__nv_bfloat162*>(dst + e) = __floats2bfloat162_rn(acc[e], acc[e + 1]);
-  if (p.lse != nullptr && lane == 0) p.lse[((long long)b * p.H + h) * p.N + n] = L;
+    for (int e = 0; e < PER; ++e) acc[e] *= inv;
+    L = m + logf(l);
+  }
+  uint32_t pk[PER / 2];
+#pragma unroll
+  for (int e = 0; e < PER / 2; ++e) pk[e] = pack_bf16(acc[2 * e], acc[2 * e + 1]);
+  uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + sub * PER);
+#pragma unroll
+  for (int e = 0; e < PER / 8; ++e)
+    dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+  if (p.lse != nullptr && sub == 0) p.lse[(long long)bh * p.N + n] = L;
 }
 
 // ---------------------------------------------------------------------------

@@ -21,10 +21,13 @@
 // end (other patterns and tiles reach the same rows). The three accumulators
 // form one [3B][N][H][64] fp32 tensor read through the same strided views.
 //
-// Warp roles (192 threads): warp 0 TMA producer (+ per-tile L and D rows),
-// warp 1 TMEM allocator and MMA issuer, warps 2..5 one thread per TMEM lane.
+// Warp roles (320 threads): warp 0 TMA producer (+ per-tile L and D rows),
+// warp 1 TMEM allocator and MMA issuer, warps 2..9 the row work: warp w
+// serves TMEM lanes 32 (w % 4) .. + 31 and column half (w - 2) / 4, so each
+// scheduler runs two row warps.
 // TMEM columns: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256,320),
-// dK [320,384), dQ [384,448).
+// dK [320,384), dQ [384,448). P^T (hi, lo) and dS^T overwrite S^T and dP^T in
+// place, each 64-column half by the warps that read it.
 #pragma once
 
 #include "common.cuh"
@@ -47,6 +50,9 @@ struct BwdParams {
 
 struct BwdCfg {
   static constexpr int D = 64;
+  static constexpr int NCG = 2;                    // column groups of the row warps
+  static constexpr int ROW_WARPS = 4 * NCG;
+  static constexpr int THREADS = 64 + 32 * ROW_WARPS;
   static constexpr int STAGES = 2;
   static constexpr int TILE = BM * 128;  // 128 rows x 64 bf16
   static constexpr int OFF_K = 0;
@@ -79,7 +85,7 @@ __device__ __forceinline__ void stage_row32(uint8_t* chunk, int row, const uint3
   }
 }
 
-__global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant__ BwdParams p) {
+__global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __grid_constant__ BwdParams p) {
   using C = BwdCfg;
   constexpr int D = C::D;
   extern __shared__ uint8_t smem_raw[];
@@ -110,7 +116,7 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
   const uint32_t b_ds = b_sdp + 8u;
   const uint32_t b_dq = b_sdp + 16u;
   const uint32_t b_kv2 = b_sdp + 24u;
-  const uint32_t b_grp = b_sdp + 32u;  // sync point of the four row warps (bounded, unlike bar.sync)
+  const uint32_t b_grp = b_sdp + 32u;  // sync point of the row warps (bounded, unlike bar.sync)
   const uint32_t sSTG = base + C::OFF_STG;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
@@ -131,10 +137,10 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
       mbar_init(b_qempty(s), 1);
     }
     mbar_init(b_sdp, 1);
-    mbar_init(b_ds, 4);
+    mbar_init(b_ds, C::ROW_WARPS);
     mbar_init(b_dq, 1);
     mbar_init(b_kv2, 1);
-    mbar_init(b_grp, 4);
+    mbar_init(b_grp, C::ROW_WARPS);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -243,7 +249,8 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint64_t bq = sw128_desc(sQ + s * C::TILE + kk * 2048, C::TILE, 1024);
-          mma_ts(tmem + C::TM_DK, tmem + C::TM_DP + kk * 8, bq, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
+          const uint32_t a_ds = tmem + C::TM_DP + (kk >> 2) * 64 + (kk & 3) * 8;
+          mma_ts(tmem + C::TM_DK, a_ds, bq, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(b_kv2);
 #pragma unroll
@@ -260,13 +267,14 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
   } else {
     // ------------------------------------------------------------ lanes = rows
     const int q4 = warp & 3;
+    const int cg = (warp - 2) >> 2;          // column half: S^T / dP^T columns [64 cg, 64 cg + 64)
     const int c = q4 * 32 + lane;            // key row of S^T / dP^T / dV / dK, query row of dQ
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const bool key_valid = u * BN + c < si.n;
     const float sc = p.scale_log2;
     bool ok = true;
     uint32_t gphase = 0;
-    // all four row warps meet here; every wait is bounded
+    // all row warps meet here; every wait is bounded
     auto group_sync = [&]() -> bool {
       __syncwarp();
       if (lane == 0) mbar_arrive(b_grp);
@@ -288,7 +296,7 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
       const bool diag = p.causal && t == u;
       uint32_t plo_prev[16];
 #pragma unroll 1
-      for (int c4 = 0; c4 < BM / 32; ++c4) {
+      for (int c4 = 2 * cg; c4 < 2 * cg + 2; ++c4) {
         uint32_t sv[32], dv[32];
         tmem_ld32_sync(tl + C::TM_S + c4 * 32, sv);
         tmem_ld32_sync(tl + C::TM_DP + c4 * 32, dv);
@@ -312,9 +320,10 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
           plo[e / 2] = pack_bf16(pr[0] - hf.x, pr[1] - hf.y);
           dk[e / 2] = pack_bf16(ds[0], ds[1]);
         }
-        // P^T (hi, lo) and dS^T go over already-read columns of S^T and dP^T.
-        // Query columns [64h, 64h + 64) of P^T: hi at TM_S + 64h + [0, 32),
-        // lo at TM_S + 64h + [32, 64); dS^T is packed densely at TM_DP.
+        // P^T (hi, lo) and dS^T go over already-read columns of S^T and dP^T,
+        // inside the 64-column half this warp reads. Query columns
+        // [64h, 64h + 64): P^T hi at TM_S + 64h + [0, 32), lo at
+        // TM_S + 64h + [32, 64), dS^T at TM_DP + 64h + [0, 32).
         const int half = c4 >> 1;
         if ((c4 & 1) == 0) {
           tmem_st16_sync(tl + C::TM_S + half * 64, pk);
@@ -325,7 +334,7 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
           tmem_st16_sync(tl + C::TM_S + half * 64 + 32, plo_prev);
           tmem_st16_sync(tl + C::TM_S + half * 64 + 48, plo);
         }
-        tmem_st16_sync(tl + C::TM_DP + c4 * 16, dk);
+        tmem_st16_sync(tl + C::TM_DP + half * 64 + (c4 & 1) * 16, dk);
         // dS (query-major) into SMEM for dQ = dS K: row c of chunk (j / 64)
         // holds dS[j][c] for 64 consecutive j, 16-byte pieces XOR-swizzled by c % 8
         {
@@ -360,11 +369,10 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
         break;
       }
       uint8_t* stg = base_g + C::OFF_STG + (it & 1) * C::STG_BYTES;
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        uint32_t r[32];
-        tmem_ld32_sync(tl + C::TM_DQ + c4 * 32, r);
-        stage_row32(stg + c4 * (C::STG_BYTES / 2), c, r, p.tau);
+      {
+        uint32_t r[32];  // dQ columns [32 cg, 32 cg + 32)
+        tmem_ld32_sync(tl + C::TM_DQ + cg * 32, r);
+        stage_row32(stg + cg * (C::STG_BYTES / 2), c, r, p.tau);
       }
       fence_proxy_async_smem();
       if (!group_sync()) {
@@ -391,13 +399,12 @@ __global__ void __launch_bounds__(192, 1) bwd_tile_kernel(const __grid_constant_
     }
     if (ok) {
       uint8_t* stg = base_g + C::OFF_STG;
-#pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        uint32_t r[32];
-        tmem_ld32_sync(tl + C::TM_DV + c4 * 32, r);
-        stage_row32(stg + c4 * (C::STG_BYTES / 2), c, r, 1.f);
-        tmem_ld32_sync(tl + C::TM_DK + c4 * 32, r);
-        stage_row32(stg + C::STG_BYTES + c4 * (C::STG_BYTES / 2), c, r, p.tau);
+      {
+        uint32_t r[32];  // dV, dK columns [32 cg, 32 cg + 32)
+        tmem_ld32_sync(tl + C::TM_DV + cg * 32, r);
+        stage_row32(stg + cg * (C::STG_BYTES / 2), c, r, 1.f);
+        tmem_ld32_sync(tl + C::TM_DK + cg * 32, r);
+        stage_row32(stg + C::STG_BYTES + cg * (C::STG_BYTES / 2), c, r, p.tau);
       }
       fence_proxy_async_smem();
       ok = group_sync();

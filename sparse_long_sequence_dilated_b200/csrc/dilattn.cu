@@ -353,7 +353,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   if (e != cudaSuccess) return cuda_fail(e, "bwd_prep_kernel launch");
   int rc = trace_mark(g_trace_begin, stream);
   if (rc != DILATTN_OK) return rc;
-  bwd_tile_kernel<<<(unsigned)units, 192, BwdCfg::SMEM_BYTES, stream>>>(p);
+  bwd_tile_kernel<<<(unsigned)units, BwdCfg::THREADS, BwdCfg::SMEM_BYTES, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd_tile_kernel launch");
   rc = trace_mark(g_trace_end, stream);

@@ -230,12 +230,11 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::MIN_BLOCKS)
       }
       tc_fence_after();
       float s[BN];
+      {
+        uint32_t raw[BN];
+        tmem_ld128_sync(tl + C::TM_S, raw);
 #pragma unroll
-      for (int c4 = 0; c4 < BN / 32; ++c4) {
-        uint32_t r[32];
-        tmem_ld32_sync(tl + C::TM_S + c4 * 32, r);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) s[c4 * 32 + c] = __uint_as_float(r[c]);
+        for (int c = 0; c < BN; ++c) s[c] = __uint_as_float(raw[c]);
       }
       tc_fence_before();
       __syncwarp();
@@ -253,20 +252,34 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::MIN_BLOCKS)
         for (int c = 0; c < BN; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      float mx = s[0];
+      float mx8[8];
 #pragma unroll
-      for (int c = 1; c < BN; ++c) mx = fmaxf(mx, s[c]);
-      const float m_new = fmaxf(m_run, mx * sc);
-      const float alpha = ex2(m_run - m_new);
+      for (int k = 0; k < 8; ++k) mx8[k] = s[k];
+#pragma unroll
+      for (int c = 8; c < BN; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      // The exponent reference m_run moves only when the tile's max exceeds it
+      // by more than 8 (log2 units); otherwise P <= 2^8 and O is not rescaled.
+      // out = O / l and lse = m_run + log2(l) use the same reference, so the
+      // result is unchanged.
+      const float m_tile = mx * sc;
+      const bool move = m_tile > m_run + 8.f;
+      const float m_new = move ? m_tile : m_run;
+      const float alpha = move ? ex2(m_run - m_new) : 1.f;
       uint32_t pk[BN / 2];
-      float sum = 0.f;
+      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < BN / 2; ++c) {
-        const float p0 = ex2(fmaf(s[2 * c], sc, -m_new));
-        const float p1 = ex2(fmaf(s[2 * c + 1], sc, -m_new));
-        sum += p0 + p1;
+        const float x0 = fmaf(s[2 * c], sc, -m_new);
+        const float x1 = fmaf(s[2 * c + 1], sc, -m_new);
+        // one column in four takes the FMA-pipe exp2, the rest the MUFU ex2
+        const float p0 = ex2(x0);
+        const float p1 = (c & 1) ? ex2_poly(x1) : ex2(x1);
+        sum4[c & 3] += p0 + p1;
         pk[c] = pack_bf16(p0, p1);
       }
+      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
       l_run = l_run * alpha + sum;
       m_run = m_new;
 
@@ -277,7 +290,7 @@ __global__ void __launch_bounds__(192, FwdCfg<D>::MIN_BLOCKS)
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha < 1.f)) {
+        if (__any_sync(0xffffffffu, move)) {
 #pragma unroll
           for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t r[32];

@@ -21,13 +21,15 @@
 // end (other patterns and tiles reach the same rows). The three accumulators
 // form one [3B][N][H][64] fp32 tensor read through the same strided views.
 //
-// Warp roles (320 threads): warp 0 TMA producer (+ per-tile L and D rows),
-// warp 1 TMEM allocator and MMA issuer, warps 2..9 the row work: warp w
-// serves TMEM lanes 32 (w % 4) .. + 31 and column half (w - 2) / 4, so each
-// scheduler runs two row warps.
+// Warp roles (576 threads): warp 0 TMA producer (+ per-tile L and D rows),
+// warp 1 TMEM allocator and MMA issuer, warps 2..17 the row work: warp w
+// serves TMEM lanes 32 (w % 4) .. + 31 and column quarter (w - 2) / 4, so each
+// scheduler runs four row warps.
 // TMEM columns: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256,320),
 // dK [320,384), dQ [384,448). P^T (hi, lo) and dS^T overwrite S^T and dP^T in
-// place, each 64-column half by the warps that read it.
+// place, each 32-column quarter by the warps that read it: query columns
+// [32q, 32q + 32) keep P^T hi at TM_S + 32q + [0, 16), lo at TM_S + 32q + [16, 32)
+// and dS^T at TM_DP + 32q + [0, 16).
 #pragma once
 
 #include "common.cuh"
@@ -50,7 +52,7 @@ struct BwdParams {
 
 struct BwdCfg {
   static constexpr int D = 64;
-  static constexpr int NCG = 2;                    // column groups of the row warps
+  static constexpr int NCG = 4;                    // column quarters of the row warps
   static constexpr int ROW_WARPS = 4 * NCG;
   static constexpr int THREADS = 64 + 32 * ROW_WARPS;
   static constexpr int STAGES = 2;
@@ -70,18 +72,19 @@ struct BwdCfg {
   static constexpr int TMEM_COLS = 512;
 };
 
-// Thread `row` writes 32 fp32 (one 128-byte row of a [128][32] chunk with
-// 128-byte swizzle: 16-byte piece k lands at k ^ (row % 8)), scaled by `scale`.
-__device__ __forceinline__ void stage_row32(uint8_t* chunk, int row, const uint32_t (&r)[32],
-                                            float scale) {
+// Thread `row` writes 16 fp32 = 16-byte pieces [piece0, piece0 + 4) of one
+// 128-byte row of a [128][32] fp32 chunk with 128-byte swizzle (piece k lands
+// at k ^ (row % 8)), scaled by `scale`.
+__device__ __forceinline__ void stage_row16(uint8_t* chunk, int row, int piece0,
+                                            const uint32_t (&r)[16], float scale) {
   uint8_t* rowp = chunk + row * 128;
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
+  for (int k = 0; k < 4; ++k) {
     const float4 v = make_float4(__uint_as_float(r[4 * k]) * scale,
                                  __uint_as_float(r[4 * k + 1]) * scale,
                                  __uint_as_float(r[4 * k + 2]) * scale,
                                  __uint_as_float(r[4 * k + 3]) * scale);
-    *reinterpret_cast<float4*>(rowp + ((k ^ (row & 7)) * 16)) = v;
+    *reinterpret_cast<float4*>(rowp + (((piece0 + k) ^ (row & 7)) * 16)) = v;
   }
 }
 
@@ -242,14 +245,14 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint64_t bdo = sw128_desc(sDO + s * C::TILE + kk * 2048, C::TILE, 1024);
-          const uint32_t a_hi = tmem + C::TM_S + (kk >> 2) * 64 + (kk & 3) * 8;
+          const uint32_t a_hi = tmem + C::TM_S + (kk >> 1) * 32 + (kk & 1) * 8;
           mma_ts(tmem + C::TM_DV, a_hi, bdo, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tmem + C::TM_DV, a_hi + 32, bdo, kIdKV, 1u);
+          mma_ts(tmem + C::TM_DV, a_hi + 16, bdo, kIdKV, 1u);
         }
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint64_t bq = sw128_desc(sQ + s * C::TILE + kk * 2048, C::TILE, 1024);
-          const uint32_t a_ds = tmem + C::TM_DP + (kk >> 2) * 64 + (kk & 3) * 8;
+          const uint32_t a_ds = tmem + C::TM_DP + (kk >> 1) * 32 + (kk & 1) * 8;
           mma_ts(tmem + C::TM_DK, a_ds, bq, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
         }
         mma_commit(b_kv2);
@@ -267,7 +270,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   } else {
     // ------------------------------------------------------------ lanes = rows
     const int q4 = warp & 3;
-    const int cg = (warp - 2) >> 2;          // column half: S^T / dP^T columns [64 cg, 64 cg + 64)
+    const int cg = (warp - 2) >> 2;          // column quarter: S^T / dP^T columns [32 cg, 32 cg + 32)
     const int c = q4 * 32 + lane;            // key row of S^T / dP^T / dV / dK, query row of dQ
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const bool key_valid = u * BN + c < si.n;
@@ -291,26 +294,23 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         break;
       }
       tc_fence_after();
-      const float* Ls = sL + s * BM;
-      const float* Ds = sD + s * BM;
+      const float* Ls = sL + s * BM + cg * 32;
+      const float* Ds = sD + s * BM + cg * 32;
       const bool diag = p.causal && t == u;
-      uint32_t plo_prev[16];
-#pragma unroll 1
-      for (int c4 = 2 * cg; c4 < 2 * cg + 2; ++c4) {
+      {
         uint32_t sv[32], dv[32];
-        tmem_ld32_sync(tl + C::TM_S + c4 * 32, sv);
-        tmem_ld32_sync(tl + C::TM_DP + c4 * 32, dv);
+        tmem_ld32x2_sync(tl + C::TM_S + cg * 32, tl + C::TM_DP + cg * 32, sv, dv);
         uint32_t pk[16], plo[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float pr[2], ds[2];
 #pragma unroll
           for (int f = 0; f < 2; ++f) {
-            const int j = c4 * 32 + e + f;
-            float pv = ex2(fmaf(__uint_as_float(sv[e + f]), sc, -Ls[j]));
+            const int j = cg * 32 + e + f;
+            float pv = ex2(fmaf(__uint_as_float(sv[e + f]), sc, -Ls[e + f]));
             if (!key_valid || (diag && j < c)) pv = 0.f;
             pr[f] = pv;
-            ds[f] = pv * (__uint_as_float(dv[e + f]) - Ds[j]);
+            ds[f] = pv * (__uint_as_float(dv[e + f]) - Ds[e + f]);
           }
           // P = hi + lo, both bf16: dV takes both halves, so P's own rounding
           // (2^-9 relative) does not reach dV on top of dV's final bf16 rounding
@@ -320,26 +320,15 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           plo[e / 2] = pack_bf16(pr[0] - hf.x, pr[1] - hf.y);
           dk[e / 2] = pack_bf16(ds[0], ds[1]);
         }
-        // P^T (hi, lo) and dS^T go over already-read columns of S^T and dP^T,
-        // inside the 64-column half this warp reads. Query columns
-        // [64h, 64h + 64): P^T hi at TM_S + 64h + [0, 32), lo at
-        // TM_S + 64h + [32, 64), dS^T at TM_DP + 64h + [0, 32).
-        const int half = c4 >> 1;
-        if ((c4 & 1) == 0) {
-          tmem_st16_sync(tl + C::TM_S + half * 64, pk);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) plo_prev[e] = plo[e];
-        } else {
-          tmem_st16_sync(tl + C::TM_S + half * 64 + 16, pk);
-          tmem_st16_sync(tl + C::TM_S + half * 64 + 32, plo_prev);
-          tmem_st16_sync(tl + C::TM_S + half * 64 + 48, plo);
-        }
-        tmem_st16_sync(tl + C::TM_DP + half * 64 + (c4 & 1) * 16, dk);
+        // in place over this quarter's own (already read) columns
+        tmem_st16(tl + C::TM_S + cg * 32, pk);
+        tmem_st16(tl + C::TM_S + cg * 32 + 16, plo);
+        tmem_st16(tl + C::TM_DP + cg * 32, dk);
         // dS (query-major) into SMEM for dQ = dS K: row c of chunk (j / 64)
         // holds dS[j][c] for 64 consecutive j, 16-byte pieces XOR-swizzled by c % 8
         {
-          const int chunk = c4 >> 1;
-          const int piece0 = (c4 & 1) * 4;
+          const int chunk = cg >> 1;
+          const int piece0 = (cg & 1) * 4;
           uint8_t* rowp = base_g + C::OFF_DS + chunk * C::TILE + c * 128;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -348,6 +337,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
                 make_uint4(dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
           }
         }
+        tmem_wait_st();
       }
       fence_proxy_async_smem();
       tc_fence_before();
@@ -370,9 +360,9 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       }
       uint8_t* stg = base_g + C::OFF_STG + (it & 1) * C::STG_BYTES;
       {
-        uint32_t r[32];  // dQ columns [32 cg, 32 cg + 32)
-        tmem_ld32_sync(tl + C::TM_DQ + cg * 32, r);
-        stage_row32(stg + cg * (C::STG_BYTES / 2), c, r, p.tau);
+        uint32_t r[16];  // dQ columns [16 cg, 16 cg + 16)
+        tmem_ld16_sync(tl + C::TM_DQ + cg * 16, r);
+        stage_row16(stg + (cg >> 1) * (C::STG_BYTES / 2), c, (cg & 1) * 4, r, p.tau);
       }
       fence_proxy_async_smem();
       if (!group_sync()) {
@@ -400,11 +390,11 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
     if (ok) {
       uint8_t* stg = base_g + C::OFF_STG;
       {
-        uint32_t r[32];  // dV, dK columns [32 cg, 32 cg + 32)
-        tmem_ld32_sync(tl + C::TM_DV + cg * 32, r);
-        stage_row32(stg + cg * (C::STG_BYTES / 2), c, r, 1.f);
-        tmem_ld32_sync(tl + C::TM_DK + cg * 32, r);
-        stage_row32(stg + C::STG_BYTES + cg * (C::STG_BYTES / 2), c, r, p.tau);
+        uint32_t r[16];  // dV, dK columns [16 cg, 16 cg + 16)
+        tmem_ld16_sync(tl + C::TM_DV + cg * 16, r);
+        stage_row16(stg + (cg >> 1) * (C::STG_BYTES / 2), c, (cg & 1) * 4, r, 1.f);
+        tmem_ld16_sync(tl + C::TM_DK + cg * 16, r);
+        stage_row16(stg + C::STG_BYTES + (cg >> 1) * (C::STG_BYTES / 2), c, (cg & 1) * 4, r, p.tau);
       }
       fence_proxy_async_smem();
       ok = group_sync();

@@ -21,10 +21,10 @@
 // end (other patterns and tiles reach the same rows). The three accumulators
 // form one [3B][N][H][64] fp32 tensor read through the same strided views.
 //
-// Warp roles (576 threads): warp 0 TMA producer (+ per-tile L and D rows),
-// warp 1 TMEM allocator and MMA issuer, warps 2..17 the row work: warp w
-// serves TMEM lanes 32 (w % 4) .. + 31 and column quarter (w - 2) / 4, so each
-// scheduler runs four row warps.
+// Warp roles (64 + 128 NCG threads): warp 0 TMA producer (+ per-tile L and D
+// rows), warp 1 TMEM allocator and MMA issuer, warps 2.. the row work: warp w
+// serves TMEM lanes 32 (w % 4) .. + 31 and column group (w - 2) / 4, i.e. the
+// CPT = 4 / NCG consecutive 32-column chunks of that group.
 // TMEM columns: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256,320),
 // dK [320,384), dQ [384,448). P^T (hi, lo) and dS^T overwrite S^T and dP^T in
 // place, each 32-column quarter by the warps that read it: query columns
@@ -52,7 +52,8 @@ struct BwdParams {
 
 struct BwdCfg {
   static constexpr int D = 64;
-  static constexpr int NCG = 4;                    // column quarters of the row warps
+  static constexpr int NCG = 2;                    // column groups of the row warps
+  static constexpr int CPT = 4 / NCG;              // 32-column chunks per row thread
   static constexpr int ROW_WARPS = 4 * NCG;
   static constexpr int THREADS = 64 + 32 * ROW_WARPS;
   static constexpr int STAGES = 2;
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   } else {
     // ------------------------------------------------------------ lanes = rows
     const int q4 = warp & 3;
-    const int cg = (warp - 2) >> 2;          // column quarter: S^T / dP^T columns [32 cg, 32 cg + 32)
+    const int cg = (warp - 2) >> 2;          // column group: chunks [CPT cg, CPT cg + CPT)
     const int c = q4 * 32 + lane;            // key row of S^T / dP^T / dV / dK, query row of dQ
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const bool key_valid = u * BN + c < si.n;
@@ -294,41 +295,53 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         break;
       }
       tc_fence_after();
-      const float* Ls = sL + s * BM + cg * 32;
-      const float* Ds = sD + s * BM + cg * 32;
       const bool diag = p.causal && t == u;
-      {
-        uint32_t sv[32], dv[32];
-        tmem_ld32x2_sync(tl + C::TM_S + cg * 32, tl + C::TM_DP + cg * 32, sv, dv);
+#pragma unroll 1
+      for (int q = cg * C::CPT; q < cg * C::CPT + C::CPT; ++q) {
+        const float4* L4 = reinterpret_cast<const float4*>(sL + s * BM + q * 32);
+        const float4* D4 = reinterpret_cast<const float4*>(sD + s * BM + q * 32);
         uint32_t pk[16], plo[16], dk[16];
+        {
+          uint32_t sv[32], dv[32];
+          tmem_ld32x2_sync(tl + C::TM_S + q * 32, tl + C::TM_DP + q * 32, sv, dv);
+          // key rows past the segment, and (on the diagonal) queries before the
+          // key, get P = 0; elsewhere no mask is needed
+          const int jmin = !key_valid ? 1 << 30 : (diag ? c - q * 32 : 0);
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pr[2], ds[2];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 Lq = L4[e4], Dq = D4[e4];
+            const float lv[4] = {Lq.x, Lq.y, Lq.z, Lq.w};
+            const float dd[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
+            float pr[4], ds[4];
 #pragma unroll
-          for (int f = 0; f < 2; ++f) {
-            const int j = cg * 32 + e + f;
-            float pv = ex2(fmaf(__uint_as_float(sv[e + f]), sc, -Ls[e + f]));
-            if (!key_valid || (diag && j < c)) pv = 0.f;
-            pr[f] = pv;
-            ds[f] = pv * (__uint_as_float(dv[e + f]) - Ds[e + f]);
+            for (int f = 0; f < 4; ++f) {
+              const int e = 4 * e4 + f;
+              float pv = ex2(fmaf(__uint_as_float(sv[e]), sc, -lv[f]));
+              pv = e >= jmin ? pv : 0.f;
+              pr[f] = pv;
+              ds[f] = pv * (__uint_as_float(dv[e]) - dd[f]);
+            }
+#pragma unroll
+            for (int f = 0; f < 4; f += 2) {
+              // P = hi + lo, both bf16: dV takes both halves, so P's own rounding
+              // (2^-9 relative) does not reach dV on top of dV's final bf16 rounding
+              const __nv_bfloat162 hi = __floats2bfloat162_rn(pr[f], pr[f + 1]);
+              const float2 hf = __bfloat1622float2(hi);
+              pk[2 * e4 + f / 2] = *reinterpret_cast<const uint32_t*>(&hi);
+              plo[2 * e4 + f / 2] = pack_bf16(pr[f] - hf.x, pr[f + 1] - hf.y);
+              dk[2 * e4 + f / 2] = pack_bf16(ds[f], ds[f + 1]);
+            }
           }
-          // P = hi + lo, both bf16: dV takes both halves, so P's own rounding
-          // (2^-9 relative) does not reach dV on top of dV's final bf16 rounding
-          const __nv_bfloat162 hi = __floats2bfloat162_rn(pr[0], pr[1]);
-          const float2 hf = __bfloat1622float2(hi);
-          pk[e / 2] = *reinterpret_cast<const uint32_t*>(&hi);
-          plo[e / 2] = pack_bf16(pr[0] - hf.x, pr[1] - hf.y);
-          dk[e / 2] = pack_bf16(ds[0], ds[1]);
         }
-        // in place over this quarter's own (already read) columns
-        tmem_st16(tl + C::TM_S + cg * 32, pk);
-        tmem_st16(tl + C::TM_S + cg * 32 + 16, plo);
-        tmem_st16(tl + C::TM_DP + cg * 32, dk);
+        // in place over this chunk's own (already read) columns
+        tmem_st16(tl + C::TM_S + q * 32, pk);
+        tmem_st16(tl + C::TM_S + q * 32 + 16, plo);
+        tmem_st16(tl + C::TM_DP + q * 32, dk);
         // dS (query-major) into SMEM for dQ = dS K: row c of chunk (j / 64)
         // holds dS[j][c] for 64 consecutive j, 16-byte pieces XOR-swizzled by c % 8
         {
-          const int chunk = cg >> 1;
-          const int piece0 = (cg & 1) * 4;
+          const int chunk = q >> 1;
+          const int piece0 = (q & 1) * 4;
           uint8_t* rowp = base_g + C::OFF_DS + chunk * C::TILE + c * 128;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
@@ -337,8 +350,8 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
                 make_uint4(dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
           }
         }
-        tmem_wait_st();
       }
+      tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
@@ -359,10 +372,12 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         break;
       }
       uint8_t* stg = base_g + C::OFF_STG + (it & 1) * C::STG_BYTES;
-      {
-        uint32_t r[16];  // dQ columns [16 cg, 16 cg + 16)
-        tmem_ld16_sync(tl + C::TM_DQ + cg * 16, r);
-        stage_row16(stg + (cg >> 1) * (C::STG_BYTES / 2), c, (cg & 1) * 4, r, p.tau);
+#pragma unroll
+      for (int k = 0; k < C::CPT; ++k) {
+        const int col = (cg * C::CPT + k) * 16;  // dQ columns [col, col + 16)
+        uint32_t r[16];
+        tmem_ld16_sync(tl + C::TM_DQ + col, r);
+        stage_row16(stg + (col >> 5) * (C::STG_BYTES / 2), c, ((col >> 4) & 1) * 4, r, p.tau);
       }
       fence_proxy_async_smem();
       if (!group_sync()) {
@@ -389,12 +404,15 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
     }
     if (ok) {
       uint8_t* stg = base_g + C::OFF_STG;
-      {
-        uint32_t r[16];  // dV, dK columns [16 cg, 16 cg + 16)
-        tmem_ld16_sync(tl + C::TM_DV + cg * 16, r);
-        stage_row16(stg + (cg >> 1) * (C::STG_BYTES / 2), c, (cg & 1) * 4, r, 1.f);
-        tmem_ld16_sync(tl + C::TM_DK + cg * 16, r);
-        stage_row16(stg + C::STG_BYTES + (cg >> 1) * (C::STG_BYTES / 2), c, (cg & 1) * 4, r, p.tau);
+#pragma unroll
+      for (int k = 0; k < C::CPT; ++k) {
+        const int col = (cg * C::CPT + k) * 16;  // dV, dK columns [col, col + 16)
+        uint32_t r[16];
+        tmem_ld16_sync(tl + C::TM_DV + col, r);
+        stage_row16(stg + (col >> 5) * (C::STG_BYTES / 2), c, ((col >> 4) & 1) * 4, r, 1.f);
+        tmem_ld16_sync(tl + C::TM_DK + col, r);
+        stage_row16(stg + C::STG_BYTES + (col >> 5) * (C::STG_BYTES / 2), c, ((col >> 4) & 1) * 4,
+                    r, p.tau);
       }
       fence_proxy_async_smem();
       ok = group_sync();

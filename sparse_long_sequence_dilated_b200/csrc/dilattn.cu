@@ -269,7 +269,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   if (units > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
   int rc = trace_mark(g_trace_begin, stream);
   if (rc != DILATTN_OK) return rc;
-  fwd_tile_kernel<D><<<(unsigned)units, 192, FwdCfg<D>::SMEM_BYTES, stream>>>(p);
+  fwd_tile_kernel<D><<<(unsigned)units, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM_BYTES, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd_tile_kernel launch");
   rc = trace_mark(g_trace_end, stream);

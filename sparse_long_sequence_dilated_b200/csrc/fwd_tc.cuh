@@ -50,14 +50,15 @@ struct FwdParams {
 template <int D>
 struct FwdCfg {
   static constexpr int KCH = D / 64;                 // 128-byte column chunks per row
-  static constexpr int STAGES = 2;                   // K/V ring depth
+  static constexpr int KST = 3;                      // K ring depth (a stage frees after its S MMA)
+  static constexpr int VST = 2;                      // V ring depth (a stage frees after its PV MMA)
   static constexpr int CHUNK_BYTES = BM * 128;       // 128 rows x 64 bf16
   static constexpr int Q_BYTES = KCH * CHUNK_BYTES;
   static constexpr int KV_BYTES = KCH * CHUNK_BYTES;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 2048 + 1024;  // + exchange + alignment slack
   static constexpr int TM_S = 0, TM_P = 128, TM_O = 192;
   static constexpr int TMEM_COLS = (TM_O + D <= 256) ? 256 : 512;
@@ -91,9 +92,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   const uint32_t bars = base + C::OFF_BAR;
   const uint32_t b_qfull = bars;
   auto b_kfull = [&](int s) { return bars + 8u + 8u * s; };
-  auto b_vfull = [&](int s) { return bars + 8u + 8u * C::STAGES + 8u * s; };
-  auto b_empty = [&](int s) { return bars + 8u + 16u * C::STAGES + 8u * s; };
-  const uint32_t b_sfull = bars + 8u + 24u * C::STAGES;
+  auto b_kempty = [&](int s) { return bars + 8u + 8u * C::KST + 8u * s; };
+  auto b_vfull = [&](int s) { return bars + 8u + 16u * C::KST + 8u * s; };
+  auto b_vempty = [&](int s) { return bars + 8u + 16u * C::KST + 8u * C::VST + 8u * s; };
+  const uint32_t b_sfull = bars + 8u + 16u * C::KST + 16u * C::VST;
   const uint32_t b_sfree = b_sfull + 8u;
   const uint32_t b_pfull = b_sfull + 16u;
   const uint32_t b_odone = b_sfull + 24u;
@@ -103,10 +105,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
 
   if (threadIdx.x == 0) {
     mbar_init(b_qfull, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < C::KST; ++s) {
       mbar_init(b_kfull(s), 1);
+      mbar_init(b_kempty(s), 1);
+    }
+    for (int s = 0; s < C::VST; ++s) {
       mbar_init(b_vfull(s), 1);
-      mbar_init(b_empty(s), 1);
+      mbar_init(b_vempty(s), 1);
     }
     mbar_init(b_sfull, 1);
     mbar_init(b_sfree, C::SM_WARPS);
@@ -140,6 +145,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // lane 0 streams Q then the K ring, lane 1 the V ring, independently
     if (lane == 0) {
       int ph, m;
       view_coords(g, si, wu.t * BM, ph, m);
@@ -148,16 +154,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         tma_load_5d(sQ + c * C::CHUNK_BYTES, mq, b_qfull, c * 64, wu.h, ph, m, wu.b);
       int issued = 0;
       for (int it = 0; it < nkv; ++it) {
-        const int s = it % C::STAGES;
-        if (!mbar_wait(b_empty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, p.err)) break;
+        const int s = it % C::KST;
+        if (!mbar_wait(b_kempty(s), ((it / C::KST) & 1) ^ 1, abort_flag, p.err)) break;
         view_coords(g, si, it * BN, ph, m);
         mbar_arrive_expect_tx(b_kfull(s), C::KV_BYTES);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_5d(sK + s * C::KV_BYTES + c * C::CHUNK_BYTES, mk, b_kfull(s), c * 64, wu.h, ph,
-                      m, wu.b);
-        mbar_arrive_expect_tx(b_vfull(s), C::KV_BYTES);
-        for (int c = 0; c < C::KCH; ++c)
-          tma_load_5d(sV + s * C::KV_BYTES + c * C::CHUNK_BYTES, mv, b_vfull(s), c * 64, wu.h, ph,
                       m, wu.b);
         ++issued;
       }
@@ -165,60 +167,92 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         // Drain copies still in flight before the CTA's shared memory goes away.
         volatile int no_abort = 0;
         mbar_wait(b_qfull, 0, &no_abort, nullptr, 200000000ull);
-        for (int it = issued - C::STAGES; it < issued; ++it) {
-          if (it < 0) continue;
-          const int s = it % C::STAGES;
-          const uint32_t par = (it / C::STAGES) & 1;
-          mbar_wait(b_kfull(s), par, &no_abort, nullptr, 200000000ull);
-          mbar_wait(b_vfull(s), par, &no_abort, nullptr, 200000000ull);
-        }
+        for (int it = issued - C::KST; it < issued; ++it)
+          if (it >= 0)
+            mbar_wait(b_kfull(it % C::KST), (it / C::KST) & 1, &no_abort, nullptr, 200000000ull);
+      }
+    } else if (lane == 1) {
+      int ph, m, issued = 0;
+      for (int it = 0; it < nkv; ++it) {
+        const int s = it % C::VST;
+        if (!mbar_wait(b_vempty(s), ((it / C::VST) & 1) ^ 1, abort_flag, p.err)) break;
+        view_coords(g, si, it * BN, ph, m);
+        mbar_arrive_expect_tx(b_vfull(s), C::KV_BYTES);
+        for (int c = 0; c < C::KCH; ++c)
+          tma_load_5d(sV + s * C::KV_BYTES + c * C::CHUNK_BYTES, mv, b_vfull(s), c * 64, wu.h, ph,
+                      m, wu.b);
+        ++issued;
+      }
+      if (*abort_flag) {
+        volatile int no_abort = 0;
+        for (int it = issued - C::VST; it < issued; ++it)
+          if (it >= 0)
+            mbar_wait(b_vfull(it % C::VST), (it / C::VST) & 1, &no_abort, nullptr, 200000000ull);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Event loop: S(j) = Q K_j^T as soon as K_j is resident and the softmax has
+    // read S(j-1); PV(j) as soon as P(j) and V_j are ready. Neither waits for
+    // the other's operands.
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16(BM, BN, 0, 0);  // Q (K-major) x K (K-major)
       constexpr uint32_t kIdO = idesc_bf16(BM, D, 0, 1);   // P (TMEM) x V (MN-major)
-      auto issue_s = [&](int s) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-          const uint64_t a = sw128_desc(sQ + off, 16, 1024);
-          const uint64_t bd = sw128_desc(sK + s * C::KV_BYTES + off, 16, 1024);
-          mma_ss(tmem + C::TM_S, a, bd, kIdS, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int s, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = sw128_desc(sV + s * C::KV_BYTES + kk * 2048, C::CHUNK_BYTES, 1024);
-          mma_ts(tmem + C::TM_O, tmem + C::TM_P + kk * 8, bd, kIdO, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(b_qfull, 0, abort_flag, p.err) &&
-                mbar_wait(b_kfull(0), 0, abort_flag, p.err);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-        mma_commit(b_sfull);
-      }
-      for (int it = 0; ok && it < nkv; ++it) {
-        if (it + 1 < nkv) {
-          const int s1 = (it + 1) % C::STAGES;
-          if (!mbar_wait(b_kfull(s1), ((it + 1) / C::STAGES) & 1, abort_flag, p.err)) break;
-          if (!mbar_wait(b_sfree, it & 1, abort_flag, p.err)) break;
+      bool ok = mbar_wait(b_qfull, 0, abort_flag, p.err);
+      int ns = 0, npv = 0;
+      uint32_t spins = 0;
+      unsigned long long t0 = 0;
+      while (ok && npv < nkv) {
+        bool progressed = false;
+        if (ns < nkv && mbar_test(b_kfull(ns % C::KST), (ns / C::KST) & 1) &&
+            (ns == 0 || mbar_test(b_sfree, (ns - 1) & 1))) {
           tc_fence_after();
-          issue_s(s1);
+          const int ks = ns % C::KST;
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+            const uint64_t a = sw128_desc(sQ + off, 16, 1024);
+            const uint64_t bd = sw128_desc(sK + ks * C::KV_BYTES + off, 16, 1024);
+            mma_ss(tmem + C::TM_S, a, bd, kIdS, kk > 0 ? 1u : 0u);
+          }
           mma_commit(b_sfull);
+          mma_commit(b_kempty(ks));
+          ++ns;
+          progressed = true;
         }
-        if (!mbar_wait(b_pfull, it & 1, abort_flag, p.err)) break;
-        const int s = it % C::STAGES;
-        if (!mbar_wait(b_vfull(s), (it / C::STAGES) & 1, abort_flag, p.err)) break;
-        tc_fence_after();
-        issue_pv(s, it > 0);
-        mma_commit(b_empty(s));
-        mma_commit(b_odone);
+        if (npv < ns && mbar_test(b_pfull, npv & 1) &&
+            mbar_test(b_vfull(npv % C::VST), (npv / C::VST) & 1)) {
+          tc_fence_after();
+          const int vs = npv % C::VST;
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t bd =
+                sw128_desc(sV + vs * C::KV_BYTES + kk * 2048, C::CHUNK_BYTES, 1024);
+            mma_ts(tmem + C::TM_O, tmem + C::TM_P + kk * 8, bd, kIdO,
+                   (npv > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(b_vempty(vs));
+          mma_commit(b_odone);
+          ++npv;
+          progressed = true;
+        }
+        if (progressed) {
+          spins = 0;
+        } else if ((++spins & 1023u) == 0) {
+          // bounded like mbar_wait: give up after 4 s without progress or on abort
+          if (*abort_flag || *reinterpret_cast<volatile int*>(p.err) != 0) {
+            *abort_flag = 1;
+            ok = false;
+          } else if (t0 == 0) {
+            t0 = globaltimer_ns();
+          } else if (globaltimer_ns() - t0 > 4000000000ull) {
+            atomicExch(p.err, (int)kErrWaitTimeout);
+            *abort_flag = 1;
+            ok = false;
+          }
+        }
+        if (progressed) t0 = 0;
       }
     }
     __syncwarp();

@@ -459,3 +459,57 @@ __device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 }  // namespace dil
+
+namespace dil {
+// Packed fp32 pairs (sm_100): one instruction operates on two floats held in
+// a 64-bit register pair.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  return ((uint64_t)__float_as_uint(hi) << 32) | (uint64_t)__float_as_uint(lo);
+}
+__device__ __forceinline__ float f2_lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2_hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// bf16x2 of (lo, hi), round to nearest even, one instruction.
+__device__ __forceinline__ uint32_t pack_bf16_rn(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+// ex2_poly on a pair with packed arithmetic (same steps, same constants):
+// clamp at -125, j = rint(x) via x + 1.5 * 2^23, f = x - j, Horner for 2^f,
+// then j added to the exponent field. (t_bits << 23) equals j << 23 modulo
+// 2^32 because the rounding constant's own bits shift out.
+__device__ __forceinline__ uint64_t ex2_poly2(uint64_t x2) {
+  const float xl = fmaxf(f2_lo(x2), -125.f), xh = fmaxf(f2_hi(x2), -125.f);
+  const uint64_t xc = f2_pack(xl, xh);
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(xc, magic);
+  const uint64_t f = f2_sub(xc, f2_sub(t, magic));
+  uint64_t p = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f,
+                      f2_pack(2.426111251e-01f, 2.426111251e-01f));
+  p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
+  p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
+  const uint32_t lo = (uint32_t)p + ((uint32_t)t << 23);
+  const uint32_t hi = (uint32_t)(p >> 32) + ((uint32_t)(t >> 32) << 23);
+  return ((uint64_t)hi << 32) | lo;
+}
+}  // namespace dil

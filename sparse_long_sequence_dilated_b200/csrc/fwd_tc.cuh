@@ -18,12 +18,13 @@
 //   warp 0      TMA producer: Q tile once, then a ring of K/V tiles.
 //   warp 1      TMEM allocator and single-thread MMA issuer:
 //               S = Q K^T (SMEM x SMEM -> TMEM), O += P V (TMEM x SMEM -> TMEM).
-//   warps 2..9  softmax: warp w takes TMEM lanes 32 (w % 4) .. + 31 (one query
-//               row per thread) and column half (w - 2) / 4 of S. The two
-//               halves of a row swap partial maxima through shared memory,
-//               agree on one exponent reference, keep their own partial sums,
-//               write their half of P (bf16, TMEM) and rescale / store their
-//               half of O.
+//   warps 2..5  softmax: warp w takes TMEM lanes 32 (w % 4) .. + 31, one query
+//               row per thread: fp32 row max (3-input max), P = exp2(S*scale - m)
+//               with packed fp32x2 arithmetic (5 of every 8 column pairs on the
+//               MUFU ex2, 3 on an FMA-pipe polynomial), P stored to TMEM as
+//               bf16, O rescaled in TMEM when the reference max moves, epilogue.
+// Rows are one per thread: at d = 64 the softmax, not the MMA, bounds a tile,
+// so its issue slots are the budget every choice above is made against.
 // TMEM columns: S [0,128), P [128,192) (bf16 pairs), O [192, 192+D).
 #pragma once
 
@@ -59,13 +60,12 @@ struct FwdCfg {
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
-  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 2048 + 1024;  // + exchange + alignment slack
+  static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
   static constexpr int TM_S = 0, TM_P = 128, TM_O = 192;
   static constexpr int TMEM_COLS = (TM_O + D <= 256) ? 256 : 512;
   static constexpr int MIN_BLOCKS = (D == 64) ? 2 : 1;
-  static constexpr int SM_WARPS = 8;             // softmax warps: 4 lane quarters x 2 column halves
+  static constexpr int SM_WARPS = 4;             // softmax warps: one query row per thread
   static constexpr int THREADS = 64 + 32 * SM_WARPS;
-  static constexpr int OFF_XCH = OFF_BAR + 256;  // [2 parity][2 halves][128 rows] fp32 exchange
 };
 
 template <int D>
@@ -99,7 +99,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   const uint32_t b_sfree = b_sfull + 8u;
   const uint32_t b_pfull = b_sfull + 16u;
   const uint32_t b_odone = b_sfull + 24u;
-  auto b_pair = [&](int k) { return b_sfull + 32u + 8u * k; };  // two halves of lane quarter k
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
 
@@ -117,7 +116,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     mbar_init(b_sfree, C::SM_WARPS);
     mbar_init(b_pfull, C::SM_WARPS);
     mbar_init(b_odone, 1);
-    for (int k = 0; k < 4; ++k) mbar_init(b_pair(k), 2);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -258,76 +256,49 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
-    constexpr int HC = BN / 2;   // S columns per half
-    constexpr int HO = D / 2;    // O columns per half
     const int q4 = warp & 3;
-    const int ch = (warp - 2) >> 2;
     const int row = q4 * 32 + lane;
     const int vq = wu.t * BM + row;
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
     const float sc = p.scale_log2;
-    float* xch = reinterpret_cast<float*>(base_g + C::OFF_XCH);  // [2][2][128]
+    const uint64_t sc2 = f2_pack(sc, sc);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    uint32_t pphase = 0;
-    // swap one value per row with the other half of the row (bounded wait)
-    auto swap_with_pair = [&](float mine, float& theirs) -> bool {
-      const int par = pphase & 1;
-      xch[(par * 2 + ch) * BM + row] = mine;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b_pair(q4));
-      const bool r = warp_wait(b_pair(q4), par, abort_flag, p.err);
-      ++pphase;
-      theirs = xch[(par * 2 + (ch ^ 1)) * BM + row];
-      return r;
-    };
     for (int it = 0; it < nkv; ++it) {
       if (!warp_wait(b_sfull, it & 1, abort_flag, p.err)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[HC];
-      {
-        uint32_t ra[32], rb[32];
-        tmem_ld32x2_sync(tl + C::TM_S + ch * HC, tl + C::TM_S + ch * HC + 32, ra, rb);
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          s[c] = __uint_as_float(ra[c]);
-          s[32 + c] = __uint_as_float(rb[c]);
-        }
-      }
+      uint32_t raw[BN];
+      tmem_ld128_sync(tl + C::TM_S, raw);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(b_sfree);
 
-      const int c0 = ch * HC;  // first S column of this half
       if (p.causal) {
         if (it == wu.t) {
 #pragma unroll
-          for (int c = 0; c < HC; ++c)
-            if (c0 + c > row) s[c] = -INFINITY;
+          for (int c = 0; c < BN; ++c)
+            if (c > row) raw[c] = 0xff800000u;  // -inf
         }
       } else if (it == nkv - 1) {
-        const int lim = si.n - it * BN - c0;
+        const int lim = si.n - it * BN;
 #pragma unroll
-        for (int c = 0; c < HC; ++c)
-          if (c >= lim) s[c] = -INFINITY;
+        for (int c = 0; c < BN; ++c)
+          if (c >= lim) raw[c] = 0xff800000u;
       }
-      float mx8[8];
+      // row max: four independent chains of 3-input max
+      float a0 = __uint_as_float(raw[0]), a1 = __uint_as_float(raw[1]);
+      float a2 = __uint_as_float(raw[2]), a3 = __uint_as_float(raw[3]);
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = s[k];
-#pragma unroll
-      for (int c = 8; c < HC; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], s[c]);
-      const float mx_half = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                  fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      float mx_other;
-      if (!swap_with_pair(mx_half, mx_other)) {
-        ok = false;
-        break;
+      for (int c = 4; c < BN; c += 8) {
+        a0 = max3(a0, __uint_as_float(raw[c]), __uint_as_float(raw[c + 1]));
+        a1 = max3(a1, __uint_as_float(raw[c + 2]), __uint_as_float(raw[c + 3]));
+        a2 = max3(a2, __uint_as_float(raw[c + 4]), __uint_as_float(raw[c + 5]));
+        a3 = max3(a3, __uint_as_float(raw[c + 6]), __uint_as_float(raw[c + 7]));
       }
-      // both halves compute the same row max, hence the same reference
-      const float mx = ch == 0 ? fmaxf(mx_half, mx_other) : fmaxf(mx_other, mx_half);
+      const float mx = max3(a0, a1, fmaxf(a2, a3));
       // The exponent reference m_run moves only when the tile's max exceeds it
       // by more than 8 (log2 units); otherwise P <= 2^8 and O is not rescaled.
       // out = O / l and lse = m_run + log2(l) use the same reference, so the
@@ -336,20 +307,27 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       const bool move = m_tile > m_run + 8.f;
       const float m_new = move ? m_tile : m_run;
       const float alpha = move ? ex2(m_run - m_new) : 1.f;
-      uint32_t pk[HC / 2];
-      float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+      const uint64_t negm2 = f2_pack(-m_new, -m_new);
+      uint64_t sum2a = 0, sum2b = 0;  // +0.0f pairs
+      uint32_t pk[BN / 2];
 #pragma unroll
-      for (int c = 0; c < HC / 2; ++c) {
-        const float x0 = fmaf(s[2 * c], sc, -m_new);
-        const float x1 = fmaf(s[2 * c + 1], sc, -m_new);
-        // one column in four takes the FMA-pipe exp2, the rest the MUFU ex2
-        const float p0 = ex2(x0);
-        const float p1 = (c & 1) ? ex2_poly(x1) : ex2(x1);
-        sum4[c & 3] += p0 + p1;
-        pk[c] = pack_bf16(p0, p1);
+      for (int c = 0; c < BN / 2; ++c) {
+        const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(raw[2 * c]),
+                                           __uint_as_float(raw[2 * c + 1])), sc2, negm2);
+        uint64_t p2;
+        if ((c & 7) >= 5) {
+          p2 = ex2_poly2(x2);  // 3 pairs in 8 on the FMA pipe
+        } else {
+          p2 = f2_pack(ex2(f2_lo(x2)), ex2(f2_hi(x2)));
+        }
+        if (c & 1)
+          sum2a = f2_add(sum2a, p2);
+        else
+          sum2b = f2_add(sum2b, p2);
+        pk[c] = pack_bf16_rn(f2_lo(p2), f2_hi(p2));
       }
-      const float sum = (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
-      l_run = l_run * alpha + sum;  // this half's part of the row sum
+      const uint64_t sum2 = f2_add(sum2a, sum2b);
+      l_run = l_run * alpha + (f2_lo(sum2) + f2_hi(sum2));
       m_run = m_new;
 
       if (it > 0) {
@@ -361,38 +339,34 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         tc_fence_after();
         if (__any_sync(0xffffffffu, move)) {
 #pragma unroll
-          for (int c4 = 0; c4 < HO / 32; ++c4) {
+          for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t r[32];
-            tmem_ld32_sync(tl + C::TM_O + ch * HO + c4 * 32, r);
+            tmem_ld32_sync(tl + C::TM_O + c4 * 32, r);
 #pragma unroll
             for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * alpha);
-            tmem_st32_sync(tl + C::TM_O + ch * HO + c4 * 32, r);
+            tmem_st32_sync(tl + C::TM_O + c4 * 32, r);
           }
         }
       }
-      // this half's P columns, packed two per 32-bit TMEM column
-      tmem_st16(tl + C::TM_P + ch * (HC / 2), *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
-      tmem_st16(tl + C::TM_P + ch * (HC / 2) + 16,
-                *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+#pragma unroll
+      for (int c4 = 0; c4 < BN / 32; ++c4)
+        tmem_st16(tl + C::TM_P + c4 * 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[c4 * 16]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(b_pfull);
     }
-    float l_other = 0.f;
-    if (ok) ok = swap_with_pair(l_run, l_other);
     if (ok && warp_wait(b_odone, (nkv - 1) & 1, abort_flag, p.err)) {
       tc_fence_after();
       const bool valid = vq < si.n;
       const long long prow =
           g.part_base + ((long long)(wu.b * p.H + wu.h) * g.nseg + wu.seg) * g.nmax + vq;
-      const float l_tot = ch == 0 ? l_run + l_other : l_other + l_run;
-      const float inv = 1.f / l_tot;
-      float* dst = p.part_o + prow * D + ch * HO;
+      const float inv = 1.f / l_run;
+      float* dst = p.part_o + prow * D;
 #pragma unroll
-      for (int c4 = 0; c4 < HO / 32; ++c4) {
+      for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t r[32];
-        tmem_ld32_sync(tl + C::TM_O + ch * HO + c4 * 32, r);
+        tmem_ld32_sync(tl + C::TM_O + c4 * 32, r);
         if (valid) {
 #pragma unroll
           for (int c = 0; c < 32; c += 4) {
@@ -403,7 +377,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
           }
         }
       }
-      if (valid && ch == 0) p.part_lse[prow] = (m_run + __log2f(l_tot)) * 0.69314718055994531f;
+      if (valid) p.part_lse[prow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
     }
     tc_fence_before();
   }

@@ -17,11 +17,12 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "sparse_long_sequence_dilated_b200", "csrc", "common.cuh")
 
 
-def kernel_coeffs():
+def kernel_coeffs(fn="float ex2_poly(float x)"):
     text = open(SRC, encoding="utf-8").read()
-    body = text[text.index("float ex2_poly(float x)"):]
+    body = text[text.index(fn):]
     body = body[:body.index("return")]
     nums = [float(x.rstrip("f")) for x in re.findall(r"[0-9]\.[0-9]+e[-+][0-9]+f", body)]
+    nums = list(dict.fromkeys(nums))  # the packed form repeats each constant for both lanes
     # Horner order in the source: c3, c2, c1, c0
     return np.array(nums[::-1], dtype=np.float32)
 
@@ -44,9 +45,19 @@ def ex2_poly_emulated(x, c):
 
 def test_kernel_constants_match_fit():
     want = fit_exp2_poly.remez().astype(np.float32)
-    got = kernel_coeffs()
-    assert got.shape == (4,)
-    np.testing.assert_allclose(got, want, rtol=2e-7, atol=0)
+    for fn in ("float ex2_poly(float x)", "uint64_t ex2_poly2(uint64_t x2)"):
+        got = kernel_coeffs(fn)
+        assert got.shape == (4,), fn
+        np.testing.assert_allclose(got, want, rtol=2e-7, atol=0, err_msg=fn)
+
+
+def test_exponent_shift_forms_agree():
+    # the packed form adds (t_bits << 23) instead of ((t_bits - 0x4B400000) << 23)
+    x = np.linspace(-125.0, 126.0, 100001).astype(np.float32)
+    t = (x + np.float32(12582912.0)).astype(np.float32).view(np.uint32).astype(np.uint64)
+    a = ((t - 0x4B400000) << 23) & 0xFFFFFFFF
+    b = (t << 23) & 0xFFFFFFFF
+    assert np.array_equal(a, b)
 
 
 def test_relative_error_bound():

@@ -22,6 +22,7 @@ struct PatternGeom {
   int nseg;            // ceil(N / w): number of segments
   int nmax;            // ceil(min(w, N) / r): row capacity of one segment
   int ntiles;          // ceil(nmax / BM)
+  int pstride;         // ntiles * BM: partial-buffer rows per segment (whole tiles)
   int nmod;            // N mod r: phases below it have one row more in the strided view
   long long part_base; // first row of this pattern in the partial-result buffer
 };
@@ -511,5 +512,16 @@ __device__ __forceinline__ uint64_t ex2_poly2(uint64_t x2) {
   const uint32_t lo = (uint32_t)p + ((uint32_t)t << 23);
   const uint32_t hi = (uint32_t)(p >> 32) + ((uint32_t)(t >> 32) << 23);
   return ((uint64_t)hi << 32) | lo;
+}
+}  // namespace dil
+
+namespace dil {
+// 2-D tiled TMA store from shared memory (bulk group).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1)
+      : "memory");
 }
 }  // namespace dil

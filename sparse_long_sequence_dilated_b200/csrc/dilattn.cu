@@ -164,6 +164,42 @@ int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CU
   return DILATTN_OK;
 }
 
+// 2-D view of the forward's fp32 partial outputs [rows][d] for TMA stores:
+// box 32 columns (128 bytes, 128-byte swizzle) x 128 rows.
+int partial_map(const float* ptr, long long rows, int d, CUtensorMap* out) {
+  MapKey key{ptr, (int)(rows >> 31), (int)(rows & 0x7fffffff), d, -1, -1, -1, 2};
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *out = it->second;
+      return DILATTN_OK;
+    }
+  }
+  int rc = get_encoder();
+  if (rc != DILATTN_OK) return rc;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 4};
+  cuuint32_t box[2] = {32, (cuuint32_t)BM};
+  cuuint32_t estr[2] = {1, 1};
+  CUtensorMap m;
+  CUresult cr = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims,
+                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (cr != CUDA_SUCCESS) {
+    snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)cr);
+    return DILATTN_ERR_CUDA;
+  }
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    if (g_maps.size() > 4096) g_maps.clear();
+    g_maps[key] = m;
+  }
+  *out = m;
+  return DILATTN_OK;
+}
+
 // ------------------------------------------------------------------ validation
 int check_shape(int B, int N, int H, int d, const int* w, const int* r, int npat, int causal) {
   if (B < 1 || N < 1 || H < 1 || d < 1) return DILATTN_ERR_INVALID_ARG;
@@ -198,9 +234,10 @@ long long make_geoms(int B, int N, int H, const int* w, const int* r, int npat,
     const long long span = std::min<long long>(w[i], N);
     g.nmax = (int)((span + r[i] - 1) / r[i]);
     g.ntiles = (g.nmax + BM - 1) / BM;
+    g.pstride = g.ntiles * BM;
     g.nmod = N % r[i];
     g.part_base = rows;
-    rows += (long long)B * H * g.nseg * g.nmax;
+    rows += (long long)B * H * g.nseg * g.pstride;
   }
   return rows;
 }
@@ -255,6 +292,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   p.part_o = reinterpret_cast<float*>(ws);
   p.part_lse = reinterpret_cast<float*>((char*)ws + align256((size_t)rows * D * 4));
   p.err = st->err_word;
+  {
+    int rc = partial_map(p.part_o, rows, D, &p.tm_po);
+    if (rc != DILATTN_OK) return rc;
+  }
   for (int i = 0; i < npat; ++i) {
     const void* src[3] = {q, k, v};
     CUtensorMap* dst[3] = {&p.tmq[i], &p.tmk[i], &p.tmv[i]};

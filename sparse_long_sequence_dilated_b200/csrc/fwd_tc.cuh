@@ -39,6 +39,7 @@ struct FwdParams {
   CUtensorMap tmq_t[kMaxPat]; // phases [0, N mod r), floor(N/r) + 1 rows
   CUtensorMap tmk_t[kMaxPat];
   CUtensorMap tmv_t[kMaxPat];
+  CUtensorMap tm_po;          // partial outputs [rows][D] fp32, box 32 x 128 (128-byte swizzle)
   PatternGeom pat[kMaxPat];
   int npat, B, N, H, causal;
   float scale_log2;  // log2(e) / sqrt(d)
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   const uint32_t b_sfree = b_sfull + 8u;
   const uint32_t b_pfull = b_sfull + 16u;
   const uint32_t b_odone = b_sfull + 24u;
+  const uint32_t b_epi = b_sfull + 32u;  // the four softmax warps have staged their output rows
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
 
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     mbar_init(b_sfree, C::SM_WARPS);
     mbar_init(b_pfull, C::SM_WARPS);
     mbar_init(b_odone, 1);
+    mbar_init(b_epi, 4);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -358,26 +361,41 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     }
     if (ok && warp_wait(b_odone, (nkv - 1) & 1, abort_flag, p.err)) {
       tc_fence_after();
-      const bool valid = vq < si.n;
-      const long long prow =
-          g.part_base + ((long long)(wu.b * p.H + wu.h) * g.nseg + wu.seg) * g.nmax + vq;
+      // The tile's 128 partial rows are one contiguous block of the partial
+      // buffer (segments own whole tiles there; rows past the segment land in
+      // padding no one reads). O / l goes through the now idle K ring, staged
+      // as D/32 chunks of [128 rows][32 fp32] with 128-byte swizzle, and leaves
+      // by TMA stores.
+      const long long prow0 =
+          g.part_base + ((long long)(wu.b * p.H + wu.h) * g.nseg + wu.seg) * g.pstride +
+          (long long)wu.t * BM;
       const float inv = 1.f / l_run;
-      float* dst = p.part_o + prow * D;
+      uint8_t* stg = base_g + C::OFF_K;
 #pragma unroll
       for (int c4 = 0; c4 < D / 32; ++c4) {
         uint32_t r[32];
         tmem_ld32_sync(tl + C::TM_O + c4 * 32, r);
-        if (valid) {
+        uint8_t* rowp = stg + c4 * (BM * 128) + row * 128;
 #pragma unroll
-          for (int c = 0; c < 32; c += 4) {
-            float4 o4 = make_float4(__uint_as_float(r[c]) * inv, __uint_as_float(r[c + 1]) * inv,
-                                    __uint_as_float(r[c + 2]) * inv,
-                                    __uint_as_float(r[c + 3]) * inv);
-            *reinterpret_cast<float4*>(dst + c4 * 32 + c) = o4;
-          }
+        for (int k = 0; k < 8; ++k) {
+          const float4 v = make_float4(__uint_as_float(r[4 * k]) * inv,
+                                       __uint_as_float(r[4 * k + 1]) * inv,
+                                       __uint_as_float(r[4 * k + 2]) * inv,
+                                       __uint_as_float(r[4 * k + 3]) * inv);
+          *reinterpret_cast<float4*>(rowp + ((k ^ (row & 7)) * 16)) = v;
         }
       }
-      if (valid) p.part_lse[prow] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      if (vq < si.n) p.part_lse[prow0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_epi);
+      if (warp_wait(b_epi, 0, abort_flag, p.err) && warp == 2 && lane == 0) {
+#pragma unroll
+        for (int c4 = 0; c4 < D / 32; ++c4)
+          tma_store_2d(&p.tm_po, sK + c4 * (BM * 128), c4 * 32, (int)prow0);
+        bulk_commit();
+        bulk_wait_read<0>();  // the staging buffer stays until the stores have read it
+      }
     }
     tc_fence_before();
   }

@@ -76,7 +76,7 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
     const int seg = n / g.w;
     const int rel = n - seg * g.w - h % g.r;
     if (rel < 0 || rel % g.r != 0) continue;
-    const long long pr = g.part_base + ((long long)bh * g.nseg + seg) * g.nmax + rel / g.r;
+    const long long pr = g.part_base + ((long long)bh * g.nseg + seg) * g.pstride + rel / g.r;
     const float li = __ldg(p.part_lse + pr);
     const float4* src = reinterpret_cast<const float4*>(p.part_o + pr * D + sub * PER);
     float4 x[PER / 4];

@@ -72,8 +72,10 @@ def test_fwd_rejects_missing_or_small_workspace():
 def test_workspace_sizes():
     lib = dilattn.load()
     w, r, n = _pats(((128, 1), (256, 2), (512, 4)))
-    # partial rows: sum_i B*H*nseg_i*ceil(min(w,N)/r) = 2*3*(4*128 + 2*128 + 1*128)
+    # partial rows: sum_i B*H*nseg_i*(128*ceil(ceil(min(w,N)/r)/128)) = 2*3*(4*128 + 2*128 + 1*128)
     rows = 2 * 3 * (512 + 256 + 128)
+    assert lib.dilattn_fwd_workspace_size(1, 1000, 1, 64, *_pats(((1000, 3),))) == \
+        (334 + 50) // 128 * 128 * 64 * 4 + (384 * 4 + 255) // 256 * 256  # 334 rows -> 384
     align = lambda x: (x + 255) // 256 * 256
     assert lib.dilattn_fwd_workspace_size(2, 512, 3, 64, w, r, n) == align(rows * 64 * 4) + align(rows * 4)
     t = 2 * 512 * 3 * 64 * 4

@@ -307,29 +307,35 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           // key rows past the segment, and (on the diagonal) queries before the
           // key, get P = 0; elsewhere no mask is needed
           const int jmin = !key_valid ? 1 << 30 : (diag ? c - q * 32 : 0);
+          const bool masked = jmin > 0;
+          const uint64_t sc2 = f2_pack(sc, sc);
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
             const float4 Lq = L4[e4], Dq = D4[e4];
-            const float lv[4] = {Lq.x, Lq.y, Lq.z, Lq.w};
-            const float dd[4] = {Dq.x, Dq.y, Dq.z, Dq.w};
-            float pr[4], ds[4];
+            const uint64_t nl2[2] = {f2_pack(-Lq.x, -Lq.y), f2_pack(-Lq.z, -Lq.w)};
+            const uint64_t dd2[2] = {f2_pack(Dq.x, Dq.y), f2_pack(Dq.z, Dq.w)};
 #pragma unroll
-            for (int f = 0; f < 4; ++f) {
-              const int e = 4 * e4 + f;
-              float pv = ex2(fmaf(__uint_as_float(sv[e]), sc, -lv[f]));
-              pv = e >= jmin ? pv : 0.f;
-              pr[f] = pv;
-              ds[f] = pv * (__uint_as_float(dv[e]) - dd[f]);
-            }
-#pragma unroll
-            for (int f = 0; f < 4; f += 2) {
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = 4 * e4 + 2 * h2;
+              const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
+                                         sc2, nl2[h2]);
+              float p0 = ex2(f2_lo(x2)), p1 = ex2(f2_hi(x2));
+              if (masked) {
+                p0 = e >= jmin ? p0 : 0.f;
+                p1 = e + 1 >= jmin ? p1 : 0.f;
+              }
+              const uint64_t p2 = f2_pack(p0, p1);
+              // dS = P (dP - D)
+              const uint64_t ds2 = f2_mul(
+                  p2, f2_sub(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), dd2[h2]));
               // P = hi + lo, both bf16: dV takes both halves, so P's own rounding
               // (2^-9 relative) does not reach dV on top of dV's final bf16 rounding
-              const __nv_bfloat162 hi = __floats2bfloat162_rn(pr[f], pr[f + 1]);
-              const float2 hf = __bfloat1622float2(hi);
-              pk[2 * e4 + f / 2] = *reinterpret_cast<const uint32_t*>(&hi);
-              plo[2 * e4 + f / 2] = pack_bf16(pr[f] - hf.x, pr[f + 1] - hf.y);
-              dk[2 * e4 + f / 2] = pack_bf16(ds[f], ds[f + 1]);
+              const uint32_t hi = pack_bf16_rn(p0, p1);
+              const uint64_t hi2 = f2_pack(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u));
+              const uint64_t lo2 = f2_sub(p2, hi2);
+              pk[e / 2] = hi;
+              plo[e / 2] = pack_bf16_rn(f2_lo(lo2), f2_hi(lo2));
+              dk[e / 2] = pack_bf16_rn(f2_lo(ds2), f2_hi(ds2));
             }
           }
         }

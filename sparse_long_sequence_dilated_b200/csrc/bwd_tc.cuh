@@ -14,8 +14,11 @@
 //   S^T  = K Q^T,  dP^T = V dO^T                     (SMEM x SMEM -> TMEM)
 //   P^T  = exp2(S^T tau log2e - L log2e), dS^T = P^T (dP^T - D)   (threads)
 //   dV  += P^T dO,  dK += dS^T Q                     (TMEM x SMEM -> TMEM)
-//          (P^T enters dV as two bf16 halves, hi + lo, for an fp32-grade product)
 //   dQ   = dS K                                      (SMEM x SMEM -> TMEM)
+// P and dS enter their products as two bf16 halves each, hi + lo, so the
+// products are fp32-grade: the gradients' own bf16 rounding (half an ulp is
+// 0.0078 at |g| in [2, 4)) leaves no room for a 2^-9 rounding of P or dS under
+// a 2e-2 bound.
 // dQ is staged in shared memory after every pair and added to an fp32
 // accumulator by a TMA reduce-add; dK, dV are added the same way once at the
 // end (other patterns and tiles reach the same rows). The three accumulators
@@ -26,10 +29,10 @@
 // serves TMEM lanes 32 (w % 4) .. + 31 and column group (w - 2) / 4, i.e. the
 // CPT = 4 / NCG consecutive 32-column chunks of that group.
 // TMEM columns: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256,320),
-// dK [320,384), dQ [384,448). P^T (hi, lo) and dS^T overwrite S^T and dP^T in
+// dK [320,384), dQ [384,448). P^T and dS^T (hi, lo) overwrite S^T and dP^T in
 // place, each 32-column quarter by the warps that read it: query columns
-// [32q, 32q + 32) keep P^T hi at TM_S + 32q + [0, 16), lo at TM_S + 32q + [16, 32)
-// and dS^T at TM_DP + 32q + [0, 16).
+// [32q, 32q + 32) keep P^T hi at TM_S + 32q + [0, 16), lo at TM_S + 32q + [16, 32),
+// and dS^T hi / lo at TM_DP + 32q + [0, 16) / [16, 32).
 #pragma once
 
 #include "common.cuh"
@@ -62,10 +65,11 @@ struct BwdCfg {
   static constexpr int OFF_V = OFF_K + TILE;
   static constexpr int OFF_Q = OFF_V + TILE;                 // STAGES tiles
   static constexpr int OFF_DO = OFF_Q + STAGES * TILE;       // STAGES tiles
-  static constexpr int OFF_DS = OFF_DO + STAGES * TILE;      // 2 chunks of [128 kv][64 q]
-  static constexpr int OFF_STG = OFF_DS + 2 * TILE;          // 2 x fp32 [2][128][32] staging
+  static constexpr int OFF_DS = OFF_DO + STAGES * TILE;      // dS hi: 2 chunks of [128 kv][64 q]
+  static constexpr int OFF_DSL = OFF_DS + 2 * TILE;          // dS lo, same layout
+  static constexpr int OFF_STG = OFF_DSL + 2 * TILE;         // fp32 [2][128][32] staging
   static constexpr int STG_BYTES = 2 * BM * 128;             // one 128 x 64 fp32 tile
-  static constexpr int OFF_L = OFF_STG + 2 * STG_BYTES;      // STAGES x 128 floats
+  static constexpr int OFF_L = OFF_STG + STG_BYTES;          // STAGES x 128 floats
   static constexpr int OFF_D = OFF_L + STAGES * BM * 4;      // STAGES x 128 floats
   static constexpr int OFF_BAR = OFF_D + STAGES * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
@@ -110,6 +114,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   const int lane = threadIdx.x & 31;
   const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
   const uint32_t sQ = base + C::OFF_Q, sDO = base + C::OFF_DO, sDS = base + C::OFF_DS;
+  const uint32_t sDSL = base + C::OFF_DSL;
   float* sL = reinterpret_cast<float*>(base_g + C::OFF_L);
   float* sD = reinterpret_cast<float*>(base_g + C::OFF_D);
   const uint32_t bars = base + C::OFF_BAR;
@@ -255,13 +260,16 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           const uint64_t bq = sw128_desc(sQ + s * C::TILE + kk * 2048, C::TILE, 1024);
           const uint32_t a_ds = tmem + C::TM_DP + (kk >> 1) * 32 + (kk & 1) * 8;
           mma_ts(tmem + C::TM_DK, a_ds, bq, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(tmem + C::TM_DK, a_ds + 16, bq, kIdKV, 1u);
         }
         mma_commit(b_kv2);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t a = sw128_desc(sDS + kk * 2048, C::TILE, 1024);
+          const uint64_t al = sw128_desc(sDSL + kk * 2048, C::TILE, 1024);
           const uint64_t b = sw128_desc(sK + kk * 2048, C::TILE, 1024);
           mma_ss(tmem + C::TM_DQ, a, b, kIdQ, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + C::TM_DQ, al, b, kIdQ, 1u);
         }
         mma_commit(b_qempty(s));
         mma_commit(b_dq);
@@ -300,7 +308,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       for (int q = cg * C::CPT; q < cg * C::CPT + C::CPT; ++q) {
         const float4* L4 = reinterpret_cast<const float4*>(sL + s * BM + q * 32);
         const float4* D4 = reinterpret_cast<const float4*>(sD + s * BM + q * 32);
-        uint32_t pk[16], plo[16], dk[16];
+        uint32_t pk[16], plo[16], dk[16], dkl[16];
         {
           uint32_t sv[32], dv[32];
           tmem_ld32x2_sync(tl + C::TM_S + q * 32, tl + C::TM_DP + q * 32, sv, dv);
@@ -335,7 +343,12 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
               const uint64_t lo2 = f2_sub(p2, hi2);
               pk[e / 2] = hi;
               plo[e / 2] = pack_bf16_rn(f2_lo(lo2), f2_hi(lo2));
-              dk[e / 2] = pack_bf16_rn(f2_lo(ds2), f2_hi(ds2));
+              const uint32_t dhi = pack_bf16_rn(f2_lo(ds2), f2_hi(ds2));
+              const uint64_t dhi2 =
+                  f2_pack(__uint_as_float(dhi << 16), __uint_as_float(dhi & 0xffff0000u));
+              const uint64_t dlo2 = f2_sub(ds2, dhi2);
+              dk[e / 2] = dhi;
+              dkl[e / 2] = pack_bf16_rn(f2_lo(dlo2), f2_hi(dlo2));
             }
           }
         }
@@ -343,17 +356,21 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         tmem_st16(tl + C::TM_S + q * 32, pk);
         tmem_st16(tl + C::TM_S + q * 32 + 16, plo);
         tmem_st16(tl + C::TM_DP + q * 32, dk);
+        tmem_st16(tl + C::TM_DP + q * 32 + 16, dkl);
         // dS (query-major) into SMEM for dQ = dS K: row c of chunk (j / 64)
         // holds dS[j][c] for 64 consecutive j, 16-byte pieces XOR-swizzled by c % 8
         {
           const int chunk = q >> 1;
           const int piece0 = (q & 1) * 4;
           uint8_t* rowp = base_g + C::OFF_DS + chunk * C::TILE + c * 128;
+          uint8_t* rowl = base_g + C::OFF_DSL + chunk * C::TILE + c * 128;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const int piece = (piece0 + k) ^ (c & 7);
             *reinterpret_cast<uint4*>(rowp + piece * 16) =
                 make_uint4(dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
+            *reinterpret_cast<uint4*>(rowl + piece * 16) =
+                make_uint4(dkl[4 * k], dkl[4 * k + 1], dkl[4 * k + 2], dkl[4 * k + 3]);
           }
         }
       }
@@ -372,12 +389,12 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         break;
       }
       tc_fence_after();
-      if (threadIdx.x == 64) bulk_wait_read<1>();  // the reduce that last read this buffer is done
+      if (threadIdx.x == 64) bulk_wait_read<0>();  // the previous reduce has read the staging buffer
       if (!group_sync()) {
         ok = false;
         break;
       }
-      uint8_t* stg = base_g + C::OFF_STG + (it & 1) * C::STG_BYTES;
+      uint8_t* stg = base_g + C::OFF_STG;
 #pragma unroll
       for (int k = 0; k < C::CPT; ++k) {
         const int col = (cg * C::CPT + k) * 16;  // dQ columns [col, col + 16)
@@ -393,7 +410,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       if (threadIdx.x == 64) {
         int ph, m;
         view_coords(g, si, t * BM, ph, m);
-        const uint32_t src = sSTG + (it & 1) * C::STG_BYTES;
+        const uint32_t src = sSTG;
         tma_reduce_add_5d(macc, src, 0, wu.h, ph, m, wu.b);
         tma_reduce_add_5d(macc, src + C::STG_BYTES / 2, 32, wu.h, ph, m, wu.b);
         bulk_commit();
@@ -401,9 +418,9 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       tc_fence_before();
     }
     // dK, dV of the key tile (all pairs are complete after the last dQ wait):
-    // dV -> buffer 0, tau * dK -> buffer 1, TMA reduce-add into the dv and dk
-    // accumulators (batch slots 2B + b and B + b). Rows past the segment are
-    // exact zeros (their P was forced to 0).
+    // dV -> the staging buffer, tau * dK -> the dS area (idle now), TMA
+    // reduce-add into the dv and dk accumulators (batch slots 2B + b and
+    // B + b). Rows past the segment are exact zeros (their P was forced to 0).
     if (ok) {
       if (threadIdx.x == 64) bulk_wait_read<0>();
       ok = group_sync();
@@ -417,7 +434,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         tmem_ld16_sync(tl + C::TM_DV + col, r);
         stage_row16(stg + (col >> 5) * (C::STG_BYTES / 2), c, ((col >> 4) & 1) * 4, r, 1.f);
         tmem_ld16_sync(tl + C::TM_DK + col, r);
-        stage_row16(stg + C::STG_BYTES + (col >> 5) * (C::STG_BYTES / 2), c, ((col >> 4) & 1) * 4,
+        stage_row16(base_g + C::OFF_DS + (col >> 5) * (C::STG_BYTES / 2), c, ((col >> 4) & 1) * 4,
                     r, p.tau);
       }
       fence_proxy_async_smem();
@@ -429,9 +446,8 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         view_coords(g, si, u * BN, ph, m);
         tma_reduce_add_5d(macc, sSTG, 0, wu.h, ph, m, 2 * p.B + wu.b);
         tma_reduce_add_5d(macc, sSTG + C::STG_BYTES / 2, 32, wu.h, ph, m, 2 * p.B + wu.b);
-        tma_reduce_add_5d(macc, sSTG + C::STG_BYTES, 0, wu.h, ph, m, p.B + wu.b);
-        tma_reduce_add_5d(macc, sSTG + C::STG_BYTES + C::STG_BYTES / 2, 32, wu.h, ph, m,
-                          p.B + wu.b);
+        tma_reduce_add_5d(macc, sDS, 0, wu.h, ph, m, p.B + wu.b);
+        tma_reduce_add_5d(macc, sDS + C::STG_BYTES / 2, 32, wu.h, ph, m, p.B + wu.b);
         bulk_commit();
       }
     }

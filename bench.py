@@ -236,7 +236,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         dilattn.fwd(q, k, v, pats, causal, out=out, lse=lse, workspace=ws_f)
         if trace is not None:
             dilattn.set_trace_events(trace[2], trace[3])
-        dilattn.bwd(q, k, v, out, lse, do, pats, causal, dq=dq, dk=dk, dv=dv, workspace=ws_b)
+        dilattn.bwd(q, k, v, out, lse, do, pats, causal, dq=dq, dk=dk, dv=dv, workspace=ws_b,
+                    fwd_workspace=ws_f)
         if trace is not None:
             dilattn.set_trace_events(None, None)
 
@@ -288,7 +289,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     def e2e_step():
         qd, kd, vd, dod = (host[n].to(dev, non_blocking=True) for n in NAMES)
         o, l = dilattn.fwd(qd, kd, vd, pats, causal, workspace=ws_f)
-        gq, gk, gv = dilattn.bwd(qd, kd, vd, o, l, dod, pats, causal, workspace=ws_b)
+        gq, gk, gv = dilattn.bwd(qd, kd, vd, o, l, dod, pats, causal, workspace=ws_b,
+                                 fwd_workspace=ws_f)
         for name, t in (("out", o), ("dq", gq), ("dk", gk), ("dv", gv)):
             res_host[name].copy_(t, non_blocking=True)
         lse_host.copy_(l, non_blocking=True)

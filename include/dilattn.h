@@ -77,8 +77,10 @@ const char* dilattn_last_error(void);
 /*
  * Forward. Writes out [B][N][H][d] bf16 and, unless lse is NULL,
  * lse [B][H][N] fp32. Workspace: fp32 per-pattern partial results
- * (one row of d + 1 floats per kept row of every pattern), at least
- * dilattn_fwd_workspace_size(...) bytes.
+ * (one row of d + 1 floats per kept row of every pattern, segments padded to
+ * whole 128-row tiles) followed by an fp32 copy of out; at least
+ * dilattn_fwd_workspace_size(...) bytes. Keep the workspace untouched until
+ * the matching dilattn_bwd if the backward should use that fp32 copy.
  */
 size_t dilattn_fwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
                                   int npat);
@@ -123,12 +125,20 @@ int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, 
  * full derivative of sum(out * dout). The probabilities are recomputed from
  * the saved lse. Workspace: fp32 accumulators for dq, dk, dv and the row
  * term D = rowsum(dout * out), at least dilattn_bwd_workspace_size(...) bytes.
+ *
+ * fwd_workspace: the workspace of the dilattn_fwd call that produced out and
+ * lse, untouched since (fwd_workspace_bytes >= dilattn_fwd_workspace_size).
+ * The backward then forms D from the forward's fp32 copy of out. It may be
+ * NULL: D then comes from the bf16 out, the usual convention, whose rounding
+ * (up to one bf16 ulp of out per element) moves dq and dk by up to about
+ * 1e-2 more at rows whose exact gradient is near zero.
  */
 size_t dilattn_bwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
                                   int npat);
 int dilattn_bwd(const void* q, const void* k, const void* v, const void* out,
                 const float* lse, const void* dout, void* dq, void* dk, void* dv,
                 int B, int N, int H, int d, const int* w, const int* r, int npat, int causal,
+                const void* fwd_workspace, size_t fwd_workspace_bytes,
                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*

@@ -1,5 +1,6 @@
-// Backward kernels: preprocess (D = rowsum(dO * O), zero the fp32
-// accumulators), the tcgen05 key-tile kernel, and the fp32 -> bf16 convert.
+// Backward kernels: preprocess (D = rowsum(dO * O) from the forward's fp32
+// copy of O when given, else from the bf16 O; zero the fp32 accumulators),
+// the tcgen05 key-tile kernel, and the fp32 -> bf16 convert.
 //
 // The merged forward is one softmax over the multiset union of the keys the
 // patterns give a row (LongNet pages: segments, dilation and per-head
@@ -466,6 +467,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
 struct PrepParams {
   int B, N, H;
   const __nv_bfloat16* out;
+  const float* out_f32;  // the forward's fp32 copy of out, or null
   const __nv_bfloat16* dout;
   float* drow;
   float* dq_acc;
@@ -477,9 +479,15 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(PrepParams p) {
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= (long long)p.B * p.N * p.H) return;
-  const __nv_bfloat162 o = reinterpret_cast<const __nv_bfloat162*>(p.out + row * 64)[lane];
   const __nv_bfloat162 d = reinterpret_cast<const __nv_bfloat162*>(p.dout + row * 64)[lane];
-  float acc = __low2float(o) * __low2float(d) + __high2float(o) * __high2float(d);
+  float2 o;
+  if (p.out_f32 != nullptr) {
+    o = reinterpret_cast<const float2*>(p.out_f32 + row * 64)[lane];
+  } else {
+    const __nv_bfloat162 ob = reinterpret_cast<const __nv_bfloat162*>(p.out + row * 64)[lane];
+    o = make_float2(__low2float(ob), __high2float(ob));
+  }
+  float acc = o.x * __low2float(d) + o.y * __high2float(d);
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
   const float2 z = make_float2(0.f, 0.f);

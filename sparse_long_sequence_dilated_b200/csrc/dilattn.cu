@@ -275,6 +275,12 @@ long long make_schedule(const PatternGeom* pat, int npat, int B, int H, Sched& s
   return sc.start[sc.nband];
 }
 
+// The fp32 copy of out inside a forward workspace of `rows` partial rows.
+float* fwd_out_f32(void* ws, long long rows, int d) {
+  return reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align256((size_t)rows * d * 4) +
+                                  align256((size_t)rows * 4));
+}
+
 template <int D>
 int launch_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N,
                int H, const int* w, const int* r, int npat, int causal, void* ws,
@@ -326,6 +332,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   mp.part_o = p.part_o;
   mp.part_lse = p.part_lse;
   mp.out = reinterpret_cast<__nv_bfloat16*>(out);
+  mp.out_f32 = fwd_out_f32(ws, rows, D);
   mp.lse = lse;
   const long long total_rows = (long long)B * N * H;
   const long long blocks = (total_rows + 31) / 32;
@@ -337,8 +344,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
 
 int launch_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                const void* dout, void* dq, void* dk, void* dv, int B, int N, int H,
-               const int* w, const int* r, int npat, int causal, void* ws, DeviceState* st,
-               cudaStream_t stream) {
+               const int* w, const int* r, int npat, int causal, const float* out_f32, void* ws,
+               DeviceState* st, cudaStream_t stream) {
   constexpr int D = 64;
   static_assert(sizeof(BwdParams) < 32000, "kernel parameter block too large");
   BwdParams p;
@@ -384,6 +391,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   pp.N = N;
   pp.H = H;
   pp.out = reinterpret_cast<const __nv_bfloat16*>(out);
+  pp.out_f32 = out_f32;
   pp.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
   pp.drow = drow;
   pp.dq_acc = dq_acc;
@@ -450,7 +458,8 @@ size_t dilattn_fwd_workspace_size(int B, int N, int H, int d, const int* w, cons
   if (check_shape(B, N, H, d, w, r, npat, 1) != DILATTN_OK) return 0;
   PatternGeom geo[kMaxPat];
   const long long rows = make_geoms(B, N, H, w, r, npat, geo);
-  return align256((size_t)rows * d * 4) + align256((size_t)rows * 4);
+  return align256((size_t)rows * d * 4) + align256((size_t)rows * 4) +
+         align256((size_t)B * N * H * d * 4);
 }
 
 int dilattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N,
@@ -492,8 +501,9 @@ size_t dilattn_bwd_workspace_size(int B, int N, int H, int d, const int* w, cons
 
 int dilattn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
                 const void* dout, void* dq, void* dk, void* dv, int B, int N, int H, int d,
-                const int* w, const int* r, int npat, int causal, void* workspace,
-                size_t workspace_bytes, cudaStream_t stream) {
+                const int* w, const int* r, int npat, int causal, const void* fwd_workspace,
+                size_t fwd_workspace_bytes, void* workspace, size_t workspace_bytes,
+                cudaStream_t stream) {
   int rc = check_shape(B, N, H, d, w, r, npat, causal);
   if (rc != DILATTN_OK) return rc;
   const void* ins[6] = {q, k, v, out, lse, dout};
@@ -519,8 +529,19 @@ int dilattn_bwd(const void* q, const void* k, const void* v, const void* out, co
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != DILATTN_OK) return rc;
-  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, N, H, w, r, npat, causal, workspace,
-                    st, stream);
+  const float* out_f32 = nullptr;
+  if (fwd_workspace != nullptr) {
+    if ((reinterpret_cast<uintptr_t>(fwd_workspace) & 255) != 0 ||
+        fwd_workspace_bytes < dilattn_fwd_workspace_size(B, N, H, d, w, r, npat))
+      return DILATTN_ERR_WORKSPACE;
+    PatternGeom geo[kMaxPat];
+    const long long rows = make_geoms(B, N, H, w, r, npat, geo);
+    out_f32 = fwd_out_f32(const_cast<void*>(fwd_workspace), rows, d);
+    if (overlaps(fwd_workspace, fwd_workspace_bytes, workspace, workspace_bytes))
+      return DILATTN_ERR_INVALID_ARG;
+  }
+  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, N, H, w, r, npat, causal, out_f32,
+                    workspace, st, stream);
 }
 
 int dilattn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse, int B,

@@ -46,7 +46,8 @@ struct MergeParams {
   const float* part_o;
   const float* part_lse;
   __nv_bfloat16* out;
-  float* lse;  // may be null
+  float* out_f32;  // fp32 copy of out (for the backward's D)
+  float* lse;      // may be null
 };
 
 // 8 threads per output row, each owning D/8 consecutive columns; 32 rows per
@@ -103,6 +104,10 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
     for (int e = 0; e < PER; ++e) acc[e] *= inv;
     L = m + logf(l);
   }
+  float4* dst32 = reinterpret_cast<float4*>(p.out_f32 + row * D + sub * PER);
+#pragma unroll
+  for (int e = 0; e < PER / 4; ++e)
+    dst32[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
   uint32_t pk[PER / 2];
 #pragma unroll
   for (int e = 0; e < PER / 2; ++e) pk[e] = pack_bf16(acc[2 * e], acc[2 * e + 1]);

@@ -34,7 +34,7 @@ SIGNATURES = {
     "dilattn_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
     "dilattn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _ip, _ip, _i]),
     "dilattn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i,
-                         _i, _vp, _sz, _vp]),
+                         _i, _vp, _sz, _vp, _sz, _vp]),
     "dilattn_fwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
     "dilattn_bwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip,
                              _i, _i, _vp]),
@@ -165,8 +165,12 @@ def fwd(q, k, v, patterns, causal: bool = True, out=None, lse=None, workspace=No
 
 
 def bwd(q, k, v, out, lse, dout, patterns, causal: bool = True, dq=None, dk=None, dv=None,
-        workspace=None, stream=None):
-    """Gradients (dq, dk, dv) of sum(out * dout) for the forward that produced out, lse."""
+        workspace=None, stream=None, fwd_workspace=None):
+    """Gradients (dq, dk, dv) of sum(out * dout) for the forward that produced out, lse.
+
+    ``fwd_workspace``: the workspace tensor of that forward call (bf16 only),
+    so the backward can take D = rowsum(dout * out) from the forward's fp32
+    copy of out; None uses the bf16 out."""
     torch = _torch()
     B, N, H, d = _shape(q)
     for t in (k, v, out, dout):
@@ -182,9 +186,11 @@ def bwd(q, k, v, out, lse, dout, patterns, causal: bool = True, dq=None, dk=None
         need = int(lib.dilattn_bwd_workspace_size(B, N, H, d, w, r, n))
         if workspace is None:
             workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+        fptr = fwd_workspace.data_ptr() if fwd_workspace is not None else None
+        fbytes = fwd_workspace.numel() * fwd_workspace.element_size() if fwd_workspace is not None else 0
         rc = lib.dilattn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                              lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                             dv.data_ptr(), B, N, H, d, w, r, n, int(causal),
+                             dv.data_ptr(), B, N, H, d, w, r, n, int(causal), fptr, fbytes,
                              workspace.data_ptr(), workspace.numel() * workspace.element_size(), s)
         _check(rc, "dilattn_bwd")
     elif q.dtype == torch.float32:

@@ -54,8 +54,13 @@ struct BwdParams {
   int* err;
 };
 
+#ifndef DILATTN_BWD_SPLIT_DS
+#define DILATTN_BWD_SPLIT_DS 1
+#endif
+
 struct BwdCfg {
   static constexpr int D = 64;
+  static constexpr bool SPLIT_DS = DILATTN_BWD_SPLIT_DS != 0;  // dS as bf16 hi + lo
   static constexpr int NCG = 2;                    // column groups of the row warps
   static constexpr int CPT = 4 / NCG;              // 32-column chunks per row thread
   static constexpr int ROW_WARPS = 4 * NCG;
@@ -261,7 +266,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           const uint64_t bq = sw128_desc(sQ + s * C::TILE + kk * 2048, C::TILE, 1024);
           const uint32_t a_ds = tmem + C::TM_DP + (kk >> 1) * 32 + (kk & 1) * 8;
           mma_ts(tmem + C::TM_DK, a_ds, bq, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tmem + C::TM_DK, a_ds + 16, bq, kIdKV, 1u);
+          if (C::SPLIT_DS) mma_ts(tmem + C::TM_DK, a_ds + 16, bq, kIdKV, 1u);
         }
         mma_commit(b_kv2);
 #pragma unroll
@@ -270,7 +275,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           const uint64_t al = sw128_desc(sDSL + kk * 2048, C::TILE, 1024);
           const uint64_t b = sw128_desc(sK + kk * 2048, C::TILE, 1024);
           mma_ss(tmem + C::TM_DQ, a, b, kIdQ, kk > 0 ? 1u : 0u);
-          mma_ss(tmem + C::TM_DQ, al, b, kIdQ, 1u);
+          if (C::SPLIT_DS) mma_ss(tmem + C::TM_DQ, al, b, kIdQ, 1u);
         }
         mma_commit(b_qempty(s));
         mma_commit(b_dq);

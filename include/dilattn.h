@@ -123,8 +123,10 @@ int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, 
  * Backward of dilattn_fwd: given out and lse from the forward and the
  * output gradient dout (all device), writes dq, dk, dv [B][N][H][d] bf16, the
  * full derivative of sum(out * dout). The probabilities are recomputed from
- * the saved lse. Workspace: fp32 accumulators for dq, dk, dv and the row
- * term D = rowsum(dout * out), at least dilattn_bwd_workspace_size(...) bytes.
+ * the saved lse. Workspace: fp32 accumulators for dq, dk, dv, the row term
+ * D = rowsum(dout * out) and the key-tile kernel's work counter, at least
+ * dilattn_bwd_workspace_size(...) bytes. Calls that share a workspace must
+ * not overlap on the GPU.
  *
  * fwd_workspace: the workspace of the dilattn_fwd call that produced out and
  * lse, untouched since (fwd_workspace_bytes >= dilattn_fwd_workspace_size).

@@ -10,30 +10,47 @@
 // ordinary attention-backward terms with P = exp(tau S - L), and the
 // contributions of different patterns simply add up.
 //
-// Key-tile kernel: one CTA per (pattern, segment, batch, head, key tile u),
-// looping over the segment's query tiles t (t >= u when causal). Per pair:
-//   S^T  = K Q^T,  dP^T = V dO^T                     (SMEM x SMEM -> TMEM)
-//   P^T  = exp2(S^T tau log2e - L log2e), dS^T = P^T (dP^T - D)   (threads)
-//   dV  += P^T dO,  dK += dS^T Q                     (TMEM x SMEM -> TMEM)
-//   dQ   = dS K                                      (SMEM x SMEM -> TMEM)
-// P and dS enter their products as two bf16 halves each, hi + lo, so the
-// products are fp32-grade: the gradients' own bf16 rounding (half an ulp is
-// 0.0078 at |g| in [2, 4)) leaves no room for a 2^-9 rounding of P or dS under
-// a 2e-2 bound.
-// dQ is staged in shared memory after every pair and added to an fp32
-// accumulator by a TMA reduce-add; dK, dV are added the same way once at the
-// end (other patterns and tiles reach the same rows). The three accumulators
-// form one [3B][N][H][64] fp32 tensor read through the same strided views.
+// Key-tile kernel. A unit is (pattern, segment, batch, head, key tile u); it
+// loops over the segment's query tiles t (t >= u when causal). The grid is
+// persistent, one CTA per SM; CTAs take units from a global counter in
+// group-major order: patterns with the most tiles first, then (segment,
+// batch, head) groups, then u ascending, so the key tiles of one group run at
+// the same time on different SMs and share its Q, dO tiles and dq rows in L2.
+// Each query tile is handled as two halves h of 64
+// queries so that the tensor pipe and the row threads overlap:
+//   S^T_h  = K Q_h^T,  dP^T_h = V dO_h^T                   (SMEM x SMEM -> TMEM)
+//   P^T_h  = exp2(S^T_h tau log2e - L log2e), dS^T_h = P^T_h (dP^T_h - D)  (threads)
+//   dV += P^T_h dO_h,  dK += dS^T_h Q_h                    (TMEM x SMEM -> TMEM)
+//   dQ  = dS K  (both halves; dS from SMEM)                (SMEM x SMEM -> TMEM)
+// MMA issue order per pair i: dVdK_0(i), SdP_0(i+1), dVdK_1(i), dQ(i),
+// SdP_1(i+1); the row threads work on half 1 of pair i while dVdK_0(i) and
+// SdP_0(i+1) run, and on half 0 of pair i+1 while dVdK_1(i), dQ(i) and
+// SdP_1(i+1) run. An S / dP half is overwritten only by MMAs issued after
+// the MMAs that read its P / dS, and tcgen05 MMAs of one thread execute in
+// issue order.
+// P and dS enter the products as bf16. On the first query tile of a segment
+// (rows with few keys, where single probabilities approach 1) P enters dV and
+// dS enters dK as two bf16 halves, hi + lo, so those products are fp32-grade:
+// the gradients' own bf16 rounding (half an ulp is 0.0156 at |g| in [4, 8))
+// leaves little room for a 2^-9 rounding of a large P under a 2e-2 bound.
+// Elsewhere a row spreads its weight over at least 129 keys, and the
+// rounding of P and dS averages out far inside the bound.
+// dQ goes through a double-buffered TMEM accumulator; after each pair every
+// row warp stages its 32 x 32 block in a private shared-memory slab and adds
+// it to the fp32 accumulator with a TMA reduce-add. dK, dV are added the same
+// way once per unit (other patterns and tiles reach the same rows). The three
+// accumulators form one [3B][N][H][64] fp32 tensor read through the same
+// strided views as the inputs.
 //
-// Warp roles (64 + 128 NCG threads): warp 0 TMA producer (+ per-tile L and D
-// rows), warp 1 TMEM allocator and MMA issuer, warps 2.. the row work: warp w
-// serves TMEM lanes 32 (w % 4) .. + 31 and column group (w - 2) / 4, i.e. the
-// CPT = 4 / NCG consecutive 32-column chunks of that group.
-// TMEM columns: S^T / P^T [0,128), dP^T / dS^T [128,256), dV [256,320),
-// dK [320,384), dQ [384,448). P^T and dS^T (hi, lo) overwrite S^T and dP^T in
-// place, each 32-column quarter by the warps that read it: query columns
-// [32q, 32q + 32) keep P^T hi at TM_S + 32q + [0, 16), lo at TM_S + 32q + [16, 32),
-// and dS^T hi / lo at TM_DP + 32q + [0, 16) / [16, 32).
+// Warp roles (320 threads): warp 0 TMA producer (+ per-tile L and D rows and
+// an L2 prefetch of the next unit's key tile), warp 1 TMEM allocator and MMA
+// issuer, warps 2..9 the row work: warp w serves TMEM lanes 32 (w % 4) .. + 31
+// (key rows) and column group cg = (w - 2) / 4, i.e. 32-column chunk 2h + cg
+// of half h.
+// TMEM columns: S^T [0,128) (half h at 64h), dP^T [128,256), dV [256,320),
+// dK [320,384), dQ two buffers [384,448), [448,512). P^T and dS^T (hi, lo)
+// overwrite S^T and dP^T in place: chunk q = [32q, 32q + 32) keeps hi at
+// +[0,16) and lo at +[16,32).
 #pragma once
 
 #include "common.cuh"
@@ -43,60 +60,150 @@ namespace dil {
 struct BwdParams {
   CUtensorMap tmq[kMaxPat], tmk[kMaxPat], tmv[kMaxPat], tmdo[kMaxPat];
   CUtensorMap tmq_t[kMaxPat], tmk_t[kMaxPat], tmv_t[kMaxPat], tmdo_t[kMaxPat];
+  CUtensorMap tmacc[kMaxPat], tmacc_t[kMaxPat];  // fp32 [3B][N][H][64]: dq, dk, dv; 32 x 32 boxes
   PatternGeom pat[kMaxPat];
   int npat, B, N, H, causal;
   float scale_log2;  // log2(e) / sqrt(d)
   float tau;         // 1 / sqrt(d)
-  Sched sched;
-  CUtensorMap tmacc[kMaxPat], tmacc_t[kMaxPat];  // fp32 [3B][N][H][64]: dq, dk, dv
+  int gorder[kMaxPat];           // patterns by tile count, descending
+  long long gstart[kMaxPat + 1];  // first unit of each pattern in that order
+  long long units;
+  int* counter;                   // next unit to hand out (zeroed by the preprocess)
   const float* lse;   // [B][H][N] natural log
   const float* drow;  // [B][H][N]
   int* err;
 };
 
-#ifndef DILATTN_BWD_SPLIT_DS
-#define DILATTN_BWD_SPLIT_DS 1
+// hi + lo products: 0 never, 1 on the first query tile of a segment, 2 always
+#ifndef DILATTN_BWD_SPLIT
+#define DILATTN_BWD_SPLIT 1
 #endif
 
 struct BwdCfg {
   static constexpr int D = 64;
-  static constexpr bool SPLIT_DS = DILATTN_BWD_SPLIT_DS != 0;  // dS as bf16 hi + lo
-  static constexpr int NCG = 2;                    // column groups of the row warps
-  static constexpr int CPT = 4 / NCG;              // 32-column chunks per row thread
-  static constexpr int ROW_WARPS = 4 * NCG;
+  static constexpr int SPLIT = DILATTN_BWD_SPLIT;
+  __host__ __device__ static constexpr bool split(int t) { return SPLIT == 2 || (SPLIT == 1 && t == 0); }
+  static constexpr int ROW_WARPS = 8;
   static constexpr int THREADS = 64 + 32 * ROW_WARPS;
-  static constexpr int STAGES = 2;
-  static constexpr int TILE = BM * 128;  // 128 rows x 64 bf16
+  static constexpr int TILE = BM * 128;   // 128 rows x 64 bf16
+  static constexpr int HALF = TILE / 2;   // 64 rows
+  static constexpr int SLAB = 32 * 128;   // one row warp's 32 x 32 fp32 staging block
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_Q = OFF_V + TILE;                 // STAGES tiles
-  static constexpr int OFF_DO = OFF_Q + STAGES * TILE;       // STAGES tiles
-  static constexpr int OFF_DS = OFF_DO + STAGES * TILE;      // dS hi: 2 chunks of [128 kv][64 q]
-  static constexpr int OFF_DSL = OFF_DS + 2 * TILE;          // dS lo, same layout
-  static constexpr int OFF_STG = OFF_DSL + 2 * TILE;         // fp32 [2][128][32] staging
-  static constexpr int STG_BYTES = 2 * BM * 128;             // one 128 x 64 fp32 tile
-  static constexpr int OFF_L = OFF_STG + STG_BYTES;          // STAGES x 128 floats
-  static constexpr int OFF_D = OFF_L + STAGES * BM * 4;      // STAGES x 128 floats
-  static constexpr int OFF_BAR = OFF_D + STAGES * BM * 4;
+  static constexpr int OFF_Q = OFF_V + TILE;                  // 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;             // 2 stages
+  static constexpr int OFF_DS = OFF_DO + 2 * TILE;            // 2 buffers x 2 halves x [128 keys][64 q]
+  static constexpr int OFF_STG = OFF_DS + 4 * TILE;           // ROW_WARPS slabs
+  static constexpr int OFF_L = OFF_STG + ROW_WARPS * SLAB;    // 2 stages x 128 floats
+  static constexpr int OFF_D = OFF_L + 2 * BM * 4;            // 2 stages x 128 floats
+  static constexpr int OFF_BAR = OFF_D + 2 * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
   static constexpr int TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 320, TM_DQ = 384;
   static constexpr int TMEM_COLS = 512;
 };
+static_assert(BwdCfg::SMEM_BYTES <= 232448, "backward tile kernel exceeds shared memory");
 
-// Thread `row` writes 16 fp32 = 16-byte pieces [piece0, piece0 + 4) of one
-// 128-byte row of a [128][32] fp32 chunk with 128-byte swizzle (piece k lands
-// at k ^ (row % 8)), scaled by `scale`.
-__device__ __forceinline__ void stage_row16(uint8_t* chunk, int row, int piece0,
-                                            const uint32_t (&r)[16], float scale) {
-  uint8_t* rowp = chunk + row * 128;
+// Row `row` of a [32][32] fp32 slab with 128-byte swizzle (16-byte piece k of
+// the row lands at k ^ (row % 8)), scaled by `scale`.
+__device__ __forceinline__ void stage_row32(uint8_t* slab, int row, const uint32_t (&r)[32],
+                                            float scale) {
+  uint8_t* rowp = slab + row * 128;
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < 8; ++k) {
     const float4 v = make_float4(__uint_as_float(r[4 * k]) * scale,
                                  __uint_as_float(r[4 * k + 1]) * scale,
                                  __uint_as_float(r[4 * k + 2]) * scale,
                                  __uint_as_float(r[4 * k + 3]) * scale);
-    *reinterpret_cast<float4*>(rowp + (((piece0 + k) ^ (row & 7)) * 16)) = v;
+    *reinterpret_cast<float4*>(rowp + ((k ^ (row & 7)) * 16)) = v;
   }
+}
+
+// P^T and dS^T of queries [E0, E0 + NE) of a 32-query chunk of key row c:
+// P = exp2(S tau log2e - L) (zero for e < jmin), dS = P (dP - D), packed to
+// bf16 pairs at index (e - E0) / 2; with SPLIT also the bf16 remainders
+// lo = x - hi.
+template <bool SPLIT, int E0, int NE>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32_t (&dv)[32],
+                                          const float* sLq, const float* sDq, float sc, int jmin,
+                                          uint32_t* pk, uint32_t* plo, uint32_t* dk, uint32_t* dkl) {
+  const float4* L4 = reinterpret_cast<const float4*>(sLq);
+  const float4* D4 = reinterpret_cast<const float4*>(sDq);
+  const bool masked = jmin > 0;
+  const uint64_t sc2 = f2_pack(sc, sc);
+#pragma unroll
+  for (int e4 = E0 / 4; e4 < (E0 + NE) / 4; ++e4) {
+    const float4 Lq = L4[e4], Dq = D4[e4];
+    const uint64_t nl2[2] = {f2_pack(-Lq.x, -Lq.y), f2_pack(-Lq.z, -Lq.w)};
+    const uint64_t dd2[2] = {f2_pack(Dq.x, Dq.y), f2_pack(Dq.z, Dq.w)};
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int e = 4 * e4 + 2 * h2;
+      const int o = (e - E0) / 2;
+      const uint64_t x2 =
+          f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])), sc2, nl2[h2]);
+      float p0 = ex2(f2_lo(x2)), p1 = ex2(f2_hi(x2));
+      if (masked) {
+        p0 = e >= jmin ? p0 : 0.f;
+        p1 = e + 1 >= jmin ? p1 : 0.f;
+      }
+      const uint64_t p2 = f2_pack(p0, p1);
+      const uint64_t ds2 = f2_mul(
+          p2, f2_sub(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), dd2[h2]));
+      const uint32_t hi = pack_bf16_rn(p0, p1);
+      const uint32_t dhi = pack_bf16_rn(f2_lo(ds2), f2_hi(ds2));
+      pk[o] = hi;
+      dk[o] = dhi;
+      if (SPLIT) {
+        const uint64_t lo2 =
+            f2_sub(p2, f2_pack(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)));
+        plo[o] = pack_bf16_rn(f2_lo(lo2), f2_hi(lo2));
+        const uint64_t dlo2 =
+            f2_sub(ds2, f2_pack(__uint_as_float(dhi << 16), __uint_as_float(dhi & 0xffff0000u)));
+        dkl[o] = pack_bf16_rn(f2_lo(dlo2), f2_hi(dlo2));
+      }
+    }
+  }
+}
+
+// One backward unit: (pattern, segment, batch, head, key tile u) and the
+// views its tiles are read through. False when the key tile holds no row.
+struct BwdUnit {
+  TileUnit wu;
+  PatternGeom g;
+  SegInfo si;
+  int u, t0, np;
+  const CUtensorMap *mq, *mk, *mv, *mdo, *macc;
+};
+
+__device__ __forceinline__ bool bwd_unit(const BwdParams& p, long long uu, BwdUnit& U) {
+  int a = 0;
+  while (a + 1 < p.npat && uu >= p.gstart[a + 1]) ++a;
+  const int i = p.gorder[a];
+  long long rem = uu - p.gstart[a];
+  U.g = p.pat[i];
+  U.u = (int)(rem % U.g.ntiles);  // key tile; long (small u) tiles come first
+  rem /= U.g.ntiles;
+  U.wu.pat = i;
+  U.wu.t = U.u;
+  U.wu.h = (int)(rem % p.H);
+  rem /= p.H;
+  U.wu.b = (int)(rem % p.B);
+  U.wu.seg = (int)(rem / p.B);
+  U.si = seg_info(U.g, p.N, U.wu.h, U.wu.seg);
+  const int nq = (U.si.n + BM - 1) / BM;
+  if (U.u >= nq) return false;
+  U.t0 = p.causal ? U.u : 0;
+  U.np = nq - U.t0;
+  // all tiles of a (pattern, segment, head) share one phase, hence one view
+  int ph0, m0;
+  view_coords(U.g, U.si, 0, ph0, m0);
+  const bool tv = ph0 < U.g.nmod;
+  U.mq = tv ? &p.tmq_t[i] : &p.tmq[i];
+  U.mk = tv ? &p.tmk_t[i] : &p.tmk[i];
+  U.mv = tv ? &p.tmv_t[i] : &p.tmv[i];
+  U.mdo = tv ? &p.tmdo_t[i] : &p.tmdo[i];
+  U.macc = tv ? &p.tmacc_t[i] : &p.tmacc[i];
+  return true;
 }
 
 __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __grid_constant__ BwdParams p) {
@@ -107,65 +214,46 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   const uint32_t base = (raw_s + 1023u) & ~1023u;
   uint8_t* base_g = smem_raw + (base - raw_s);
 
-  const TileUnit wu = decode_unit(p.sched, p.pat, p.B, p.H, blockIdx.x);
-  const PatternGeom g = p.pat[wu.pat];
-  const SegInfo si = seg_info(g, p.N, wu.h, wu.seg);
-  const int nq = (si.n + BM - 1) / BM;
-  const int u = g.ntiles - 1 - wu.t;  // key tile; long (small u) tiles come first
-  if (u >= nq) return;                // uniform exit: no key rows here
-  const int t0 = p.causal ? u : 0;
-  const int npairs = nq - t0;
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
   const uint32_t sQ = base + C::OFF_Q, sDO = base + C::OFF_DO, sDS = base + C::OFF_DS;
-  const uint32_t sDSL = base + C::OFF_DSL;
   float* sL = reinterpret_cast<float*>(base_g + C::OFF_L);
   float* sD = reinterpret_cast<float*>(base_g + C::OFF_D);
   const uint32_t bars = base + C::OFF_BAR;
-  const uint32_t b_kvfull = bars;
-  auto b_qfull = [&](int s) { return bars + 8u + 8u * s; };
-  auto b_qempty = [&](int s) { return bars + 8u + 8u * C::STAGES + 8u * s; };
-  const uint32_t b_sdp = bars + 8u + 16u * C::STAGES;
-  const uint32_t b_ds = b_sdp + 8u;
-  const uint32_t b_dq = b_sdp + 16u;
-  const uint32_t b_kv2 = b_sdp + 24u;
-  const uint32_t b_grp = b_sdp + 32u;  // sync point of the row warps (bounded, unlike bar.sync)
-  const uint32_t sSTG = base + C::OFF_STG;
+  const uint32_t b_kvfull = bars;         // K, V of the unit landed
+  const uint32_t b_kvempty = bars + 8u;   // every MMA of the unit is complete
+  auto b_qfull = [&](int s) { return bars + 16u + 8u * s; };    // Q, dO, L, D of stage s
+  auto b_qempty = [&](int s) { return bars + 32u + 8u * s; };
+  auto b_sdp = [&](int h) { return bars + 48u + 8u * h; };      // S^T_h, dP^T_h in TMEM
+  auto b_rows = [&](int h) { return bars + 64u + 8u * h; };     // P^T_h, dS^T_h written
+  auto b_dq = [&](int j) { return bars + 80u + 8u * j; };       // dQ buffer j complete
+  auto b_dqfree = [&](int j) { return bars + 96u + 8u * j; };   // dQ buffer j read out
+  const uint32_t b_accfree = bars + 112u;  // dV, dK of the unit read out
+  const uint32_t b_fin = bars + 120u;      // MMA pipe drained at exit
+  auto b_unit = [&](int j) { return bars + 128u + 8u * j; };    // unit index published in slot j
+  volatile int* uslot = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 232);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
 
-  int phase0, m0;
-  view_coords(g, si, 0, phase0, m0);
-  const bool tail_view = phase0 < g.nmod;
-  const CUtensorMap* mq = tail_view ? &p.tmq_t[wu.pat] : &p.tmq[wu.pat];
-  const CUtensorMap* mk = tail_view ? &p.tmk_t[wu.pat] : &p.tmk[wu.pat];
-  const CUtensorMap* mv = tail_view ? &p.tmv_t[wu.pat] : &p.tmv[wu.pat];
-  const CUtensorMap* mdo = tail_view ? &p.tmdo_t[wu.pat] : &p.tmdo[wu.pat];
-  const CUtensorMap* macc = tail_view ? &p.tmacc_t[wu.pat] : &p.tmacc[wu.pat];
-
   if (threadIdx.x == 0) {
     mbar_init(b_kvfull, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
+    mbar_init(b_kvempty, 1);
+    for (int s = 0; s < 2; ++s) {
       mbar_init(b_qfull(s), 1);
       mbar_init(b_qempty(s), 1);
+      mbar_init(b_sdp(s), 1);
+      mbar_init(b_rows(s), C::ROW_WARPS);
+      mbar_init(b_dq(s), 1);
+      mbar_init(b_dqfree(s), C::ROW_WARPS);
     }
-    mbar_init(b_sdp, 1);
-    mbar_init(b_ds, C::ROW_WARPS);
-    mbar_init(b_dq, 1);
-    mbar_init(b_kv2, 1);
-    mbar_init(b_grp, C::ROW_WARPS);
+    mbar_init(b_accfree, C::ROW_WARPS);
+    mbar_init(b_fin, 1);
+    mbar_init(b_unit(0), 1);
+    mbar_init(b_unit(1), 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
-  }
-  if (warp == 0 && lane == 0) {
-    prefetch_tmap(mq);
-    prefetch_tmap(mk);
-    prefetch_tmap(mv);
-    prefetch_tmap(mdo);
-    prefetch_tmap(macc);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -175,292 +263,404 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
-  const long long lrow0 = ((long long)wu.b * p.H + wu.h) * p.N;  // lse / D row base
   const float log2e = 1.4426950408889634f;
+  // The producer takes units from the global counter one ahead of use and
+  // publishes each in slot k & 1 (phase k >> 1); p.units marks the end.
+  // Slot k & 1 is rewritten only after the MMAs of unit k - 1 completed, by
+  // which time every role has read it.
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    int ph, m;
+    uint32_t gp = 0, k = 0;  // pairs and units issued so far
+    bool ok = true;
+    // next unit with key rows, or p.units when none is left (lane 0)
+    auto fetch = [&]() -> long long {
+      for (;;) {
+        const long long x = atomicAdd(p.counter, 1);
+        BwdUnit t;
+        if (x >= p.units) return p.units;
+        if (bwd_unit(p, x, t)) return x;
+      }
+    };
+    long long cur = 0;
     if (lane == 0) {
-      view_coords(g, si, u * BN, ph, m);
-      mbar_arrive_expect_tx(b_kvfull, 2 * C::TILE);
-      tma_load_5d(sK, mk, b_kvfull, 0, wu.h, ph, m, wu.b);
-      tma_load_5d(sV, mv, b_kvfull, 0, wu.h, ph, m, wu.b);
+      cur = fetch();
+      uslot[0] = (int)cur;
+      mbar_arrive(b_unit(0));
     }
-    int issued = 0;
-    for (int it = 0; it < npairs; ++it) {
-      const int s = it % C::STAGES;
-      const int t = t0 + it;
-      if (!warp_wait(b_qempty(s), ((it / C::STAGES) & 1) ^ 1, abort_flag, p.err)) break;
-      // merged lse (log2 units) and D for the tile's query rows; rows past the
-      // segment get L = +inf, so their probabilities are exactly zero
-#pragma unroll
-      for (int jj = 0; jj < BM / 32; ++jj) {
-        const int j = lane + 32 * jj;
-        const int vq = t * BM + j;
-        float L = INFINITY, Dv = 0.f;
-        if (vq < si.n) {
-          const long long pos = si.start + si.off + (long long)vq * g.r;
-          L = p.lse[lrow0 + pos] * log2e;
-          Dv = p.drow[lrow0 + pos];
-        }
-        sL[s * BM + j] = L;
-        sD[s * BM + j] = Dv;
+    cur = __shfl_sync(0xffffffffu, cur, 0);
+    while (cur < p.units) {
+      BwdUnit U;
+      bwd_unit(p, cur, U);
+      if (k > 0 && !warp_wait(b_kvempty, (k - 1) & 1, abort_flag, p.err)) {
+        ok = false;
+        break;
       }
-      __syncwarp();
+      long long nxt = 0;
       if (lane == 0) {
-        view_coords(g, si, t * BM, ph, m);
-        mbar_arrive_expect_tx(b_qfull(s), 2 * C::TILE);
-        tma_load_5d(sQ + s * C::TILE, mq, b_qfull(s), 0, wu.h, ph, m, wu.b);
-        tma_load_5d(sDO + s * C::TILE, mdo, b_qfull(s), 0, wu.h, ph, m, wu.b);
+        nxt = fetch();
+        uslot[(k + 1) & 1] = (int)nxt;
+        mbar_arrive(b_unit((k + 1) & 1));
+        int ph, m;
+        view_coords(U.g, U.si, U.u * BN, ph, m);
+        mbar_arrive_expect_tx(b_kvfull, 2 * C::TILE);
+        tma_load_5d(sK, U.mk, b_kvfull, 0, U.wu.h, ph, m, U.wu.b);
+        tma_load_5d(sV, U.mv, b_kvfull, 0, U.wu.h, ph, m, U.wu.b);
+        BwdUnit nx;
+        if (nxt < p.units && bwd_unit(p, nxt, nx)) {  // warm the L2 for the next unit
+          view_coords(nx.g, nx.si, nx.u * BN, ph, m);
+          tma_prefetch_l2_5d(nx.mk, 0, nx.wu.h, ph, m, nx.wu.b);
+          tma_prefetch_l2_5d(nx.mv, 0, nx.wu.h, ph, m, nx.wu.b);
+          view_coords(nx.g, nx.si, nx.t0 * BM, ph, m);
+          tma_prefetch_l2_5d(nx.mq, 0, nx.wu.h, ph, m, nx.wu.b);
+          tma_prefetch_l2_5d(nx.mdo, 0, nx.wu.h, ph, m, nx.wu.b);
+        }
       }
-      ++issued;
+      nxt = __shfl_sync(0xffffffffu, nxt, 0);
+      ++k;
+      const long long lrow0 = ((long long)U.wu.b * p.H + U.wu.h) * p.N;  // lse / D row base
+      // merged lse (log2 units) and D of query tile t, lane j holding rows
+      // j + 32 jj; rows past the segment get L = +inf, so their probabilities
+      // are exactly zero. Loaded one pair ahead, so the gather overlaps the wait.
+      float Lr[BM / 32], Dr[BM / 32];
+      auto load_ld = [&](int t) {
+#pragma unroll
+        for (int jj = 0; jj < BM / 32; ++jj) {
+          const int vq = t * BM + lane + 32 * jj;
+          Lr[jj] = INFINITY;
+          Dr[jj] = 0.f;
+          if (vq < U.si.n) {
+            const long long pos = U.si.start + U.si.off + (long long)vq * U.g.r;
+            Lr[jj] = p.lse[lrow0 + pos] * log2e;
+            Dr[jj] = p.drow[lrow0 + pos];
+          }
+        }
+      };
+      load_ld(U.t0);
+      for (int it = 0; it < U.np; ++it, ++gp) {
+        const int s = gp & 1;
+        const int t = U.t0 + it;
+        if (!warp_wait(b_qempty(s), ((gp >> 1) & 1) ^ 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) {
+          int ph, m;
+          view_coords(U.g, U.si, t * BM, ph, m);
+          mbar_expect_tx(b_qfull(s), 2 * C::TILE);
+          tma_load_5d(sQ + s * C::TILE, U.mq, b_qfull(s), 0, U.wu.h, ph, m, U.wu.b);
+          tma_load_5d(sDO + s * C::TILE, U.mdo, b_qfull(s), 0, U.wu.h, ph, m, U.wu.b);
+          if (it + 2 < U.np) {  // warm the L2 two pairs ahead
+            view_coords(U.g, U.si, (t + 2) * BM, ph, m);
+            tma_prefetch_l2_5d(U.mq, 0, U.wu.h, ph, m, U.wu.b);
+            tma_prefetch_l2_5d(U.mdo, 0, U.wu.h, ph, m, U.wu.b);
+          }
+        }
+#pragma unroll
+        for (int jj = 0; jj < BM / 32; ++jj) {
+          sL[s * BM + lane + 32 * jj] = Lr[jj];
+          sD[s * BM + lane + 32 * jj] = Dr[jj];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_qfull(s));  // the phase ends once the copies land too
+        if (it + 1 < U.np) load_ld(t + 1);
+      }
+      if (!ok) break;
+      cur = nxt;
     }
-    if (lane == 0 && *abort_flag) {
+    if (!ok && lane == 0) {
+      // Drain copies still in flight before the CTA's shared memory goes away.
       volatile int no_abort = 0;
-      mbar_wait(b_kvfull, 0, &no_abort, nullptr, 200000000ull);
-      for (int it = issued - C::STAGES; it < issued; ++it) {
-        if (it < 0) continue;
-        mbar_wait(b_qfull(it % C::STAGES), (it / C::STAGES) & 1, &no_abort, nullptr, 200000000ull);
-      }
+      if (k > 0) mbar_wait(b_kvfull, (k - 1) & 1, &no_abort, nullptr, 200000000ull);
+      for (uint32_t g = (gp >= 2 ? gp - 2 : 0); g < gp; ++g)
+        mbar_wait(b_qfull(g & 1), (g >> 1) & 1, &no_abort, nullptr, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t kIdS = idesc_bf16(BM, BM, 0, 0);   // K x Q^T, V x dO^T
-      constexpr uint32_t kIdKV = idesc_bf16(BM, D, 0, 1);   // P^T (TMEM) x dO, dS^T (TMEM) x Q
+      constexpr uint32_t kIdSh = idesc_bf16(BM, 64, 0, 0);  // K x Q_h^T, V x dO_h^T
+      constexpr uint32_t kIdKV = idesc_bf16(BM, D, 0, 1);   // P^T / dS^T (TMEM) x dO / Q
       constexpr uint32_t kIdQ = idesc_bf16(BM, D, 1, 1);    // dS (MN-major SMEM) x K
-      bool ok = mbar_wait(b_kvfull, 0, abort_flag, p.err);
-      for (int it = 0; ok && it < npairs; ++it) {
-        const int s = it % C::STAGES;
-        if (!mbar_wait(b_qfull(s), (it / C::STAGES) & 1, abort_flag, p.err)) break;
-        // the dV / dK MMAs of the previous pair (readers of TMEM P^T / dS^T) are
-        // complete; its dQ MMA (SMEM dS, TMEM dQ) may still run
-        if (it > 0 && !mbar_wait(b_kv2, (it - 1) & 1, abort_flag, p.err)) break;
+      // S^T_h = K Q_h^T and dP^T_h = V dO_h^T for the 64 queries of half h
+      auto issue_sdp = [&](uint32_t g, int h) {
+        const uint32_t qo = (g & 1) * C::TILE + h * C::HALF;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::TM_S + h * 64, sw128_desc(sK + kk * 32, 16, 1024),
+                 sw128_desc(sQ + qo + kk * 32, 16, 1024), kIdSh, kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tmem + C::TM_DP + h * 64, sw128_desc(sV + kk * 32, 16, 1024),
+                 sw128_desc(sDO + qo + kk * 32, 16, 1024), kIdSh, kk > 0 ? 1u : 0u);
+        mma_commit(b_sdp(h));
+      };
+      // dV += P^T_h dO_h, dK += dS^T_h Q_h (each hi + lo when `split`); `first`
+      // starts the accumulators
+      auto issue_dvdk = [&](uint32_t g, int h, bool first, bool split) {
+        const uint32_t qo = (g & 1) * C::TILE;
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          const int kk = 4 * h + kq;  // 16 queries
+          const uint64_t bdo = sw128_desc(sDO + qo + kk * 2048, C::TILE, 1024);
+          const uint32_t a = tmem + C::TM_S + (kk >> 1) * 32 + (kk & 1) * 8;
+          mma_ts(tmem + C::TM_DV, a, bdo, kIdKV, (first && kq == 0) ? 0u : 1u);
+          if (split) mma_ts(tmem + C::TM_DV, a + 16, bdo, kIdKV, 1u);
+        }
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          const int kk = 4 * h + kq;
+          const uint64_t bq = sw128_desc(sQ + qo + kk * 2048, C::TILE, 1024);
+          const uint32_t a = tmem + C::TM_DP + (kk >> 1) * 32 + (kk & 1) * 8;
+          mma_ts(tmem + C::TM_DK, a, bq, kIdKV, (first && kq == 0) ? 0u : 1u);
+          if (split) mma_ts(tmem + C::TM_DK, a + 16, bq, kIdKV, 1u);
+        }
+      };
+      // dQ = dS K into TMEM buffer g & 1 (dS from shared-memory buffer g & 1)
+      auto issue_dq = [&](uint32_t g) {
+        const int j = g & 1;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ss(tmem + C::TM_DQ + j * 64, sw128_desc(sDS + j * 2 * C::TILE + kk * 2048, C::TILE, 1024),
+                 sw128_desc(sK + kk * 2048, C::TILE, 1024), kIdQ, kk > 0 ? 1u : 0u);
+        mma_commit(b_dq(j));
+      };
+      uint32_t gp = 0, k = 0;
+      bool ok = true;
+      for (;; ++k) {
+        if (!mbar_wait(b_unit(k & 1), (k >> 1) & 1, abort_flag, p.err)) break;
+        const long long uu = uslot[k & 1];
+        if (uu >= p.units) break;
+        BwdUnit U;
+        bwd_unit(p, uu, U);
+        if (!mbar_wait(b_kvfull, k & 1, abort_flag, p.err) ||
+            !mbar_wait(b_qfull(gp & 1), (gp >> 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sw128_desc(sK + kk * 32, 16, 1024);
-          const uint64_t b = sw128_desc(sQ + s * C::TILE + kk * 32, 16, 1024);
-          mma_ss(tmem + C::TM_S, a, b, kIdS, kk > 0 ? 1u : 0u);
+        issue_sdp(gp, 0);
+        issue_sdp(gp, 1);
+        for (int it = 0; it < U.np; ++it, ++gp) {
+          const bool more = it + 1 < U.np;
+          if (!mbar_wait(b_rows(0), gp & 1, abort_flag, p.err) ||
+              (it == 0 && k > 0 && !mbar_wait(b_accfree, (k - 1) & 1, abort_flag, p.err))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const bool split = C::split(U.t0 + it);
+          issue_dvdk(gp, 0, it == 0, split);
+          // Then, in whichever order their inputs arrive: S / dP half 0 of the
+          // next pair (Q, dO landed) and dV / dK half 1 plus dQ of this pair
+          // (half 1 written, dQ buffer read out). S / dP half 1 of the next
+          // pair goes last: it overwrites what dV / dK half 1 reads.
+          bool need_s0 = more, need_1 = true;
+          PollGuard pg;
+          while (need_s0 || need_1) {
+            bool prog = false;
+            if (need_s0 && mbar_test(b_qfull((gp + 1) & 1), ((gp + 1) >> 1) & 1)) {
+              tc_fence_after();
+              issue_sdp(gp + 1, 0);
+              need_s0 = false;
+              prog = true;
+            }
+            if (need_1 && mbar_test(b_rows(1), gp & 1) &&
+                (gp < 2 || mbar_test(b_dqfree(gp & 1), ((gp >> 1) & 1) ^ 1))) {
+              tc_fence_after();
+              issue_dvdk(gp, 1, false, split);
+              mma_commit(b_qempty(gp & 1));
+              issue_dq(gp);
+              need_1 = false;
+              prog = true;
+            }
+            if (!pg.step(prog, abort_flag, p.err)) {
+              ok = false;
+              break;
+            }
+          }
+          if (!ok) break;
+          if (more) issue_sdp(gp + 1, 1);
+          else mma_commit(b_kvempty);
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t a = sw128_desc(sV + kk * 32, 16, 1024);
-          const uint64_t b = sw128_desc(sDO + s * C::TILE + kk * 32, 16, 1024);
-          mma_ss(tmem + C::TM_DP, a, b, kIdS, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(b_sdp);
-        if (!mbar_wait(b_ds, it & 1, abort_flag, p.err)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint64_t bdo = sw128_desc(sDO + s * C::TILE + kk * 2048, C::TILE, 1024);
-          const uint32_t a_hi = tmem + C::TM_S + (kk >> 1) * 32 + (kk & 1) * 8;
-          mma_ts(tmem + C::TM_DV, a_hi, bdo, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
-          mma_ts(tmem + C::TM_DV, a_hi + 16, bdo, kIdKV, 1u);
-        }
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk) {
-          const uint64_t bq = sw128_desc(sQ + s * C::TILE + kk * 2048, C::TILE, 1024);
-          const uint32_t a_ds = tmem + C::TM_DP + (kk >> 1) * 32 + (kk & 1) * 8;
-          mma_ts(tmem + C::TM_DK, a_ds, bq, kIdKV, (it > 0 || kk > 0) ? 1u : 0u);
-          if (C::SPLIT_DS) mma_ts(tmem + C::TM_DK, a_ds + 16, bq, kIdKV, 1u);
-        }
-        mma_commit(b_kv2);
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t a = sw128_desc(sDS + kk * 2048, C::TILE, 1024);
-          const uint64_t al = sw128_desc(sDSL + kk * 2048, C::TILE, 1024);
-          const uint64_t b = sw128_desc(sK + kk * 2048, C::TILE, 1024);
-          mma_ss(tmem + C::TM_DQ, a, b, kIdQ, kk > 0 ? 1u : 0u);
-          if (C::SPLIT_DS) mma_ss(tmem + C::TM_DQ, al, b, kIdQ, 1u);
-        }
-        mma_commit(b_qempty(s));
-        mma_commit(b_dq);
+        if (!ok) break;
       }
+      // every MMA issued so far completes before TMEM is released
+      mma_commit(b_fin);
+      volatile int no_abort = 0;
+      mbar_wait(b_fin, 0, &no_abort, nullptr, 200000000ull);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ lanes = rows
-    const int q4 = warp & 3;
-    const int cg = (warp - 2) >> 2;          // column group: chunks [CPT cg, CPT cg + CPT)
-    const int c = q4 * 32 + lane;            // key row of S^T / dP^T / dV / dK, query row of dQ
+    // ------------------------------------------------------------ row warps
+    const int rw = warp - 2;
+    const int q4 = warp & 3;   // TMEM lane quarter
+    const int cg = rw >> 2;    // column group
+    const int c = q4 * 32 + lane;  // key row of S^T / dP^T / dV / dK, query row of dQ
     const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
-    const bool key_valid = u * BN + c < si.n;
+    uint8_t* slab_g = base_g + C::OFF_STG + rw * C::SLAB;
+    const uint32_t slab = base + C::OFF_STG + rw * C::SLAB;
     const float sc = p.scale_log2;
+    uint32_t gp = 0;
     bool ok = true;
-    uint32_t gphase = 0;
-    // all row warps meet here; every wait is bounded
-    auto group_sync = [&]() -> bool {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b_grp);
-      const bool r = warp_wait(b_grp, gphase & 1, abort_flag, p.err);
-      ++gphase;
-      return r;
-    };
-    for (int it = 0; it < npairs; ++it) {
-      const int s = it % C::STAGES;
-      const int t = t0 + it;
-      if (!warp_wait(b_qfull(s), (it / C::STAGES) & 1, abort_flag, p.err) ||
-          !warp_wait(b_sdp, it & 1, abort_flag, p.err)) {
-        ok = false;
-        break;
-      }
+    // dQ of pair g (query tile t): this warp's 32 x 32 block -> slab -> TMA
+    // reduce-add into the fp32 dq accumulator. Rows past the segment hold
+    // exact zeros (their P is 0); rows past N are clipped by the view.
+    auto dq_out = [&](const BwdUnit& U, uint32_t g, int t) -> bool {
+      const int j = g & 1;
+      if (!warp_wait(b_dq(j), (g >> 1) & 1, abort_flag, p.err)) return false;
       tc_fence_after();
-      const bool diag = p.causal && t == u;
+      uint32_t r[32];
+      tmem_ld32_sync(tl + C::TM_DQ + j * 64 + cg * 32, r);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(b_dqfree(j));
+        bulk_wait_read<0>();  // this warp's previous reduce has read the slab
+      }
+      __syncwarp();
+      stage_row32(slab_g, lane, r, p.tau);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        int ph, m;
+        view_coords(U.g, U.si, t * BM + q4 * 32, ph, m);
+        tma_reduce_add_5d(U.macc, slab, cg * 32, U.wu.h, ph, m, U.wu.b);
+        bulk_commit();
+      }
+      return true;
+    };
+    for (uint32_t k = 0; ok; ++k) {
+      if (!warp_wait(b_unit(k & 1), (k >> 1) & 1, abort_flag, p.err)) break;
+      const long long uu = uslot[k & 1];
+      if (uu >= p.units) break;
+      BwdUnit U;
+      bwd_unit(p, uu, U);
+      const bool key_valid = U.u * BN + c < U.si.n;
+      int tprev = 0;
+      for (int it = 0; it < U.np; ++it, ++gp) {
+        const int s = gp & 1;
+        const int t = U.t0 + it;
+        const bool diag = p.causal && t == U.u;
+        if (!warp_wait(b_qfull(s), (gp >> 1) & 1, abort_flag, p.err)) {
+          ok = false;
+          break;
+        }
 #pragma unroll 1
-      for (int q = cg * C::CPT; q < cg * C::CPT + C::CPT; ++q) {
-        const float4* L4 = reinterpret_cast<const float4*>(sL + s * BM + q * 32);
-        const float4* D4 = reinterpret_cast<const float4*>(sD + s * BM + q * 32);
-        uint32_t pk[16], plo[16], dk[16], dkl[16];
-        {
-          uint32_t sv[32], dv[32];
-          tmem_ld32x2_sync(tl + C::TM_S + q * 32, tl + C::TM_DP + q * 32, sv, dv);
+        for (int h = 0; h < 2; ++h) {
+          if (!warp_wait(b_sdp(h), gp & 1, abort_flag, p.err)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int q = 2 * h + cg;  // this thread's 32 query columns: [32q, 32q + 32)
+          const bool split = C::split(t);
           // key rows past the segment, and (on the diagonal) queries before the
           // key, get P = 0; elsewhere no mask is needed
           const int jmin = !key_valid ? 1 << 30 : (diag ? c - q * 32 : 0);
-          const bool masked = jmin > 0;
-          const uint64_t sc2 = f2_pack(sc, sc);
+          const float* sLq = sL + s * BM + q * 32;
+          const float* sDq = sD + s * BM + q * 32;
+          // dS (query-major) into shared buffer gp & 1 for dQ = dS K: row c of
+          // half h holds dS[64h + j][c] for its 64 queries j, 16-byte pieces
+          // XOR-swizzled by c % 8
+          uint8_t* dsrow = base_g + C::OFF_DS + s * 2 * C::TILE + h * C::TILE + c * 128;
+          uint32_t sv[32], dv[32];
+          tmem_ld32x2_sync(tl + C::TM_S + q * 32, tl + C::TM_DP + q * 32, sv, dv);
+          // P^T, dS^T go in place over this chunk's own (already read) columns
+          if (!split) {
+            uint32_t pk[16], dk[16];
+            bwd_chunk<false, 0, 32>(sv, dv, sLq, sDq, sc, jmin, pk, nullptr, dk, nullptr);
+            tmem_st16(tl + C::TM_S + q * 32, pk);
+            tmem_st16(tl + C::TM_DP + q * 32, dk);
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 Lq = L4[e4], Dq = D4[e4];
-            const uint64_t nl2[2] = {f2_pack(-Lq.x, -Lq.y), f2_pack(-Lq.z, -Lq.w)};
-            const uint64_t dd2[2] = {f2_pack(Dq.x, Dq.y), f2_pack(Dq.z, Dq.w)};
+            for (int k4 = 0; k4 < 4; ++k4)
+              *reinterpret_cast<uint4*>(dsrow + (((cg * 4 + k4) ^ (c & 7)) * 16)) =
+                  make_uint4(dk[4 * k4], dk[4 * k4 + 1], dk[4 * k4 + 2], dk[4 * k4 + 3]);
+          } else {
+            // two 16-query halves; hi at +[0,16), lo at +[16,32): every column is
+            // already in registers before any store
+            {
+              uint32_t pk[8], plo[8], dk[8], dkl[8];
+              bwd_chunk<true, 0, 16>(sv, dv, sLq, sDq, sc, jmin, pk, plo, dk, dkl);
+              tmem_st8(tl + C::TM_S + q * 32, pk);
+              tmem_st8(tl + C::TM_S + q * 32 + 16, plo);
+              tmem_st8(tl + C::TM_DP + q * 32, dk);
+              tmem_st8(tl + C::TM_DP + q * 32 + 16, dkl);
 #pragma unroll
-            for (int h2 = 0; h2 < 2; ++h2) {
-              const int e = 4 * e4 + 2 * h2;
-              const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(sv[e]), __uint_as_float(sv[e + 1])),
-                                         sc2, nl2[h2]);
-              float p0 = ex2(f2_lo(x2)), p1 = ex2(f2_hi(x2));
-              if (masked) {
-                p0 = e >= jmin ? p0 : 0.f;
-                p1 = e + 1 >= jmin ? p1 : 0.f;
-              }
-              const uint64_t p2 = f2_pack(p0, p1);
-              // dS = P (dP - D)
-              const uint64_t ds2 = f2_mul(
-                  p2, f2_sub(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), dd2[h2]));
-              // P = hi + lo, both bf16: dV takes both halves, so P's own rounding
-              // (2^-9 relative) does not reach dV on top of dV's final bf16 rounding
-              const uint32_t hi = pack_bf16_rn(p0, p1);
-              const uint64_t hi2 = f2_pack(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u));
-              const uint64_t lo2 = f2_sub(p2, hi2);
-              pk[e / 2] = hi;
-              plo[e / 2] = pack_bf16_rn(f2_lo(lo2), f2_hi(lo2));
-              const uint32_t dhi = pack_bf16_rn(f2_lo(ds2), f2_hi(ds2));
-              const uint64_t dhi2 =
-                  f2_pack(__uint_as_float(dhi << 16), __uint_as_float(dhi & 0xffff0000u));
-              const uint64_t dlo2 = f2_sub(ds2, dhi2);
-              dk[e / 2] = dhi;
-              dkl[e / 2] = pack_bf16_rn(f2_lo(dlo2), f2_hi(dlo2));
+              for (int k4 = 0; k4 < 2; ++k4)
+                *reinterpret_cast<uint4*>(dsrow + (((cg * 4 + k4) ^ (c & 7)) * 16)) =
+                    make_uint4(dk[4 * k4], dk[4 * k4 + 1], dk[4 * k4 + 2], dk[4 * k4 + 3]);
+            }
+            {
+              uint32_t pk[8], plo[8], dk[8], dkl[8];
+              bwd_chunk<true, 16, 16>(sv, dv, sLq, sDq, sc, jmin, pk, plo, dk, dkl);
+              tmem_st8(tl + C::TM_S + q * 32 + 8, pk);
+              tmem_st8(tl + C::TM_S + q * 32 + 24, plo);
+              tmem_st8(tl + C::TM_DP + q * 32 + 8, dk);
+              tmem_st8(tl + C::TM_DP + q * 32 + 24, dkl);
+#pragma unroll
+              for (int k4 = 0; k4 < 2; ++k4)
+                *reinterpret_cast<uint4*>(dsrow + (((cg * 4 + 2 + k4) ^ (c & 7)) * 16)) =
+                    make_uint4(dk[4 * k4], dk[4 * k4 + 1], dk[4 * k4 + 2], dk[4 * k4 + 3]);
             }
           }
-        }
-        // in place over this chunk's own (already read) columns
-        tmem_st16(tl + C::TM_S + q * 32, pk);
-        tmem_st16(tl + C::TM_S + q * 32 + 16, plo);
-        tmem_st16(tl + C::TM_DP + q * 32, dk);
-        tmem_st16(tl + C::TM_DP + q * 32 + 16, dkl);
-        // dS (query-major) into SMEM for dQ = dS K: row c of chunk (j / 64)
-        // holds dS[j][c] for 64 consecutive j, 16-byte pieces XOR-swizzled by c % 8
-        {
-          const int chunk = q >> 1;
-          const int piece0 = (q & 1) * 4;
-          uint8_t* rowp = base_g + C::OFF_DS + chunk * C::TILE + c * 128;
-          uint8_t* rowl = base_g + C::OFF_DSL + chunk * C::TILE + c * 128;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int piece = (piece0 + k) ^ (c & 7);
-            *reinterpret_cast<uint4*>(rowp + piece * 16) =
-                make_uint4(dk[4 * k], dk[4 * k + 1], dk[4 * k + 2], dk[4 * k + 3]);
-            *reinterpret_cast<uint4*>(rowl + piece * 16) =
-                make_uint4(dkl[4 * k], dkl[4 * k + 1], dkl[4 * k + 2], dkl[4 * k + 3]);
+          tmem_wait_st();
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_rows(h));
+          // the previous pair's dQ leaves while the tensor pipe works on this one
+          if (h == 0 && it > 0 && !dq_out(U, gp - 1, tprev)) {
+            ok = false;
+            break;
           }
         }
+        if (!ok) break;
+        tprev = t;
       }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b_ds);
-
-      // dQ of this query tile (TMEM lane c = query row t*128 + c) -> staging
-      // buffer (it & 1) -> TMA reduce-add into the fp32 dq accumulator. Rows
-      // past the segment hold exact zeros (their P is 0); rows past N are
-      // clipped by the view.
-      if (!warp_wait(b_dq, it & 1, abort_flag, p.err)) {
+      if (!ok || !dq_out(U, gp - 1, tprev)) {
         ok = false;
         break;
       }
-      tc_fence_after();
-      if (threadIdx.x == 64) bulk_wait_read<0>();  // the previous reduce has read the staging buffer
-      if (!group_sync()) {
-        ok = false;
-        break;
-      }
-      uint8_t* stg = base_g + C::OFF_STG;
-#pragma unroll
-      for (int k = 0; k < C::CPT; ++k) {
-        const int col = (cg * C::CPT + k) * 16;  // dQ columns [col, col + 16)
-        uint32_t r[16];
-        tmem_ld16_sync(tl + C::TM_DQ + col, r);
-        stage_row16(stg + (col >> 5) * (C::STG_BYTES / 2), c, ((col >> 4) & 1) * 4, r, p.tau);
-      }
-      fence_proxy_async_smem();
-      if (!group_sync()) {
-        ok = false;
-        break;
-      }
-      if (threadIdx.x == 64) {
+      // dV, dK of the key tile: every MMA of the unit is complete (the last dQ
+      // commit tracks them all). Rows past the segment are exact zeros (their
+      // P was forced to 0). dv and dk are batch slots 2B + b and B + b.
+      {
+        uint32_t rv[32], rk[32];
+        tmem_ld32_sync(tl + C::TM_DV + cg * 32, rv);
+        tmem_ld32_sync(tl + C::TM_DK + cg * 32, rk);
+        tc_fence_before();
+        __syncwarp();
         int ph, m;
-        view_coords(g, si, t * BM, ph, m);
-        const uint32_t src = sSTG;
-        tma_reduce_add_5d(macc, src, 0, wu.h, ph, m, wu.b);
-        tma_reduce_add_5d(macc, src + C::STG_BYTES / 2, 32, wu.h, ph, m, wu.b);
-        bulk_commit();
-      }
-      tc_fence_before();
-    }
-    // dK, dV of the key tile (all pairs are complete after the last dQ wait):
-    // dV -> the staging buffer, tau * dK -> the dS area (idle now), TMA
-    // reduce-add into the dv and dk accumulators (batch slots 2B + b and
-    // B + b). Rows past the segment are exact zeros (their P was forced to 0).
-    if (ok) {
-      if (threadIdx.x == 64) bulk_wait_read<0>();
-      ok = group_sync();
-    }
-    if (ok) {
-      uint8_t* stg = base_g + C::OFF_STG;
-#pragma unroll
-      for (int k = 0; k < C::CPT; ++k) {
-        const int col = (cg * C::CPT + k) * 16;  // dV, dK columns [col, col + 16)
-        uint32_t r[16];
-        tmem_ld16_sync(tl + C::TM_DV + col, r);
-        stage_row16(stg + (col >> 5) * (C::STG_BYTES / 2), c, ((col >> 4) & 1) * 4, r, 1.f);
-        tmem_ld16_sync(tl + C::TM_DK + col, r);
-        stage_row16(base_g + C::OFF_DS + (col >> 5) * (C::STG_BYTES / 2), c, ((col >> 4) & 1) * 4,
-                    r, p.tau);
-      }
-      fence_proxy_async_smem();
-      ok = group_sync();
-    }
-    if (ok) {
-      if (threadIdx.x == 64) {
-        int ph, m;
-        view_coords(g, si, u * BN, ph, m);
-        tma_reduce_add_5d(macc, sSTG, 0, wu.h, ph, m, 2 * p.B + wu.b);
-        tma_reduce_add_5d(macc, sSTG + C::STG_BYTES / 2, 32, wu.h, ph, m, 2 * p.B + wu.b);
-        tma_reduce_add_5d(macc, sDS, 0, wu.h, ph, m, p.B + wu.b);
-        tma_reduce_add_5d(macc, sDS + C::STG_BYTES / 2, 32, wu.h, ph, m, p.B + wu.b);
-        bulk_commit();
+        view_coords(U.g, U.si, U.u * BN + q4 * 32, ph, m);
+        if (lane == 0) {
+          mbar_arrive(b_accfree);
+          bulk_wait_read<0>();
+        }
+        __syncwarp();
+        stage_row32(slab_g, lane, rv, 1.f);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_5d(U.macc, slab, cg * 32, U.wu.h, ph, m, 2 * p.B + U.wu.b);
+          bulk_commit();
+          bulk_wait_read<0>();
+        }
+        __syncwarp();
+        stage_row32(slab_g, lane, rk, p.tau);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_5d(U.macc, slab, cg * 32, U.wu.h, ph, m, p.B + U.wu.b);
+          bulk_commit();
+        }
       }
     }
-    if (threadIdx.x == 64) bulk_wait_all();  // shared memory stays until the reduces finish
-    tc_fence_before();
+    if (lane == 0) bulk_wait_all();  // shared memory stays until the reduces finish
+    __syncwarp();
   }
 
+  tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -478,11 +678,13 @@ struct PrepParams {
   float* dq_acc;
   float* dk_acc;
   float* dv_acc;
+  int* counter;  // the key-tile kernel's unit counter
 };
 
 __global__ void __launch_bounds__(256) bwd_prep_kernel(PrepParams p) {
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
+  if (row == 0 && threadIdx.x == 0) *p.counter = 0;
   if (row >= (long long)p.B * p.N * p.H) return;
   const __nv_bfloat162 d = reinterpret_cast<const __nv_bfloat162*>(p.dout + row * 64)[lane];
   float2 o;

@@ -530,3 +530,63 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
       : "memory");
 }
 }  // namespace dil
+
+namespace dil {
+// Warm the L2 with one 5-D tile of a tensor map (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_5d(const CUtensorMap* map, int c0, int c1, int c2,
+                                                   int c3, int c4) {
+  asm volatile(
+      "cp.async.bulk.prefetch.tensor.5d.L2.global.tile [%0, {%1, %2, %3, %4, %5}];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+      : "memory");
+}
+}  // namespace dil
+
+namespace dil {
+// 8-column TMEM store without a wait; follow a batch with tmem_wait_st().
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+      : "memory");
+}
+}  // namespace dil
+
+namespace dil {
+// Add `bytes` to the transaction count an mbarrier phase waits for, without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+}  // namespace dil
+
+namespace dil {
+// Bookkeeping of a polling loop with the same bounds as mbar_wait: step()
+// returns false once the loop has gone 4 s without progress, another warp of
+// the CTA raised *abort, or any CTA recorded an error in the device word.
+struct PollGuard {
+  uint32_t spins = 0;
+  unsigned long long t0 = 0;
+  __device__ __forceinline__ bool step(bool progressed, volatile int* abort, int* err) {
+    if (progressed) {
+      spins = 0;
+      t0 = 0;
+      return true;
+    }
+    if ((++spins & 1023u) != 0) return true;
+    if (*abort || *reinterpret_cast<volatile int*>(err) != 0) {
+      *abort = 1;
+      return false;
+    }
+    if (t0 == 0) {
+      t0 = globaltimer_ns();
+    } else if (globaltimer_ns() - t0 > 4000000000ull) {
+      atomicExch(err, (int)kErrWaitTimeout);
+      *abort = 1;
+      return false;
+    }
+    return true;
+  }
+};
+}  // namespace dil

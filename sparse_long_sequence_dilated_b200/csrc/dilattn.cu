@@ -113,20 +113,21 @@ int get_encoder() {
 // view has P = r phases and M = floor(N/r) rows; the tail view has
 // P = N mod r and M = floor(N/r) + 1. Either way every in-bounds coordinate is
 // a row below N; loads read zeros and stores/reduces skip rows past it. Box:
-// 128 bytes of columns (128-byte swizzle) x 128 rows.
-using MapKey = std::tuple<const void*, int, int, int, int, int, int, int>;
+// 128 bytes of columns (128-byte swizzle) x box_rows rows (128, or 32 for the
+// backward's per-warp reduce-adds).
+using MapKey = std::tuple<const void*, int, int, int, int, int, int, int, int>;
 std::mutex g_map_mu;
 std::map<MapKey, CUtensorMap> g_maps;
 
 int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CUtensorMap* out,
-                int f32 = 0) {
+                int f32 = 0, int box_rows = BM) {
   const long long nfloor = N / r;
   const int nmod = N % r;
   if ((tail && nmod == 0) || (!tail && nfloor == 0)) {
     memset(out, 0, sizeof(*out));  // a view no tile of this problem can address
     return DILATTN_OK;
   }
-  MapKey key{ptr, B, N, H, d, r, tail, f32};
+  MapKey key{ptr, B, N, H, d, r, tail, f32, box_rows};
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -143,7 +144,7 @@ int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CU
                         (cuuint64_t)(tail ? nfloor + 1 : nfloor), (cuuint64_t)B};
   cuuint64_t strides[4] = {(cuuint64_t)d * esz, (cuuint64_t)rowb, (cuuint64_t)(rowb * r),
                            (cuuint64_t)(rowb * N)};
-  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, 1, (cuuint32_t)BM, 1};
+  cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap m;
   CUresult cr = g_encode(&m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
@@ -167,7 +168,7 @@ int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CU
 // 2-D view of the forward's fp32 partial outputs [rows][d] for TMA stores:
 // box 32 columns (128 bytes, 128-byte swizzle) x 128 rows.
 int partial_map(const float* ptr, long long rows, int d, CUtensorMap* out) {
-  MapKey key{ptr, (int)(rows >> 31), (int)(rows & 0x7fffffff), d, -1, -1, -1, 2};
+  MapKey key{ptr, (int)(rows >> 31), (int)(rows & 0x7fffffff), d, -1, -1, -1, 2, BM};
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -378,13 +379,29 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
       if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j]);
       if (rc != DILATTN_OK) return rc;
     }
-    int rc = strided_map(dq_acc, 3 * B, N, H, D, r[i], 0, &p.tmacc[i], 1);
-    if (rc == DILATTN_OK) rc = strided_map(dq_acc, 3 * B, N, H, D, r[i], 1, &p.tmacc_t[i], 1);
+    // reduce-add targets: one row warp adds a 32-row x 32-column block
+    int rc = strided_map(dq_acc, 3 * B, N, H, D, r[i], 0, &p.tmacc[i], 1, 32);
+    if (rc == DILATTN_OK) rc = strided_map(dq_acc, 3 * B, N, H, D, r[i], 1, &p.tmacc_t[i], 1, 32);
     if (rc != DILATTN_OK) return rc;
   }
-  const long long units = make_schedule(p.pat, npat, B, H, p.sched);
+  // group-major unit order: patterns by tile count (descending, stable), then
+  // (segment, batch, head) groups, then key tiles
+  {
+    std::vector<int> order(npat);
+    for (int i = 0; i < npat; ++i) order[i] = i;
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int a, int b) { return p.pat[a].ntiles > p.pat[b].ntiles; });
+    p.gstart[0] = 0;
+    for (int a = 0; a < npat; ++a) {
+      const PatternGeom& g = p.pat[order[a]];
+      p.gorder[a] = order[a];
+      p.gstart[a + 1] = p.gstart[a] + (long long)g.nseg * B * H * g.ntiles;
+    }
+  }
+  const long long units = p.gstart[npat];
   if (units > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
   const long long rows = (long long)B * N * H;
+  p.counter = reinterpret_cast<int*>(wsb + 3 * tbytes + align256((size_t)B * H * N * 4));
 
   PrepParams pp;
   pp.B = B;
@@ -397,12 +414,17 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   pp.dq_acc = dq_acc;
   pp.dk_acc = dk_acc;
   pp.dv_acc = dv_acc;
+  pp.counter = p.counter;
   bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(pp);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd_prep_kernel launch");
   int rc = trace_mark(g_trace_begin, stream);
   if (rc != DILATTN_OK) return rc;
-  bwd_tile_kernel<<<(unsigned)units, BwdCfg::THREADS, BwdCfg::SMEM_BYTES, stream>>>(p);
+  // persistent: one CTA per SM walks the longest-first unit list with stride gridDim.x
+  p.units = units;
+  const long long grid = std::min<long long>(units, (long long)st->num_sms);
+  if (grid > 0)
+    bwd_tile_kernel<<<(unsigned)grid, BwdCfg::THREADS, BwdCfg::SMEM_BYTES, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd_tile_kernel launch");
   rc = trace_mark(g_trace_end, stream);
@@ -496,7 +518,7 @@ size_t dilattn_bwd_workspace_size(int B, int N, int H, int d, const int* w, cons
                                   int npat) {
   if (check_shape(B, N, H, d, w, r, npat, 1) != DILATTN_OK) return 0;
   const size_t t = (size_t)B * N * H * d * 4;
-  return 3 * align256(t) + align256((size_t)B * H * N * 4);
+  return 3 * align256(t) + align256((size_t)B * H * N * 4) + 256;  // + the unit counter
 }
 
 int dilattn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,

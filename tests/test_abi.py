@@ -81,7 +81,9 @@ def test_workspace_sizes():
     assert lib.dilattn_fwd_workspace_size(2, 512, 3, 64, w, r, n) == \
         align(rows * 64 * 4) + align(rows * 4) + align(2 * 512 * 3 * 64 * 4)
     t = 2 * 512 * 3 * 64 * 4
-    assert lib.dilattn_bwd_workspace_size(2, 512, 3, 64, w, r, n) == 3 * align(t) + align(2 * 3 * 512 * 4)
+    # dq, dk, dv accumulators, D, then 256 bytes for the key-tile kernel's unit counter
+    assert lib.dilattn_bwd_workspace_size(2, 512, 3, 64, w, r, n) == \
+        3 * align(t) + align(2 * 3 * 512 * 4) + 256
     assert lib.dilattn_fwd_workspace_size(0, 512, 3, 64, w, r, n) == 0
 
 

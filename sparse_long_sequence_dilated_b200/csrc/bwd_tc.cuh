@@ -90,13 +90,14 @@ struct BwdCfg {
   static constexpr int SLAB = 32 * 128;   // one row warp's 32 x 32 fp32 staging block
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
-  static constexpr int OFF_Q = OFF_V + TILE;                  // 2 stages
-  static constexpr int OFF_DO = OFF_Q + 2 * TILE;             // 2 stages
-  static constexpr int OFF_DS = OFF_DO + 2 * TILE;            // 2 buffers x 2 halves x [128 keys][64 q]
-  static constexpr int OFF_STG = OFF_DS + 4 * TILE;           // ROW_WARPS slabs
-  static constexpr int OFF_L = OFF_STG + ROW_WARPS * SLAB;    // 2 stages x 128 floats
-  static constexpr int OFF_D = OFF_L + 2 * BM * 4;            // 2 stages x 128 floats
-  static constexpr int OFF_BAR = OFF_D + 2 * BM * 4;
+  static constexpr int QST = 3;                               // Q / dO / L / D stages
+  static constexpr int OFF_Q = OFF_V + TILE;
+  static constexpr int OFF_DO = OFF_Q + QST * TILE;
+  static constexpr int OFF_DS = OFF_DO + QST * TILE;          // 2 halves x [128 keys][64 q]
+  static constexpr int OFF_STG = OFF_DS + 2 * TILE;           // ROW_WARPS slabs
+  static constexpr int OFF_L = OFF_STG + ROW_WARPS * SLAB;    // QST x 128 floats
+  static constexpr int OFF_D = OFF_L + QST * BM * 4;          // QST x 128 floats
+  static constexpr int OFF_BAR = OFF_D + QST * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
   static constexpr int TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 320, TM_DQ = 384;
   static constexpr int TMEM_COLS = 512;
@@ -223,8 +224,8 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   const uint32_t bars = base + C::OFF_BAR;
   const uint32_t b_kvfull = bars;         // K, V of the unit landed
   const uint32_t b_kvempty = bars + 8u;   // every MMA of the unit is complete
-  auto b_qfull = [&](int s) { return bars + 16u + 8u * s; };    // Q, dO, L, D of stage s
-  auto b_qempty = [&](int s) { return bars + 32u + 8u * s; };
+  auto b_qfull = [&](int s) { return bars + 144u + 8u * s; };   // Q, dO, L, D of stage s
+  auto b_qempty = [&](int s) { return bars + 168u + 8u * s; };
   auto b_sdp = [&](int h) { return bars + 48u + 8u * h; };      // S^T_h, dP^T_h in TMEM
   auto b_rows = [&](int h) { return bars + 64u + 8u * h; };     // P^T_h, dS^T_h written
   auto b_dq = [&](int j) { return bars + 80u + 8u * j; };       // dQ buffer j complete
@@ -239,9 +240,11 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   if (threadIdx.x == 0) {
     mbar_init(b_kvfull, 1);
     mbar_init(b_kvempty, 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < C::QST; ++s) {
       mbar_init(b_qfull(s), 1);
       mbar_init(b_qempty(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(b_sdp(s), 1);
       mbar_init(b_rows(s), C::ROW_WARPS);
       mbar_init(b_dq(s), 1);
@@ -338,9 +341,9 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       };
       load_ld(U.t0);
       for (int it = 0; it < U.np; ++it, ++gp) {
-        const int s = gp & 1;
+        const int s = gp % C::QST;
         const int t = U.t0 + it;
-        if (!warp_wait(b_qempty(s), ((gp >> 1) & 1) ^ 1, abort_flag, p.err)) {
+        if (!warp_wait(b_qempty(s), ((gp / C::QST) & 1) ^ 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
@@ -372,37 +375,44 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       // Drain copies still in flight before the CTA's shared memory goes away.
       volatile int no_abort = 0;
       if (k > 0) mbar_wait(b_kvfull, (k - 1) & 1, &no_abort, nullptr, 200000000ull);
-      for (uint32_t g = (gp >= 2 ? gp - 2 : 0); g < gp; ++g)
-        mbar_wait(b_qfull(g & 1), (g >> 1) & 1, &no_abort, nullptr, 200000000ull);
+      for (uint32_t g = (gp >= C::QST ? gp - C::QST : 0); g < gp; ++g)
+        mbar_wait(b_qfull(g % C::QST), (g / C::QST) & 1, &no_abort, nullptr, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop; one elected lane issues each MMA group.
+    {
       constexpr uint32_t kIdSh = idesc_bf16(BM, 64, 0, 0);  // K x Q_h^T, V x dO_h^T
       constexpr uint32_t kIdKV = idesc_bf16(BM, D, 0, 1);   // P^T / dS^T (TMEM) x dO / Q
       constexpr uint32_t kIdQ = idesc_bf16(BM, D, 1, 1);    // dS (MN-major SMEM) x K
+      // Descriptors are built once; each MMA only adds a byte offset to the
+      // low word, which keeps the issuing thread's work per MMA small (it
+      // shares its scheduler with two row warps).
+      const SDesc dKk = sdesc_sw128(sK, 16, 1024), dVk = sdesc_sw128(sV, 16, 1024);
+      const SDesc dQk = sdesc_sw128(sQ, 16, 1024), dDOk = sdesc_sw128(sDO, 16, 1024);
+      const SDesc dQm = sdesc_sw128(sQ, C::TILE, 1024), dDOm = sdesc_sw128(sDO, C::TILE, 1024);
+      const SDesc dDSm = sdesc_sw128(sDS, C::TILE, 1024), dKm = sdesc_sw128(sK, C::TILE, 1024);
       // S^T_h = K Q_h^T and dP^T_h = V dO_h^T for the 64 queries of half h
       auto issue_sdp = [&](uint32_t g, int h) {
-        const uint32_t qo = (g & 1) * C::TILE + h * C::HALF;
+        const uint32_t qo = (g % C::QST) * C::TILE + h * C::HALF;
+        const uint32_t ts = tmem + C::TM_S + h * 64, tp = tmem + C::TM_DP + h * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::TM_S + h * 64, sw128_desc(sK + kk * 32, 16, 1024),
-                 sw128_desc(sQ + qo + kk * 32, 16, 1024), kIdSh, kk > 0 ? 1u : 0u);
+          mma_ss(ts, dKk.at(kk * 32), dQk.at(qo + kk * 32), kIdSh, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tmem + C::TM_DP + h * 64, sw128_desc(sV + kk * 32, 16, 1024),
-                 sw128_desc(sDO + qo + kk * 32, 16, 1024), kIdSh, kk > 0 ? 1u : 0u);
+          mma_ss(tp, dVk.at(kk * 32), dDOk.at(qo + kk * 32), kIdSh, kk > 0 ? 1u : 0u);
         mma_commit(b_sdp(h));
       };
       // dV += P^T_h dO_h, dK += dS^T_h Q_h (each hi + lo when `split`); `first`
       // starts the accumulators
       auto issue_dvdk = [&](uint32_t g, int h, bool first, bool split) {
-        const uint32_t qo = (g & 1) * C::TILE;
+        const uint32_t qo = (g % C::QST) * C::TILE;
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
           const int kk = 4 * h + kq;  // 16 queries
-          const uint64_t bdo = sw128_desc(sDO + qo + kk * 2048, C::TILE, 1024);
+          const uint64_t bdo = dDOm.at(qo + kk * 2048);
           const uint32_t a = tmem + C::TM_S + (kk >> 1) * 32 + (kk & 1) * 8;
           mma_ts(tmem + C::TM_DV, a, bdo, kIdKV, (first && kq == 0) ? 0u : 1u);
           if (split) mma_ts(tmem + C::TM_DV, a + 16, bdo, kIdKV, 1u);
@@ -410,47 +420,55 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
           const int kk = 4 * h + kq;
-          const uint64_t bq = sw128_desc(sQ + qo + kk * 2048, C::TILE, 1024);
+          const uint64_t bq = dQm.at(qo + kk * 2048);
           const uint32_t a = tmem + C::TM_DP + (kk >> 1) * 32 + (kk & 1) * 8;
           mma_ts(tmem + C::TM_DK, a, bq, kIdKV, (first && kq == 0) ? 0u : 1u);
           if (split) mma_ts(tmem + C::TM_DK, a + 16, bq, kIdKV, 1u);
         }
       };
-      // dQ = dS K into TMEM buffer g & 1 (dS from shared-memory buffer g & 1)
+      // dQ = dS K into TMEM buffer g & 1 (dS from shared memory)
       auto issue_dq = [&](uint32_t g) {
         const int j = g & 1;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ss(tmem + C::TM_DQ + j * 64, sw128_desc(sDS + j * 2 * C::TILE + kk * 2048, C::TILE, 1024),
-                 sw128_desc(sK + kk * 2048, C::TILE, 1024), kIdQ, kk > 0 ? 1u : 0u);
+          mma_ss(tmem + C::TM_DQ + j * 64, dDSm.at(kk * 2048), dKm.at(kk * 2048), kIdQ,
+                 kk > 0 ? 1u : 0u);
         mma_commit(b_dq(j));
+      };
+      // warp-uniform non-blocking test of a barrier phase
+      auto test = [&](uint32_t bar, uint32_t par) -> bool {
+        return __shfl_sync(0xffffffffu, mbar_test(bar, par) ? 1 : 0, 0) != 0;
       };
       uint32_t gp = 0, k = 0;
       bool ok = true;
       for (;; ++k) {
-        if (!mbar_wait(b_unit(k & 1), (k >> 1) & 1, abort_flag, p.err)) break;
+        if (!warp_wait(b_unit(k & 1), (k >> 1) & 1, abort_flag, p.err)) break;
         const long long uu = uslot[k & 1];
         if (uu >= p.units) break;
         BwdUnit U;
         bwd_unit(p, uu, U);
-        if (!mbar_wait(b_kvfull, k & 1, abort_flag, p.err) ||
-            !mbar_wait(b_qfull(gp & 1), (gp >> 1) & 1, abort_flag, p.err)) {
+        if (!warp_wait(b_kvfull, k & 1, abort_flag, p.err) ||
+            !warp_wait(b_qfull(gp % C::QST), (gp / C::QST) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        issue_sdp(gp, 0);
-        issue_sdp(gp, 1);
+        if (elect_one_sync()) {
+          issue_sdp(gp, 0);
+          issue_sdp(gp, 1);
+        }
+        __syncwarp();
         for (int it = 0; it < U.np; ++it, ++gp) {
           const bool more = it + 1 < U.np;
-          if (!mbar_wait(b_rows(0), gp & 1, abort_flag, p.err) ||
-              (it == 0 && k > 0 && !mbar_wait(b_accfree, (k - 1) & 1, abort_flag, p.err))) {
+          if (!warp_wait(b_rows(0), gp & 1, abort_flag, p.err) ||
+              (it == 0 && k > 0 && !warp_wait(b_accfree, (k - 1) & 1, abort_flag, p.err))) {
             ok = false;
             break;
           }
           tc_fence_after();
           const bool split = C::split(U.t0 + it);
-          issue_dvdk(gp, 0, it == 0, split);
+          if (elect_one_sync()) issue_dvdk(gp, 0, it == 0, split);
+          __syncwarp();
           // Then, in whichever order their inputs arrive: S / dP half 0 of the
           // next pair (Q, dO landed) and dV / dK half 1 plus dQ of this pair
           // (half 1 written, dQ buffer read out). S / dP half 1 of the next
@@ -459,34 +477,42 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           PollGuard pg;
           while (need_s0 || need_1) {
             bool prog = false;
-            if (need_s0 && mbar_test(b_qfull((gp + 1) & 1), ((gp + 1) >> 1) & 1)) {
+            if (need_s0 && test(b_qfull((gp + 1) % C::QST), ((gp + 1) / C::QST) & 1)) {
               tc_fence_after();
-              issue_sdp(gp + 1, 0);
+              if (elect_one_sync()) issue_sdp(gp + 1, 0);
+              __syncwarp();
               need_s0 = false;
               prog = true;
             }
-            if (need_1 && mbar_test(b_rows(1), gp & 1) &&
-                (gp < 2 || mbar_test(b_dqfree(gp & 1), ((gp >> 1) & 1) ^ 1))) {
+            if (need_1 && test(b_rows(1), gp & 1) &&
+                (gp < 2 || test(b_dqfree(gp & 1), ((gp >> 1) & 1) ^ 1))) {
               tc_fence_after();
-              issue_dvdk(gp, 1, false, split);
-              mma_commit(b_qempty(gp & 1));
-              issue_dq(gp);
+              if (elect_one_sync()) {
+                issue_dvdk(gp, 1, false, split);
+                mma_commit(b_qempty(gp % C::QST));
+                issue_dq(gp);
+              }
+              __syncwarp();
               need_1 = false;
               prog = true;
             }
-            if (!pg.step(prog, abort_flag, p.err)) {
+            if (!__all_sync(0xffffffffu, pg.step(prog, abort_flag, p.err))) {
               ok = false;
               break;
             }
           }
           if (!ok) break;
-          if (more) issue_sdp(gp + 1, 1);
-          else mma_commit(b_kvempty);
+          if (elect_one_sync()) {
+            if (more) issue_sdp(gp + 1, 1);
+            else mma_commit(b_kvempty);
+          }
+          __syncwarp();
         }
         if (!ok) break;
       }
       // every MMA issued so far completes before TMEM is released
-      mma_commit(b_fin);
+      if (elect_one_sync()) mma_commit(b_fin);
+      __syncwarp();
       volatile int no_abort = 0;
       mbar_wait(b_fin, 0, &no_abort, nullptr, 200000000ull);
     }
@@ -539,10 +565,10 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       const bool key_valid = U.u * BN + c < U.si.n;
       int tprev = 0;
       for (int it = 0; it < U.np; ++it, ++gp) {
-        const int s = gp & 1;
+        const int s = gp % C::QST;
         const int t = U.t0 + it;
         const bool diag = p.causal && t == U.u;
-        if (!warp_wait(b_qfull(s), (gp >> 1) & 1, abort_flag, p.err)) {
+        if (!warp_wait(b_qfull(s), (gp / C::QST) & 1, abort_flag, p.err)) {
           ok = false;
           break;
         }
@@ -560,59 +586,63 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           const int jmin = !key_valid ? 1 << 30 : (diag ? c - q * 32 : 0);
           const float* sLq = sL + s * BM + q * 32;
           const float* sDq = sD + s * BM + q * 32;
-          // dS (query-major) into shared buffer gp & 1 for dQ = dS K: row c of
-          // half h holds dS[64h + j][c] for its 64 queries j, 16-byte pieces
+          // dS (query-major) into shared memory for dQ = dS K: row c of half h
+          // holds dS[64h + j][c] for its 64 queries j, 16-byte pieces
           // XOR-swizzled by c % 8
-          uint8_t* dsrow = base_g + C::OFF_DS + s * 2 * C::TILE + h * C::TILE + c * 128;
-          uint32_t sv[32], dv[32];
-          tmem_ld32x2_sync(tl + C::TM_S + q * 32, tl + C::TM_DP + q * 32, sv, dv);
-          // P^T, dS^T go in place over this chunk's own (already read) columns
-          if (!split) {
-            uint32_t pk[16], dk[16];
-            bwd_chunk<false, 0, 32>(sv, dv, sLq, sDq, sc, jmin, pk, nullptr, dk, nullptr);
-            tmem_st16(tl + C::TM_S + q * 32, pk);
-            tmem_st16(tl + C::TM_DP + q * 32, dk);
+          uint8_t* dsrow = base_g + C::OFF_DS + h * C::TILE + c * 128;
+          uint32_t dk[16];
+          {
+            uint32_t sv[32], dv[32];
+            tmem_ld32x2_sync(tl + C::TM_S + q * 32, tl + C::TM_DP + q * 32, sv, dv);
+            // P^T, dS^T go in place over this chunk's own (already read) columns
+            if (!split) {
+              uint32_t pk[16];
+              bwd_chunk<false, 0, 32>(sv, dv, sLq, sDq, sc, jmin, pk, nullptr, dk, nullptr);
+              tmem_st16(tl + C::TM_S + q * 32, pk);
+              tmem_st16(tl + C::TM_DP + q * 32, dk);
+            } else {
+              // two 16-query halves; hi at +[0,16), lo at +[16,32): every column
+              // is already in registers before any store
+              {
+                uint32_t pk[8], plo[8], dkl[8];
+                bwd_chunk<true, 0, 16>(sv, dv, sLq, sDq, sc, jmin, pk, plo, dk, dkl);
+                tmem_st8(tl + C::TM_S + q * 32, pk);
+                tmem_st8(tl + C::TM_S + q * 32 + 16, plo);
+                tmem_st8(tl + C::TM_DP + q * 32, dk);
+                tmem_st8(tl + C::TM_DP + q * 32 + 16, dkl);
+              }
+              {
+                uint32_t pk[8], plo[8], dkl[8];
+                bwd_chunk<true, 16, 16>(sv, dv, sLq, sDq, sc, jmin, pk, plo, dk + 8, dkl);
+                tmem_st8(tl + C::TM_S + q * 32 + 8, pk);
+                tmem_st8(tl + C::TM_S + q * 32 + 24, plo);
+                tmem_st8(tl + C::TM_DP + q * 32 + 8, dk + 8);
+                tmem_st8(tl + C::TM_DP + q * 32 + 24, dkl);
+              }
+            }
+          }
+          auto store_ds = [&]() {
 #pragma unroll
             for (int k4 = 0; k4 < 4; ++k4)
               *reinterpret_cast<uint4*>(dsrow + (((cg * 4 + k4) ^ (c & 7)) * 16)) =
                   make_uint4(dk[4 * k4], dk[4 * k4 + 1], dk[4 * k4 + 2], dk[4 * k4 + 3]);
-          } else {
-            // two 16-query halves; hi at +[0,16), lo at +[16,32): every column is
-            // already in registers before any store
-            {
-              uint32_t pk[8], plo[8], dk[8], dkl[8];
-              bwd_chunk<true, 0, 16>(sv, dv, sLq, sDq, sc, jmin, pk, plo, dk, dkl);
-              tmem_st8(tl + C::TM_S + q * 32, pk);
-              tmem_st8(tl + C::TM_S + q * 32 + 16, plo);
-              tmem_st8(tl + C::TM_DP + q * 32, dk);
-              tmem_st8(tl + C::TM_DP + q * 32 + 16, dkl);
-#pragma unroll
-              for (int k4 = 0; k4 < 2; ++k4)
-                *reinterpret_cast<uint4*>(dsrow + (((cg * 4 + k4) ^ (c & 7)) * 16)) =
-                    make_uint4(dk[4 * k4], dk[4 * k4 + 1], dk[4 * k4 + 2], dk[4 * k4 + 3]);
-            }
-            {
-              uint32_t pk[8], plo[8], dk[8], dkl[8];
-              bwd_chunk<true, 16, 16>(sv, dv, sLq, sDq, sc, jmin, pk, plo, dk, dkl);
-              tmem_st8(tl + C::TM_S + q * 32 + 8, pk);
-              tmem_st8(tl + C::TM_S + q * 32 + 24, plo);
-              tmem_st8(tl + C::TM_DP + q * 32 + 8, dk);
-              tmem_st8(tl + C::TM_DP + q * 32 + 24, dkl);
-#pragma unroll
-              for (int k4 = 0; k4 < 2; ++k4)
-                *reinterpret_cast<uint4*>(dsrow + (((cg * 4 + 2 + k4) ^ (c & 7)) * 16)) =
-                    make_uint4(dk[4 * k4], dk[4 * k4 + 1], dk[4 * k4 + 2], dk[4 * k4 + 3]);
-            }
-          }
+          };
+          // The single dS buffer is free once the previous pair's dQ MMA has
+          // completed: half 0 waits for that in dq_out below (except on a
+          // unit's first pair, where the previous unit's last dq_out did).
+          if (h == 1 || it == 0) store_ds();
           tmem_wait_st();
           fence_proxy_async_smem();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(b_rows(h));
           // the previous pair's dQ leaves while the tensor pipe works on this one
-          if (h == 0 && it > 0 && !dq_out(U, gp - 1, tprev)) {
-            ok = false;
-            break;
+          if (h == 0 && it > 0) {
+            if (!dq_out(U, gp - 1, tprev)) {
+              ok = false;
+              break;
+            }
+            store_ds();
           }
         }
         if (!ok) break;

@@ -590,3 +590,34 @@ struct PollGuard {
   }
 };
 }  // namespace dil
+
+namespace dil {
+// A shared-memory matrix descriptor kept as two 32-bit words. The start
+// address field (addr >> 4) sits in the low 14 bits of `lo`, so advancing by
+// a byte offset that keeps the address inside the 256 KB shared window is a
+// single add of offset >> 4; `hi` (stride, version, swizzle) never changes.
+struct SDesc {
+  uint32_t lo, hi;
+  __device__ __forceinline__ uint64_t at(uint32_t byte_off) const {
+    return ((uint64_t)hi << 32) | (uint64_t)(lo + (byte_off >> 4));
+  }
+};
+__device__ __forceinline__ SDesc sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  const uint64_t d = sw128_desc(saddr, lbo_bytes, sbo_bytes);
+  return SDesc{(uint32_t)d, (uint32_t)(d >> 32)};
+}
+}  // namespace dil
+
+namespace dil {
+// One lane of a converged warp (elect.sync): the lane that issues
+// single-thread tcgen05 / TMA instructions on behalf of the warp.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 r;\n\t"
+      "elect.sync r|p, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+}  // namespace dil

@@ -196,64 +196,55 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     // ------------------------------------------------------------ MMA issuer
     // Event loop: S(j) = Q K_j^T as soon as K_j is resident and the softmax has
     // read S(j-1); PV(j) as soon as P(j) and V_j are ready. Neither waits for
-    // the other's operands.
-    if (lane == 0) {
+    // the other's operands. The whole warp runs the loop; one elected lane
+    // issues each MMA group (descriptors are built once and advanced by adds).
+    {
       constexpr uint32_t kIdS = idesc_bf16(BM, BN, 0, 0);  // Q (K-major) x K (K-major)
       constexpr uint32_t kIdO = idesc_bf16(BM, D, 0, 1);   // P (TMEM) x V (MN-major)
-      bool ok = mbar_wait(b_qfull, 0, abort_flag, p.err);
+      const SDesc dQ = sdesc_sw128(sQ, 16, 1024), dK = sdesc_sw128(sK, 16, 1024);
+      const SDesc dV = sdesc_sw128(sV, C::CHUNK_BYTES, 1024);
+      auto test = [&](uint32_t bar, uint32_t par) -> bool {
+        return __shfl_sync(0xffffffffu, mbar_test(bar, par) ? 1 : 0, 0) != 0;
+      };
+      bool ok = warp_wait(b_qfull, 0, abort_flag, p.err);
       int ns = 0, npv = 0;
-      uint32_t spins = 0;
-      unsigned long long t0 = 0;
+      PollGuard pg;
       while (ok && npv < nkv) {
         bool progressed = false;
-        if (ns < nkv && mbar_test(b_kfull(ns % C::KST), (ns / C::KST) & 1) &&
-            (ns == 0 || mbar_test(b_sfree, (ns - 1) & 1))) {
+        if (ns < nkv && test(b_kfull(ns % C::KST), (ns / C::KST) & 1) &&
+            (ns == 0 || test(b_sfree, (ns - 1) & 1))) {
           tc_fence_after();
-          const int ks = ns % C::KST;
+          const uint32_t ko = (ns % C::KST) * C::KV_BYTES;
+          if (elect_one_sync()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-            const uint64_t a = sw128_desc(sQ + off, 16, 1024);
-            const uint64_t bd = sw128_desc(sK + ks * C::KV_BYTES + off, 16, 1024);
-            mma_ss(tmem + C::TM_S, a, bd, kIdS, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+              mma_ss(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(b_sfull);
+            mma_commit(b_kempty(ns % C::KST));
           }
-          mma_commit(b_sfull);
-          mma_commit(b_kempty(ks));
+          __syncwarp();
           ++ns;
           progressed = true;
         }
-        if (npv < ns && mbar_test(b_pfull, npv & 1) &&
-            mbar_test(b_vfull(npv % C::VST), (npv / C::VST) & 1)) {
+        if (npv < ns && test(b_pfull, npv & 1) &&
+            test(b_vfull(npv % C::VST), (npv / C::VST) & 1)) {
           tc_fence_after();
-          const int vs = npv % C::VST;
+          const uint32_t vo = (npv % C::VST) * C::KV_BYTES;
+          if (elect_one_sync()) {
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t bd =
-                sw128_desc(sV + vs * C::KV_BYTES + kk * 2048, C::CHUNK_BYTES, 1024);
-            mma_ts(tmem + C::TM_O, tmem + C::TM_P + kk * 8, bd, kIdO,
-                   (npv > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / 16; ++kk)
+              mma_ts(tmem + C::TM_O, tmem + C::TM_P + kk * 8, dV.at(vo + kk * 2048), kIdO,
+                     (npv > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(b_vempty(npv % C::VST));
+            mma_commit(b_odone);
           }
-          mma_commit(b_vempty(vs));
-          mma_commit(b_odone);
+          __syncwarp();
           ++npv;
           progressed = true;
         }
-        if (progressed) {
-          spins = 0;
-        } else if ((++spins & 1023u) == 0) {
-          // bounded like mbar_wait: give up after 4 s without progress or on abort
-          if (*abort_flag || *reinterpret_cast<volatile int*>(p.err) != 0) {
-            *abort_flag = 1;
-            ok = false;
-          } else if (t0 == 0) {
-            t0 = globaltimer_ns();
-          } else if (globaltimer_ns() - t0 > 4000000000ull) {
-            atomicExch(p.err, (int)kErrWaitTimeout);
-            *abort_flag = 1;
-            ok = false;
-          }
-        }
-        if (progressed) t0 = 0;
+        if (!__all_sync(0xffffffffu, pg.step(progressed, abort_flag, p.err))) ok = false;
       }
     }
     __syncwarp();

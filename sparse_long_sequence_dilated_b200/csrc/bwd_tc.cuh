@@ -22,7 +22,7 @@
 //   P^T_h  = exp2(S^T_h tau log2e - L log2e), dS^T_h = P^T_h (dP^T_h - D)  (threads)
 //   dV += P^T_h dO_h,  dK += dS^T_h Q_h                    (TMEM x SMEM -> TMEM)
 //   dQ  = dS K  (both halves; dS from SMEM)                (SMEM x SMEM -> TMEM)
-// MMA issue order per pair i: dVdK_0(i), SdP_0(i+1), dVdK_1(i), dQ(i),
+// MMA issue order per pair i: dVdK_0(i), SdP_0(i+1), dQ(i), dVdK_1(i),
 // SdP_1(i+1); the row threads work on half 1 of pair i while dVdK_0(i) and
 // SdP_0(i+1) run, and on half 0 of pair i+1 while dVdK_1(i), dQ(i) and
 // SdP_1(i+1) run. An S / dP half is overwritten only by MMAs issued after
@@ -488,9 +488,9 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
                 (gp < 2 || test(b_dqfree(gp & 1), ((gp >> 1) & 1) ^ 1))) {
               tc_fence_after();
               if (elect_one_sync()) {
+                issue_dq(gp);  // first: the row warps wait for it before their next dS store
                 issue_dvdk(gp, 1, false, split);
                 mma_commit(b_qempty(gp % C::QST));
-                issue_dq(gp);
               }
               __syncwarp();
               need_1 = false;

@@ -30,6 +30,12 @@
 
 #include "common.cuh"
 
+// Column pairs, of every 8, whose exp2 runs as a polynomial on the FMA pipe
+// instead of the MUFU unit.
+#ifndef DILATTN_FWD_POLY
+#define DILATTN_FWD_POLY 0
+#endif
+
 namespace dil {
 
 struct FwdParams {
@@ -309,8 +315,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(raw[2 * c]),
                                            __uint_as_float(raw[2 * c + 1])), sc2, negm2);
         uint64_t p2;
-        if ((c & 7) >= 5) {
-          p2 = ex2_poly2(x2);  // 3 pairs in 8 on the FMA pipe
+        if ((c & 7) >= 8 - DILATTN_FWD_POLY) {
+          p2 = ex2_poly2(x2);  // DILATTN_FWD_POLY pairs in 8 on the FMA pipe
         } else {
           p2 = f2_pack(ex2(f2_lo(x2)), ex2(f2_hi(x2)));
         }

@@ -200,6 +200,74 @@ def run_reference(args, rank: int, world: int):
 # ---------------------------------------------------------------------------
 # GPU leg
 # ---------------------------------------------------------------------------
+SWEEP = ("sweep_8192", "sweep_131072", "sweep_1048576")  # the length sweep, fwd + bwd
+WIDE = "wide_128k"                                         # d = 128, forward
+
+
+def sweep_detail(dilattn, dev, steps: int = 3, warmup: int = 2):
+    """Tile-kernel and whole-call times for the length sweep (N = 8K, 128K, 1M; fwd + bwd)
+    and the wide d = 128 forward, each on i.i.d. N(0, 1) bf16 inputs drawn on the device
+    (the kernels' cost does not depend on the values), L2 flushed before every call."""
+    import torch
+
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    res = []
+    for name in SWEEP + (WIDE,):
+        wl = WORKLOADS[name]
+        B, N, H, d, pats = wl.B, wl.N, wl.H, wl.d, wl.patterns
+        t = [torch.randn((B, N, H, d), generator=gen, device=dev, dtype=torch.float32)
+             .to(torch.bfloat16) for _ in range(4)]
+        q, k, v, do = t
+        ws_f = torch.empty(dilattn.fwd_workspace_size(B, N, H, d, pats), dtype=torch.uint8,
+                           device=dev)
+        with_bwd = wl.backward and d == 64
+        tiles = [ev() for _ in range(4)]
+        for e in tiles:
+            e.record()
+        ftile, btile, fwhole, bwhole = [], [], [], []
+        for i in range(warmup + steps):
+            a, b, c = ev(), ev(), ev()
+            flush_buf.fill_(1)
+            a.record()
+            dilattn.set_trace_events(tiles[0], tiles[1])
+            out, lse = dilattn.fwd(q, k, v, pats, wl.causal, workspace=ws_f)
+            b.record()
+            if with_bwd:
+                dilattn.set_trace_events(tiles[2], tiles[3])
+                dilattn.bwd(q, k, v, out, lse, do, pats, wl.causal, fwd_workspace=ws_f)
+            c.record()
+            dilattn.set_trace_events(None, None)
+            torch.cuda.synchronize()
+            if i >= warmup:
+                ftile.append(tiles[0].elapsed_time(tiles[1]))
+                fwhole.append(a.elapsed_time(b))
+                if with_bwd:
+                    btile.append(tiles[2].elapsed_time(tiles[3]))
+                    bwhole.append(b.elapsed_time(c))
+        fw = flops.fwd_flops(B, N, H, d, pats, wl.causal)
+        ent = {"workload": name, "B": B, "N": N, "H": H, "d": d,
+               "fwd_tile_ms": statistics.median(ftile), "fwd_ms": statistics.median(fwhole),
+               "fwd_tile_tflops": fw / statistics.median(ftile) / 1e9,
+               "fwd_tflops": fw / statistics.median(fwhole) / 1e9}
+        if with_bwd:
+            bw = flops.bwd_flops(B, N, H, d, pats, wl.causal)
+            ent.update({"bwd_tile_ms": statistics.median(btile), "bwd_ms": statistics.median(bwhole),
+                        "bwd_tile_tflops": bw / statistics.median(btile) / 1e9,
+                        "step_tflops": (fw + bw) / (statistics.median(fwhole)
+                                                    + statistics.median(bwhole)) / 1e9,
+                        "tokens_per_s": B * N / ((statistics.median(fwhole)
+                                                  + statistics.median(bwhole)) * 1e-3)})
+        res.append(ent)
+        del q, k, v, do, t, ws_f
+        torch.cuda.empty_cache()
+    if dilattn.device_error() != 0:
+        raise RuntimeError("a kernel reported a device-side error in the length sweep")
+    return res
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import numpy as np
     import torch
@@ -354,6 +422,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "gpu_launches": 5 * K,
         "clocks": clocks,
     }
+    if world == 1 and not args.no_sweep:
+        line["detail"]["length_sweep"] = sweep_detail(dilattn, dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
@@ -371,6 +441,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the length sweep (N = 8K, 128K, 1M) and the wide d = 128 forward")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -200,6 +200,30 @@ def run_reference(args, rank: int, world: int):
 # ---------------------------------------------------------------------------
 # GPU leg
 # ---------------------------------------------------------------------------
+# ---------------------------------------------------------------------------
+# multi-rank host logic (one process per GPU; also run with gloo on CPU in tests)
+# ---------------------------------------------------------------------------
+def rank_seed(base_seed: int, rank: int) -> int:
+    """Every rank draws its own batch: the workload's seed plus the rank."""
+    return base_seed + rank
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of the ranks' values of x (a time): the job ends with its slowest rank."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, work_per_rank: float, ms: float, calls: int = 1) -> float:
+    """Whole-job throughput: all ranks' effective FLOPs over the max-over-ranks time."""
+    return world * work_per_rank * calls / (ms * 1e-3) / 1e12
+
+
 SWEEP = ("sweep_8192", "sweep_131072", "sweep_1048576")  # the length sweep, fwd + bwd
 WIDE = "wide_128k"                                         # d = 128, forward
 
@@ -286,7 +310,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     pats = wl.patterns
     causal = wl.causal
 
-    inp = make_inputs(B, N, H, d, wl.seed + rank, wl.dtype, NAMES)
+    inp = make_inputs(B, N, H, d, rank_seed(wl.seed, rank), wl.dtype, NAMES)
     host = {n: torch.from_numpy(np.ascontiguousarray(inp[n + "_bits"]).view(np.int16))
             .view(torch.bfloat16).pin_memory() for n in NAMES}
     q, k, v, do = (host[n].to(dev) for n in NAMES)
@@ -342,10 +366,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     step_ms = sum(a.elapsed_time(b) for a, b in step_ev)
     fwd_tile_ms = sum(t[0].elapsed_time(t[1]) for t in tile_ev) / K
     bwd_tile_ms = sum(t[2].elapsed_time(t[3]) for t in tile_ev) / K
-    if world > 1:
-        t = torch.tensor([step_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+    step_ms = max_over_ranks(step_ms, world, dev)
     ms_per_step = step_ms / K
 
     # e2e through the public API: pinned host inputs in, results back out
@@ -374,19 +395,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     if dilattn.device_error() != 0:
         raise RuntimeError("a kernel reported a device-side error")
 
     fwd_work = flops.fwd_flops(B, N, H, d, pats, causal)
     bwd_work = flops.bwd_flops(B, N, H, d, pats, causal)
     step_work = fwd_work + bwd_work
-    value = world * step_work / (ms_per_step * 1e-3) / 1e12
-    e2e_value = world * step_work * K / (e2e_ms * 1e-3) / 1e12
+    value = job_tflops(world, step_work, ms_per_step)
+    e2e_value = job_tflops(world, step_work, e2e_ms, K)
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     fwd_tile_tf = fwd_work / (fwd_tile_ms * 1e-3) / 1e12

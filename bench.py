@@ -42,13 +42,16 @@ METRIC = "dilated-attn fwd/bwd effective TFLOP/s & tokens/s at N=32K–1M; % of 
 UNIT = "TFLOP/s"
 DEFAULT_WORKLOAD = "longnet_base_32k"
 PEAK_FALLBACK = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
-KERNEL_SOURCES = ("common.cuh", "fwd_tc.cuh", "bwd_tc.cuh", "simt.cuh")  # device code only
+# device-code files each tile kernel is built from (the DRAM-traffic record of a
+# kernel stays valid while these are unchanged)
+KERNEL_SOURCES = {"fwd_tile_kernel": ("common.cuh", "fwd_tc.cuh"),
+                  "bwd_tile_kernel": ("common.cuh", "bwd_tc.cuh")}
 NAMES = ("q", "k", "v", "dout")
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "sparse_long_sequence_dilated_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -71,7 +74,7 @@ def load_traffic(kernel: str, workload: str):
     with open(path) as f:
         rec = json.load(f)
     ent = rec.get(kernel, {}).get(workload)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("dram_bytes_per_launch")
 

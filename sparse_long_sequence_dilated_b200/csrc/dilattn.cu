@@ -336,7 +336,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   mp.out_f32 = fwd_out_f32(ws, rows, D);
   mp.lse = lse;
   const long long total_rows = (long long)B * N * H;
-  const long long blocks = (total_rows + 31) / 32;
+  constexpr int rows_per_block = 256 / DILATTN_MERGE_TPR;
+  const long long blocks = (total_rows + rows_per_block - 1) / rows_per_block;
   merge_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(mp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "merge_kernel launch");

@@ -50,14 +50,20 @@ struct MergeParams {
   float* lse;      // may be null
 };
 
-// 8 threads per output row, each owning D/8 consecutive columns; 32 rows per
-// 256-thread block. Single pass with a running max, so every partial load is
+// DILATTN_MERGE_TPR threads per output row (default 4; 8 and 16 were measured
+// slower at d = 64), each owning D / TPR consecutive columns; 256 / TPR rows
+// per 256-thread block. Single pass with a running max, so every partial load is
 // independent of the previous pattern's result.
+#ifndef DILATTN_MERGE_TPR
+#define DILATTN_MERGE_TPR 4
+#endif
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ MergeParams p) {
-  constexpr int PER = D / 8;  // floats per thread: 8 (d = 64) or 16 (d = 128)
-  const long long row = (long long)blockIdx.x * 32 + (threadIdx.x >> 3);
-  const int sub = threadIdx.x & 7;
+  constexpr int TPR = DILATTN_MERGE_TPR;  // threads per output row
+  constexpr int PER = D / TPR;            // floats per thread
+  static_assert(PER % 4 == 0, "each thread owns whole float4 groups");
+  const long long row = (long long)blockIdx.x * (256 / TPR) + (threadIdx.x / TPR);
+  const int sub = threadIdx.x % TPR;
   const long long total = (long long)p.B * p.N * p.H;
   if (row >= total) return;
   const int h = (int)(row % p.H);
@@ -111,10 +117,16 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
   uint32_t pk[PER / 2];
 #pragma unroll
   for (int e = 0; e < PER / 2; ++e) pk[e] = pack_bf16(acc[2 * e], acc[2 * e + 1]);
-  uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + sub * PER);
+  if (PER % 8 == 0) {
+    uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + sub * PER);
 #pragma unroll
-  for (int e = 0; e < PER / 8; ++e)
-    dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+    for (int e = 0; e < PER / 8; ++e)
+      dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+  } else {
+    uint2* dst = reinterpret_cast<uint2*>(p.out + row * D + sub * PER);
+#pragma unroll
+    for (int e = 0; e < PER / 4; ++e) dst[e] = make_uint2(pk[2 * e], pk[2 * e + 1]);
+  }
   if (p.lse != nullptr && sub == 0) p.lse[(long long)bh * p.N + n] = L;
 }
 

@@ -421,7 +421,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   if (e != cudaSuccess) return cuda_fail(e, "bwd_prep_kernel launch");
   int rc = trace_mark(g_trace_begin, stream);
   if (rc != DILATTN_OK) return rc;
-  // persistent: one CTA per SM walks the longest-first unit list with stride gridDim.x
+  // persistent: one CTA per SM, each taking units of the longest-first list from the counter
   p.units = units;
   const long long grid = std::min<long long>(units, (long long)st->num_sms);
   if (grid > 0)

@@ -14,15 +14,18 @@
 // the pattern's normalised output O_i and its log-sum-exp for those rows to
 // an fp32 partial buffer; the merge kernel combines patterns.
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer: Q tile once, then a ring of K/V tiles.
-//   warp 1      TMEM allocator and single-thread MMA issuer:
+// Warp roles (192 threads, two CTAs per SM at d = 64):
+//   warp 0      TMA producer: lane 0 loads the Q tile once, then the K ring;
+//               lane 1 the V ring.
+//   warp 1      TMEM allocator and MMA issuer (the whole warp runs the event
+//               loop, one elected lane issues each group):
 //               S = Q K^T (SMEM x SMEM -> TMEM), O += P V (TMEM x SMEM -> TMEM).
 //   warps 2..5  softmax: warp w takes TMEM lanes 32 (w % 4) .. + 31, one query
 //               row per thread: fp32 row max (3-input max), P = exp2(S*scale - m)
-//               with packed fp32x2 arithmetic (5 of every 8 column pairs on the
-//               MUFU ex2, 3 on an FMA-pipe polynomial), P stored to TMEM as
-//               bf16, O rescaled in TMEM when the reference max moves, epilogue.
+//               with packed fp32x2 arithmetic and the exp2 on the MUFU unit
+//               (DILATTN_FWD_POLY moves a share to an FMA-pipe polynomial), P
+//               stored to TMEM as bf16, O rescaled in TMEM when the reference
+//               max moves, epilogue.
 // Rows are one per thread: at d = 64 the softmax, not the MMA, bounds a tile,
 // so its issue slots are the budget every choice above is made against.
 // TMEM columns: S [0,128), P [128,192) (bf16 pairs), O [192, 192+D).

@@ -53,6 +53,17 @@ def test_bf16_small(pats, causal):
 
 
 @pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,N,H,pats", [
+    (1, 1, 2, [(1, 1)]),                          # one row
+    (1, 127, 2, [(128, 1), (64, 2), (256, 4)]),   # w > N, one partial tile
+    (3, 129, 1, [(128, 1), (129, 3)]),            # a tail of one row past a tile
+    (1, 5, 8, [(5, 8), (4, 1)]),                  # r > N: heads 5..7 keep no rows of (5, 8)
+])
+def test_bf16_edge_sizes(B, N, H, pats, causal):
+    _run_full(B, N, H, 64, pats, causal, "bf16", seed=14)
+
+
+@pytest.mark.parametrize("causal", [True, False])
 def test_f32_small(causal):
     _run_full(1, 600, 3, 64, [(128, 1), (300, 3), (600, 4)], causal, "f32", seed=12)
 

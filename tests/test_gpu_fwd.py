@@ -43,6 +43,22 @@ def test_bf16_small(pats, causal):
     _run_full(2, 1100, 3, 64, pats, causal, "bf16", seed=1)
 
 
+# degenerate sizes: one row; one partial tile with w > N; a tail of one row past
+# a tile; r > N (heads whose offset h mod r is >= N keep no rows at all)
+EDGE = [
+    (1, 1, 2, [(1, 1)]),
+    (1, 127, 2, [(128, 1), (64, 2), (256, 4)]),
+    (3, 129, 1, [(128, 1), (129, 3)]),
+    (1, 5, 8, [(5, 8), (4, 1)]),
+]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("B,N,H,pats", EDGE)
+def test_bf16_edge_sizes(B, N, H, pats, causal):
+    _run_full(B, N, H, 64, pats, causal, "bf16", seed=4)
+
+
 def test_bf16_d128_small():
     _run_full(1, 1536, 4, 128, [(256, 1), (512, 2), (1536, 4)], True, "bf16", seed=2)
 

@@ -99,10 +99,23 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            return
+        # nvidia-smi takes a moment to start: let its first sample land, and
+        # keep only the samples taken after this point (the timed region)
+        self.skip = 0
+        t_end = time.time() + 3.0
+        while time.time() < t_end:
+            self.fh.flush()
+            with open(self.path) as f:
+                n = sum(1 for line in f if line.count(",") >= 8)
+            if n > 0:
+                self.skip = n
+                break
+            time.sleep(0.01)
 
     def stop(self):
         if self.proc is None:
@@ -116,7 +129,9 @@ class ClockSampler:
         self.fh.close()
         rows = []
         with open(self.path) as f:
-            for line in f:
+            for i, line in enumerate(f):
+                if i < self.skip:
+                    continue
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) < 9:
                     continue
@@ -506,7 +521,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))

@@ -180,16 +180,18 @@ __device__ __forceinline__ bool bwd_unit(const BwdParams& p, long long uu, BwdUn
   int a = 0;
   while (a + 1 < p.npat && uu >= p.gstart[a + 1]) ++a;
   const int i = p.gorder[a];
-  long long rem = uu - p.gstart[a];
+  // the host rejects 2^31 units or more: 32-bit unsigned arithmetic (fast divisions)
+  uint32_t rem = (uint32_t)(uu - p.gstart[a]);
   U.g = p.pat[i];
-  U.u = (int)(rem % U.g.ntiles);  // key tile; long (small u) tiles come first
-  rem /= U.g.ntiles;
+  const uint32_t q1 = rem / (uint32_t)U.g.ntiles;
+  U.u = (int)(rem - q1 * (uint32_t)U.g.ntiles);  // key tile; long (small u) tiles come first
   U.wu.pat = i;
   U.wu.t = U.u;
-  U.wu.h = (int)(rem % p.H);
-  rem /= p.H;
-  U.wu.b = (int)(rem % p.B);
-  U.wu.seg = (int)(rem / p.B);
+  const uint32_t q2 = q1 / (uint32_t)p.H;
+  U.wu.h = (int)(q1 - q2 * (uint32_t)p.H);
+  const uint32_t q3 = q2 / (uint32_t)p.B;
+  U.wu.b = (int)(q2 - q3 * (uint32_t)p.B);
+  U.wu.seg = (int)q3;
   U.si = seg_info(U.g, p.N, U.wu.h, U.wu.seg);
   const int nq = (U.si.n + BM - 1) / BM;
   if (U.u >= nq) return false;

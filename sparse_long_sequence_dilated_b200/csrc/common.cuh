@@ -35,14 +35,18 @@ struct SegInfo {
   int off;
 };
 
+// Lengths, offsets and strides are below 2^31 (N and w, r are int), so the
+// division runs in 32-bit unsigned arithmetic, which the GPU does in a few
+// instructions rather than the 64-bit software sequence.
 __host__ __device__ inline SegInfo seg_info(const PatternGeom& g, int N, int h, int s) {
   SegInfo si;
   si.start = (long long)s * g.w;
   long long end = si.start + g.w;
   if (end > N) end = N;
   si.off = h % g.r;
-  long long len = end - si.start;
-  si.n = len > si.off ? (int)((len - si.off + g.r - 1) / g.r) : 0;
+  const int len = (int)(end - si.start);
+  si.n = len > si.off ? (int)(((uint32_t)(len - si.off) + (uint32_t)(g.r - 1)) / (uint32_t)g.r)
+                      : 0;
   return si;
 }
 
@@ -301,38 +305,48 @@ struct TileUnit {
   int pat, seg, b, h, t;
 };
 
+// Unit index -> unit. The host rejects schedules of 2^31 units or more, so
+// every quantity here fits 32-bit unsigned arithmetic (fast divisions).
 __device__ __forceinline__ TileUnit decode_unit(const Sched& sc, const PatternGeom* pat, int B,
-                                                int H, long long u) {
+                                                int H, long long u64) {
+  const uint32_t u = (uint32_t)u64;
   int j = 0;
-  while (j + 1 < sc.nband && u >= sc.start[j + 1]) ++j;
-  const long long u2 = u - sc.start[j];
+  while (j + 1 < sc.nband && u >= (uint32_t)sc.start[j + 1]) ++j;
+  const uint32_t u2 = u - (uint32_t)sc.start[j];
+  const uint32_t per = (uint32_t)sc.per_level[j];
+  const uint32_t lvl = u2 / per;
   TileUnit w;
-  w.t = sc.nt[j] - 1 - (int)(u2 / sc.per_level[j]);
-  long long rem = u2 % sc.per_level[j];
+  w.t = sc.nt[j] - 1 - (int)lvl;
+  uint32_t rem = u2 - lvl * per;
   w.pat = sc.order[0];
   for (int a = 0; a < sc.npat_active[j]; ++a) {
     const int i = sc.order[a];
-    const long long cnt = (long long)pat[i].nseg * B * H;
+    const uint32_t cnt = (uint32_t)pat[i].nseg * (uint32_t)B * (uint32_t)H;
     if (rem < cnt) {
       w.pat = i;
       break;
     }
     rem -= cnt;
   }
-  w.h = (int)(rem % H);
-  rem /= H;
-  w.b = (int)(rem % B);
-  w.seg = (int)(rem / B);
+  const uint32_t bs = rem / (uint32_t)H;
+  w.h = (int)(rem - bs * (uint32_t)H);
+  const uint32_t sg = bs / (uint32_t)B;
+  w.b = (int)(bs - sg * (uint32_t)B);
+  w.seg = (int)sg;
   return w;
 }
 
 // Coordinates of kept row v of a segment in the strided TMA view: the row's
 // position is phase + m * r.
+// Every kept row of a segment has the phase of its row 0 and sits v view rows
+// after it; start + off < N + r < 2^32, so one 32-bit division serves.
 __device__ __forceinline__ void view_coords(const PatternGeom& g, const SegInfo& si, int v,
                                             int& phase, int& m) {
-  const long long pos = si.start + si.off + (long long)v * g.r;
-  phase = (int)(pos % g.r);
-  m = (int)(pos / g.r);
+  const uint32_t base = (uint32_t)(si.start + si.off);
+  const uint32_t r = (uint32_t)g.r;
+  const uint32_t m0 = base / r;
+  phase = (int)(base - m0 * r);
+  m = (int)m0 + v;
 }
 
 // Bounded wait taken by all 32 lanes of a warp, with a warp-uniform result.

@@ -103,6 +103,8 @@ class ClockSampler:
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            self.fh.close()
+            os.unlink(self.path)
             return
         # nvidia-smi takes a moment to start: let its first sample land, and
         # keep only the samples taken after this point (the timed region)

@@ -2,6 +2,8 @@
 
 The record must come from samples taken inside the timed region only, report the
 median SM clock of the samples under load, and name every throttle reason seen."""
+import os
+
 import bench
 
 IDLE = "0, 1005, 1965, 120.50, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active\n"
@@ -63,4 +65,4 @@ def test_missing_nvidia_smi(monkeypatch):
     s.start()
     rec = s.stop()
     assert rec["samples"] == 0 and rec["reasons"] == ["nvidia-smi unavailable"]
-    assert not __import__("os").path.exists(s.path)  # no temporary file left behind
+    assert not os.path.exists(s.path)  # no temporary file left behind

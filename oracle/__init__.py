@@ -8,8 +8,10 @@ from .dilated import (  # noqa: F401
     kept_rows,
     selection_signature,
     fwd,
+    fwd_head,
     fwd_per_pattern,
     bwd,
+    bwd_head,
     fwd_rows,
     bwd_rows,
     multiplicity,

@@ -133,79 +133,135 @@ def fwd_per_pattern(q: np.ndarray, k: np.ndarray, v: np.ndarray,
 # Step 4: merge through the log-sum-exp of the denominators (DarcStar
 # commentary: the shared denominator must stay exact)
 # ---------------------------------------------------------------------------
-def _merge(O_i: np.ndarray, lse_i: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
-    """O = sum_i exp(lse_i - L) O_i with L = log sum_i exp(lse_i).
+def _merge(pieces, lse_i: np.ndarray, N: int, d: int) -> Tuple[np.ndarray, np.ndarray]:
+    """O = sum_i exp(lse_i - L) O_i with L = log sum_i exp(lse_i), for one head.
 
-    exp(lse_i - L) = Z_i / sum_j Z_j = alpha_i. Rows with every lse_i = -inf
-    (selected by no pattern) get L = -inf and O = 0; the -inf - (-inf) case
-    is never evaluated.
+    pieces[i] lists pattern i's (kept rows, O_i rows) per segment; lse_i is
+    [npat, N] with -inf where pattern i keeps no row. exp(lse_i - L) =
+    Z_i / sum_j Z_j = alpha_i. Rows with every lse_i = -inf (selected by no
+    pattern) get L = -inf and O = 0; the -inf - (-inf) case is never
+    evaluated.
     """
-    npat, B, H, N = lse_i.shape
-    mx = lse_i.max(axis=0)                          # [B, H, N]
+    mx = lse_i.max(axis=0)                          # [N]
     sel = np.isfinite(mx)
     mx_safe = np.where(sel, mx, 0.0)
     with np.errstate(invalid="ignore"):
         wts = np.where(sel[None], np.exp(lse_i - mx_safe[None]), 0.0)   # Z_i / exp(mx)
     tot = wts.sum(axis=0)
     L = np.where(sel, mx_safe + np.log(np.where(sel, tot, 1.0)), -np.inf)
-    alpha = np.where(sel[None], wts / np.where(sel, tot, 1.0)[None], 0.0)  # [npat, B, H, N]
-    O = np.einsum("pbhn,pbnhd->bnhd", alpha, O_i)
+    alpha = np.where(sel[None], wts / np.where(sel, tot, 1.0)[None], 0.0)  # [npat, N]
+    O = np.zeros((N, d))
+    for i, segs in enumerate(pieces):
+        for idx, O_seg in segs:
+            O[idx] += alpha[i, idx][:, None] * O_seg
     return O, L
+
+
+def fwd_head(q_h: np.ndarray, k_h: np.ndarray, v_h: np.ndarray, h: int,
+             patterns: Sequence[Pattern], causal: bool = True) -> Tuple[np.ndarray, np.ndarray]:
+    """Merged dilated attention of one (batch, head) slice.
+
+    q_h, k_h, v_h: [N, d]; h is the head index, which selects every pattern's
+    offset h mod r. Returns out [N, d] and lse [N] (float64, natural log).
+    Heads and batches never interact, so this is the whole method for one
+    slice: steps 1-3 per pattern and segment, then the step-4 merge.
+    """
+    q_h = np.asarray(q_h, dtype=np.float64)
+    k_h = np.asarray(k_h, dtype=np.float64)
+    v_h = np.asarray(v_h, dtype=np.float64)
+    N, d = q_h.shape
+    tau = 1.0 / math.sqrt(d)
+    lse_i = np.full((len(patterns), N), -np.inf)
+    pieces = []
+    for i, (w, r) in enumerate(patterns):
+        segs = []
+        for idx in kept_rows(N, w, r, h):
+            if idx.size == 0:
+                continue
+            O, lse = _segment_attention(q_h[idx], k_h[idx], v_h[idx], tau, causal)
+            segs.append((idx, O))
+            lse_i[i, idx] = lse
+        pieces.append(segs)
+    return _merge(pieces, lse_i, N, d)
 
 
 def fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, patterns: Sequence[Pattern],
         causal: bool = True) -> Tuple[np.ndarray, np.ndarray]:
     """Merged dilated attention: out [B, N, H, d] float64, lse [B, H, N] float64 (natural log)."""
-    O_i, lse_i = fwd_per_pattern(q, k, v, patterns, causal)
-    return _merge(O_i, lse_i)
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, N, H, d = q.shape
+    out = np.zeros((B, N, H, d))
+    lse = np.full((B, H, N), -np.inf)
+    for b in range(B):
+        for h in range(H):
+            out[b, :, h], lse[b, h] = fwd_head(q[b, :, h], k[b, :, h], v[b, :, h], h,
+                                               patterns, causal)
+    return out, lse
 
 
 # ---------------------------------------------------------------------------
 # Step 5: backward, recomputing the probabilities from the merged lse
 # ---------------------------------------------------------------------------
-def bwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.ndarray,
-        patterns: Sequence[Pattern], causal: bool = True, out: np.ndarray = None,
-        lse: np.ndarray = None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
-    """Gradients (dq, dk, dv) of sum(out * dout), all [B, N, H, d] float64.
+def bwd_head(q_h: np.ndarray, k_h: np.ndarray, v_h: np.ndarray, do_h: np.ndarray, h: int,
+             patterns: Sequence[Pattern], causal: bool = True, out_h: np.ndarray = None,
+             lse_h: np.ndarray = None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Gradients (dq, dk, dv) [N, d] of sum(out * dout) for one (batch, head) slice.
 
     Because the merged output is one softmax over the multiset union of the
     keys the patterns give a row, the probability of key c for row a under
     pattern i is exp(s_ac - L_a) with the merged L, and
     D_a = sum(dO_a * O_a) is the softmax-backward row term. Per (pattern,
     segment): dV += P^T dO, dP = dO V^T, dS = P * (dP - D), dQ += tau dS K,
-    dK += tau dS^T Q.
+    dK += tau dS^T Q. out_h / lse_h default to this oracle's own forward.
     """
-    q = np.asarray(q, dtype=np.float64)
-    k = np.asarray(k, dtype=np.float64)
-    v = np.asarray(v, dtype=np.float64)
-    dout = np.asarray(dout, dtype=np.float64)
-    if out is None or lse is None:
-        out, lse = fwd(q, k, v, patterns, causal)
-    out = np.asarray(out, dtype=np.float64)
-    lse = np.asarray(lse, dtype=np.float64)
-    B, N, H, d = q.shape
+    q_h = np.asarray(q_h, dtype=np.float64)
+    k_h = np.asarray(k_h, dtype=np.float64)
+    v_h = np.asarray(v_h, dtype=np.float64)
+    do_h = np.asarray(do_h, dtype=np.float64)
+    if out_h is None or lse_h is None:
+        out_h, lse_h = fwd_head(q_h, k_h, v_h, h, patterns, causal)
+    out_h = np.asarray(out_h, dtype=np.float64)
+    lse_h = np.asarray(lse_h, dtype=np.float64)
+    N, d = q_h.shape
     tau = 1.0 / math.sqrt(d)
-    Drow = np.einsum("bnhd,bnhd->bhn", dout, out)
-    dq = np.zeros_like(q)
-    dk = np.zeros_like(k)
-    dv = np.zeros_like(v)
+    Drow = np.einsum("nd,nd->n", do_h, out_h)
+    dq = np.zeros_like(q_h)
+    dk = np.zeros_like(k_h)
+    dv = np.zeros_like(v_h)
     for (w, r) in patterns:
-        for b in range(B):
-            for h in range(H):
-                for idx in kept_rows(N, w, r, h):
-                    if idx.size == 0:
-                        continue
-                    Qs, Ks, Vs, dOs = q[b, idx, h], k[b, idx, h], v[b, idx, h], dout[b, idx, h]
-                    S = tau * (Qs @ Ks.T)
-                    Ls = lse[b, h, idx]
-                    P = np.exp(S - Ls[:, None])
-                    if causal:
-                        P = np.tril(P)
-                    dv[b, idx, h] += P.T @ dOs
-                    dP = dOs @ Vs.T
-                    dS = P * (dP - Drow[b, h, idx][:, None])
-                    dq[b, idx, h] += tau * (dS @ Ks)
-                    dk[b, idx, h] += tau * (dS.T @ Qs)
+        for idx in kept_rows(N, w, r, h):
+            if idx.size == 0:
+                continue
+            Qs, Ks, Vs, dOs = q_h[idx], k_h[idx], v_h[idx], do_h[idx]
+            S = tau * (Qs @ Ks.T)
+            P = np.exp(S - lse_h[idx][:, None])
+            if causal:
+                P = np.tril(P)
+            dv[idx] += P.T @ dOs
+            dP = dOs @ Vs.T
+            dS = P * (dP - Drow[idx][:, None])
+            dq[idx] += tau * (dS @ Ks)
+            dk[idx] += tau * (dS.T @ Qs)
+    return dq, dk, dv
+
+
+def bwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, dout: np.ndarray,
+        patterns: Sequence[Pattern], causal: bool = True, out: np.ndarray = None,
+        lse: np.ndarray = None) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Gradients (dq, dk, dv) of sum(out * dout), all [B, N, H, d] float64 (bwd_head per slice)."""
+    q = np.asarray(q, dtype=np.float64)
+    B, N, H, d = q.shape
+    dq = np.zeros((B, N, H, d))
+    dk = np.zeros((B, N, H, d))
+    dv = np.zeros((B, N, H, d))
+    for b in range(B):
+        for h in range(H):
+            o_h = None if out is None else out[b, :, h]
+            l_h = None if lse is None else lse[b, h]
+            dq[b, :, h], dk[b, :, h], dv[b, :, h] = bwd_head(
+                q[b, :, h], k[b, :, h], v[b, :, h], dout[b, :, h], h, patterns, causal, o_h, l_h)
     return dq, dk, dv
 
 

@@ -373,13 +373,13 @@ def test_planted_global_residue_offset_is_caught(monkeypatch):
 
 def test_planted_unweighted_merge_is_caught(monkeypatch):
     # mistake: average the pattern outputs instead of weighting by Z_i
-    def bad_merge(O_i, lse_i):
-        sel = np.isfinite(lse_i)
-        cnt = sel.sum(axis=0)
-        wts = np.where(sel, 1.0, 0.0) / np.maximum(cnt, 1)[None]
-        O = np.einsum("pbhn,pbnhd->bnhd", wts, O_i)
-        mx = lse_i.max(axis=0)
-        return O, mx
+    def bad_merge(pieces, lse_i, N, d):
+        cnt = np.isfinite(lse_i).sum(axis=0)
+        O = np.zeros((N, d))
+        for segs in pieces:
+            for idx, O_seg in segs:
+                O[idx] += O_seg / np.maximum(cnt[idx], 1)[:, None]
+        return O, lse_i.max(axis=0)
     monkeypatch.setattr(odl, "_merge", bad_merge)
     assert _zero_score_case_fails(odl.fwd)
 

@@ -178,9 +178,27 @@ int dilattn_set_trace_events(cudaEvent_t tile_begin, cudaEvent_t tile_end);
 /*
  * Reads and clears the library's device-side error word on the current
  * device after synchronising `stream`. *code receives 0 when no kernel
- * reported a failure (a bounded wait that ran out sets a nonzero code).
+ * reported a failure, else the code of the last failure (1: a bounded wait
+ * ran out). Every kernel launch carries its own tag, and its waits give up
+ * early only on a failure of that same launch, so a failure that nobody has
+ * read yet does not cut short the work of later calls; it stays readable
+ * until this call clears it. The word's device address is looked up once
+ * per device and cached: it does not survive cudaDeviceReset (nor does the
+ * scratch of dilattn_fwd_noalloc).
  */
 int dilattn_device_error(cudaStream_t stream, int* code);
+
+/*
+ * Self-test of the failure path (no counterpart in the LongNet pages). One
+ * CTA with two warps: warp 0 waits on an mbarrier that nothing ever arrives
+ * on, with a limit of limit_ns (1 .. 10^9); warp 1 waits on another such
+ * barrier with the kernels' ordinary 4 s limit and must give up as soon as
+ * warp 0 raises the CTA's abort flag. The kernel then returns, leaving code 1
+ * in the device error word. result: device int[4], 16-byte aligned:
+ * result[0], result[1] = 1 if warp 0's / warp 1's wait completed (neither may),
+ * else 0; result[2], result[3] = the nanoseconds each waited (capped at 2e9).
+ */
+int dilattn_selftest_wait_timeout(unsigned long long limit_ns, int* result, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

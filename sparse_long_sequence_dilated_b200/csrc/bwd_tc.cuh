@@ -71,7 +71,7 @@ struct BwdParams {
   int* counter;                   // next unit to hand out (zeroed by the preprocess)
   const float* lse;   // [B][H][N] natural log
   const float* drow;  // [B][H][N]
-  int* err;
+  ErrCtx err;  // device error word and this launch's tag
 };
 
 // hi + lo products: 0 never, 1 on the first query tile of a segment, 2 always
@@ -376,9 +376,9 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
     if (!ok && lane == 0) {
       // Drain copies still in flight before the CTA's shared memory goes away.
       volatile int no_abort = 0;
-      if (k > 0) mbar_wait(b_kvfull, (k - 1) & 1, &no_abort, nullptr, 200000000ull);
+      if (k > 0) mbar_wait(b_kvfull, (k - 1) & 1, &no_abort, ErrCtx{}, 200000000ull);
       for (uint32_t g = (gp >= C::QST ? gp - C::QST : 0); g < gp; ++g)
-        mbar_wait(b_qfull(g % C::QST), (g / C::QST) & 1, &no_abort, nullptr, 200000000ull);
+        mbar_wait(b_qfull(g % C::QST), (g / C::QST) & 1, &no_abort, ErrCtx{}, 200000000ull);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       if (elect_one_sync()) mma_commit(b_fin);
       __syncwarp();
       volatile int no_abort = 0;
-      mbar_wait(b_fin, 0, &no_abort, nullptr, 200000000ull);
+      mbar_wait(b_fin, 0, &no_abort, ErrCtx{}, 200000000ull);
     }
     __syncwarp();
   } else {

@@ -96,24 +96,42 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Where a kernel reports a failure: the device error word and this launch's
+// tag. A failure stores (tag << 8) | code. Waits give up early only on a
+// failure carrying their own launch's tag, so an error left unread from an
+// earlier call does not cut short the waits of later calls.
+struct ErrCtx {
+  int* word = nullptr;
+  int tag = 0;
+  __device__ __forceinline__ bool raised() const {
+    if (word == nullptr) return false;
+    const int v = *reinterpret_cast<volatile int*>(word);
+    return v != 0 && (v >> 8) == tag;
+  }
+  __device__ __forceinline__ void raise(int code) const {
+    if (word != nullptr) atomicExch(word, (tag << 8) | code);
+  }
+};
+
 // Bounded wait on an mbarrier phase. Gives up after `limit_ns` of global time,
-// as soon as another warp of the CTA has raised *abort, or once any CTA has
-// recorded an error in the device error word; a timeout records
-// kErrWaitTimeout there and raises *abort.
+// as soon as another warp of the CTA has raised *abort, or once any CTA of the
+// same launch has recorded a failure; a timeout records kErrWaitTimeout and
+// raises *abort.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* err, unsigned long long limit_ns = 4000000000ull) {
+                                          const ErrCtx& err,
+                                          unsigned long long limit_ns = 4000000000ull) {
   if (mbar_try_wait(bar, parity)) return true;
   unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0) {
       if (*abort) return false;
-      if (err != nullptr && *reinterpret_cast<volatile int*>(err) != 0) {
-        *abort = 1;  // another CTA already gave up: stop waiting
+      if (err.raised()) {
+        *abort = 1;  // another CTA of this launch already gave up: stop waiting
         return false;
       }
       if (globaltimer_ns() - t0 > limit_ns) {
-        if (err) atomicExch(err, (int)kErrWaitTimeout);
+        err.raise(kErrWaitTimeout);
         *abort = 1;
         return false;
       }
@@ -351,7 +369,7 @@ __device__ __forceinline__ void view_coords(const PatternGeom& g, const SegInfo&
 
 // Bounded wait taken by all 32 lanes of a warp, with a warp-uniform result.
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                          int* err) {
+                                          const ErrCtx& err) {
   const bool ok = mbar_wait(bar, parity, abort, err);
   return __all_sync(0xffffffffu, ok);
 }
@@ -578,25 +596,25 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 namespace dil {
 // Bookkeeping of a polling loop with the same bounds as mbar_wait: step()
 // returns false once the loop has gone 4 s without progress, another warp of
-// the CTA raised *abort, or any CTA recorded an error in the device word.
+// the CTA raised *abort, or any CTA of the launch recorded a failure.
 struct PollGuard {
   uint32_t spins = 0;
   unsigned long long t0 = 0;
-  __device__ __forceinline__ bool step(bool progressed, volatile int* abort, int* err) {
+  __device__ __forceinline__ bool step(bool progressed, volatile int* abort, const ErrCtx& err) {
     if (progressed) {
       spins = 0;
       t0 = 0;
       return true;
     }
     if ((++spins & 1023u) != 0) return true;
-    if (*abort || *reinterpret_cast<volatile int*>(err) != 0) {
+    if (*abort || err.raised()) {
       *abort = 1;
       return false;
     }
     if (t0 == 0) {
       t0 = globaltimer_ns();
     } else if (globaltimer_ns() - t0 > 4000000000ull) {
-      atomicExch(err, (int)kErrWaitTimeout);
+      err.raise(kErrWaitTimeout);
       *abort = 1;
       return false;
     }

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -22,9 +23,40 @@ namespace dil {
 
 __device__ int g_dev_error;  // device-side error word (bounded waits that ran out)
 
+// Self-test of the failure path: warp 0 waits on an mbarrier that nothing
+// arrives on, with a limit of limit_ns; warp 1 waits on another one with the
+// kernels' ordinary 4 s limit and must give up as soon as warp 0 has raised
+// the CTA's abort flag. result[0], result[1]: 1 if the warp's wait completed
+// (it must not), 0 if it gave up; result[2], result[3]: nanoseconds each
+// warp waited.
+__global__ void selftest_wait_kernel(ErrCtx err, unsigned long long limit_ns, int* result) {
+  __shared__ __align__(8) uint64_t bars[2];
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars[0]), 1);
+    mbar_init(smem_u32(&bars[1]), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) {
+    const unsigned long long t0 = globaltimer_ns();
+    const bool ok = warp == 0
+        ? mbar_wait(smem_u32(&bars[0]), 0, &abort_flag, err, limit_ns)
+        : mbar_wait(smem_u32(&bars[1]), 0, &abort_flag, err);
+    result[warp] = ok ? 1 : 0;
+    result[2 + warp] = (int)min(globaltimer_ns() - t0, 2000000000ull);
+  }
+}
+
 namespace {
 
 thread_local char g_last_error[512] = "";
+
+// Launch tags for the device error word (see ErrCtx): 1 .. 2^23 - 1, cycling.
+std::atomic<unsigned> g_launch_tag{0};
+int next_tag() { return (int)(g_launch_tag.fetch_add(1u) % 0x7FFFFFu) + 1; }
 
 
 int cuda_fail(cudaError_t e, const char* what) {
@@ -298,7 +330,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   const long long rows = make_geoms(B, N, H, w, r, npat, p.pat);
   p.part_o = reinterpret_cast<float*>(ws);
   p.part_lse = reinterpret_cast<float*>((char*)ws + align256((size_t)rows * D * 4));
-  p.err = st->err_word;
+  p.err = ErrCtx{st->err_word, next_tag()};
   {
     int rc = partial_map(p.part_o, rows, D, &p.tm_po);
     if (rc != DILATTN_OK) return rc;
@@ -370,7 +402,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   float* drow = reinterpret_cast<float*>(wsb + 3 * tbytes);
   p.drow = drow;
   p.lse = lse;
-  p.err = st->err_word;
+  p.err = ErrCtx{st->err_word, next_tag()};
   for (int i = 0; i < npat; ++i) {
     const void* src[4] = {q, k, v, dout};
     CUtensorMap* dst[4] = {&p.tmq[i], &p.tmk[i], &p.tmv[i], &p.tmdo[i]};
@@ -675,7 +707,19 @@ int dilattn_device_error(cudaStream_t stream, int* code) {
   const int zero = 0;
   e = cudaMemcpy(st->err_word, &zero, sizeof(int), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemcpy");
-  *code = v;
+  *code = v & 0xff;  // the word holds (launch tag << 8) | code
+  return DILATTN_OK;
+}
+
+int dilattn_selftest_wait_timeout(unsigned long long limit_ns, int* result, cudaStream_t stream) {
+  if (result == nullptr || !aligned16(result) || limit_ns == 0 || limit_ns > 1000000000ull)
+    return DILATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  selftest_wait_kernel<<<1, 64, 0, stream>>>(ErrCtx{st->err_word, next_tag()}, limit_ns, result);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selftest_wait_kernel launch");
   return DILATTN_OK;
 }
 
@@ -688,7 +732,7 @@ namespace dil {
 
 // Scratch of dilattn_fwd_noalloc. In host code this name is only a stand-in
 // for the device array: kernels get the address cudaGetSymbolAddress returns.
-__device__ __align__(256) unsigned char g_noalloc_scratch[DILATTN_NOALLOC_SCRATCH_BYTES];
+static __device__ __align__(256) unsigned char g_noalloc_scratch[DILATTN_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 std::mutex g_noalloc_mu;

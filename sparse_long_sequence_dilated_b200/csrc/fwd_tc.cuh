@@ -55,7 +55,7 @@ struct FwdParams {
   Sched sched;
   float* part_o;    // [rows][D]
   float* part_lse;  // [rows] natural-log lse of each pattern's partial
-  int* err;
+  ErrCtx err;  // device error word and this launch's tag
 };
 
 template <int D>
@@ -176,10 +176,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       if (*abort_flag) {
         // Drain copies still in flight before the CTA's shared memory goes away.
         volatile int no_abort = 0;
-        mbar_wait(b_qfull, 0, &no_abort, nullptr, 200000000ull);
+        mbar_wait(b_qfull, 0, &no_abort, ErrCtx{}, 200000000ull);
         for (int it = issued - C::KST; it < issued; ++it)
           if (it >= 0)
-            mbar_wait(b_kfull(it % C::KST), (it / C::KST) & 1, &no_abort, nullptr, 200000000ull);
+            mbar_wait(b_kfull(it % C::KST), (it / C::KST) & 1, &no_abort, ErrCtx{}, 200000000ull);
       }
     } else if (lane == 1) {
       int ph, m, issued = 0;
@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         volatile int no_abort = 0;
         for (int it = issued - C::VST; it < issued; ++it)
           if (it >= 0)
-            mbar_wait(b_vfull(it % C::VST), (it / C::VST) & 1, &no_abort, nullptr, 200000000ull);
+            mbar_wait(b_vfull(it % C::VST), (it / C::VST) & 1, &no_abort, ErrCtx{}, 200000000ull);
       }
     }
     __syncwarp();

@@ -41,6 +41,7 @@ SIGNATURES = {
     "dilattn_selection": (_i, [_vp, _i, _i, _ip, _ip, _i, _vp]),
     "dilattn_set_trace_events": (_i, [_vp, _vp]),
     "dilattn_device_error": (_i, [_vp, _ip]),
+    "dilattn_selftest_wait_timeout": (_i, [_c.c_ulonglong, _vp, _vp]),
 }
 
 _lib = None
@@ -218,6 +219,15 @@ def device_error(stream=None) -> int:
     rc = load().dilattn_device_error(_stream_handle(stream), _c.byref(code))
     _check(rc, "dilattn_device_error")
     return int(code.value)
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None):
+    """Run the failure-path self-test; returns the device int[4] result tensor."""
+    torch = _torch()
+    res = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    rc = load().dilattn_selftest_wait_timeout(int(limit_ns), res.data_ptr(), _stream_handle(stream))
+    _check(rc, "dilattn_selftest_wait_timeout")
+    return res
 
 
 def set_trace_events(begin=None, end=None):

@@ -32,6 +32,13 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, name), name
 
 
+def test_noalloc_scratch_constant_matches_header():
+    text = open(HEADER, encoding="utf-8").read()
+    m = re.search(r"#define DILATTN_NOALLOC_SCRATCH_BYTES \((\d+)u \* 1024u \* 1024u\)", text)
+    assert m is not None
+    assert dilattn.NOALLOC_SCRATCH_BYTES == int(m.group(1)) * 1024 * 1024
+
+
 def test_status_strings():
     assert dilattn.status_string(0) == "DILATTN_OK"
     assert dilattn.status_string(4) == "DILATTN_ERR_WORKSPACE"

@@ -1,8 +1,8 @@
 """GPU parity of the forward pass against the float64 oracle (same seeded inputs).
 
-Sizes the oracle finishes in seconds cover several tiles and ragged tails in
-full; the full-size workloads are checked on sampled rows the oracle computes
-one by one, with the same launch configuration the benchmark times.
+Sizes the oracle finishes in seconds cover several tiles, ragged tails and
+degenerate shapes in full; the full-size workloads are compared element by
+element in tests/test_gpu_scale.py.
 """
 import numpy as np
 import pytest
@@ -78,9 +78,8 @@ def test_unselected_rows_zero():
     check_lse(to_f64(lse), want_l, 2e-2)
 
 
-@pytest.mark.parametrize("name", ["longnet_base_32k", "train_check_2k"])
-def test_workload_full(name):
-    wl = WORKLOADS[name]
+def test_train_check_workload_full():
+    wl = WORKLOADS["train_check_2k"]
     _run_full(wl.B, wl.N, wl.H, wl.d, wl.patterns, wl.causal, wl.dtype, wl.seed)
 
 
@@ -93,33 +92,3 @@ def test_selection_bit_exact(N, H, pats):
     sig = dilattn.selection(N, H, pats).cpu().numpy().view(np.uint32)
     want = oracle.selection_signature(N, H, pats)
     assert np.array_equal(sig, want)
-
-
-def _sampled_rows(B, N, H, n_rows, seed):
-    rng = np.random.default_rng(seed)
-    rows = set()
-    for n in (0, 1, N - 1, N - 2, N // 2):
-        for h in (0, H - 1):
-            rows.add((0, h, n))
-    while len(rows) < n_rows:
-        rows.add((int(rng.integers(0, B)), int(rng.integers(0, H)), int(rng.integers(0, N))))
-    return sorted(rows)
-
-
-@pytest.mark.parametrize("name", ["sweep_131072", "sweep_1048576", "wide_128k"])
-def test_workload_sampled(name):
-    wl = WORKLOADS[name]
-    inp = make_inputs(wl.B, wl.N, wl.H, wl.d, wl.seed, wl.dtype)
-    q, k, v = to_device(inp)
-    out, lse = dilattn.fwd(q, k, v, wl.patterns, wl.causal)
-    torch.cuda.synchronize()
-    assert dilattn.device_error() == 0
-    rows = _sampled_rows(wl.B, wl.N, wl.H, 48, 7)
-    want_o, want_l = oracle.fwd_rows(inp["q"], inp["k"], inp["v"], wl.patterns, rows, wl.causal)
-    idx_b = torch.tensor([r[0] for r in rows])
-    idx_h = torch.tensor([r[1] for r in rows])
-    idx_n = torch.tensor([r[2] for r in rows])
-    got_o = to_f64(out.cpu()[idx_b, idx_n, idx_h])
-    got_l = to_f64(lse.cpu()[idx_b, idx_h, idx_n])
-    check_close(got_o, want_o, "bf16", name)
-    check_lse(got_l, want_l, 2e-2, name)

@@ -1,0 +1,94 @@
+"""Full-size GPU parity: every output element against the float64 oracle.
+
+The CUDA path runs each workload exactly as the benchmark launches it; the
+oracle then runs over (batch, head) slices in parallel worker processes
+(tests/oracle_pool.py) and every element of out, lse, dq, dk and dv is
+compared under the stated bounds (bf16: max-abs <= 2e-2 and relative L2 <=
+5e-3 per tensor; lse: the -inf pattern exactly, max-abs <= 2e-2).
+
+Covered in full, forward and backward: the length sweep at N = 8192, 32768,
+131072 and 262144, the LongNet-base layer (N = 32768, r up to 12) and the
+training step at its timed size (B = 4, N = 32768). Covered in full, forward:
+the length sweep at N = 1048576. The wide d = 128 model (B = 2, N = 131072,
+H = 32) is compared on a declared subset of whole (batch, head) slices,
+exact for those slices.
+"""
+import numpy as np
+import pytest
+import torch
+
+from sparse_long_sequence_dilated_b200 import dilattn
+from sparse_long_sequence_dilated_b200.workloads import WORKLOADS, make_inputs
+from tests import oracle_pool
+
+pytestmark = pytest.mark.gpu
+
+# declared (batch, head) slices of the wide model: both batches and eight heads
+# spread over the offsets h mod r of every dilation r = 2 .. 64
+WIDE_PAIRS = [(b, h) for b in (0, 1) for h in (0, 1, 6, 8, 13, 22, 27, 31)]
+
+
+def _bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _inputs(wl, names):
+    inp = make_inputs(wl.B, wl.N, wl.H, wl.d, wl.seed, wl.dtype, names)
+    return {n: inp[n + "_bits"] for n in names}
+
+
+def _dev(bits):
+    return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _report(name, summ):
+    print(name, {k: (f"{a:.3e}", None if r is None else f"{r:.3e}") for k, (a, r) in summ.items()})
+
+
+@pytest.mark.parametrize("name", ["sweep_8192", "sweep_32768", "sweep_131072", "sweep_262144",
+                                  "longnet_base_32k", "train_b4_32k"])
+def test_full_forward_backward(name):
+    wl = WORKLOADS[name]
+    names = ("q", "k", "v", "dout")
+    bits = _inputs(wl, names)
+    q, k, v, do = (_dev(bits[n]) for n in names)
+    ws = torch.empty(dilattn.fwd_workspace_size(wl.B, wl.N, wl.H, wl.d, wl.patterns),
+                     dtype=torch.uint8, device="cuda")
+    out, lse = dilattn.fwd(q, k, v, wl.patterns, wl.causal, workspace=ws)
+    dq, dk, dv = dilattn.bwd(q, k, v, out, lse, do, wl.patterns, wl.causal, fwd_workspace=ws)
+    # the plain convention: D from the bf16 out the forward returned
+    nq, nk, nv = dilattn.bwd(q, k, v, out, lse, do, wl.patterns, wl.causal)
+    torch.cuda.synchronize()
+    assert dilattn.device_error() == 0
+    got = {"out": _bits(out), "lse": lse.cpu().numpy(), "dq": _bits(dq), "dk": _bits(dk),
+           "dv": _bits(dv), "dq@bf16_out": _bits(nq), "dk@bf16_out": _bits(nk),
+           "dv@bf16_out": _bits(nv)}
+    del q, k, v, do, out, lse, dq, dk, dv, nq, nk, nv, ws
+    torch.cuda.empty_cache()
+    stats = oracle_pool.run("bwd", bits, got, wl.patterns, wl.causal)
+    _report(name, oracle_pool.check(stats, "bf16", 2e-2, name))
+
+
+def _forward_only(wl, pairs=None):
+    names = ("q", "k", "v")
+    bits = _inputs(wl, names)
+    q, k, v = (_dev(bits[n]) for n in names)
+    out, lse = dilattn.fwd(q, k, v, wl.patterns, wl.causal)
+    torch.cuda.synchronize()
+    assert dilattn.device_error() == 0
+    got = {"out": _bits(out), "lse": lse.cpu().numpy()}
+    del q, k, v, out, lse
+    torch.cuda.empty_cache()
+    stats = oracle_pool.run("fwd", bits, got, wl.patterns, wl.causal, pairs)
+    if pairs is not None:
+        assert all(len(v) == len(pairs) for v in stats.values())
+    _report(wl.name, oracle_pool.check(stats, "bf16", 2e-2, wl.name))
+
+
+def test_full_forward_1m():
+    _forward_only(WORKLOADS["sweep_1048576"])
+
+
+def test_wide_forward_declared_heads():
+    assert len(set(WIDE_PAIRS)) == len(WIDE_PAIRS)
+    _forward_only(WORKLOADS["wide_128k"], WIDE_PAIRS)

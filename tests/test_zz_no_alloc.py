@@ -6,8 +6,9 @@ start-up and forbids cudaMalloc afterwards. For them the library keeps the
 forward's scratch (per-pattern partial results) in a fixed 64 MiB array of its
 own. These tests run that entry point through the C ABI and compare it with
 dilattn_fwd, which uses a caller workspace, on two calls in a row with
-different inputs, so scratch left over from the first call would show up in
-the second; and they check that a problem too large for the array is refused.
+different shapes, patterns and inputs, so scratch read from the wrong place
+or left over from the first call would show up in the second; and they check
+that a problem too large for the array is refused.
 
 This file is named to be collected last: a failure here stops a -x run only
 after every other test has run.
@@ -36,23 +37,31 @@ def _noalloc(q, k, v, out, lse, pats):
     assert rc == 0, (dilattn.status_string(rc), dilattn.last_error())
 
 
+# two problems with different scratch layouts: the second call reuses the
+# array with other pattern counts, segment sizes and row offsets, so an entry
+# read from the wrong place (or left over from the first call) shows up
+CALLS = [
+    (2, 2048, 8, PATS, 21),
+    (1, 3000, 6, [(300, 1), (700, 3), (3000, 5)], 22),
+]
+
+
 @pytest.mark.parametrize("d", [64, 128])
 def test_noalloc_matches_workspace_forward_on_two_calls(d):
-    B, N, H = 2, 2048, 8
-    assert dilattn.fwd_workspace_size(B, N, H, d, PATS) <= dilattn.NOALLOC_SCRATCH_BYTES
     calls = []
-    for seed in (21, 22):
+    for B, N, H, pats, seed in CALLS:
+        assert dilattn.fwd_workspace_size(B, N, H, d, pats) <= dilattn.NOALLOC_SCRATCH_BYTES
         q, k, v = to_device(make_inputs(B, N, H, d, seed, "bf16"))
         out = torch.empty_like(q)
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-        calls.append((q, k, v, out, lse))
-    # two calls in a row on the shared scratch, different inputs
-    for q, k, v, out, lse in calls:
-        _noalloc(q, k, v, out, lse, PATS)
+        calls.append((q, k, v, out, lse, pats))
+    # two calls in a row on the shared scratch
+    for q, k, v, out, lse, pats in calls:
+        _noalloc(q, k, v, out, lse, pats)
     torch.cuda.synchronize()
     assert dilattn.device_error() == 0
-    for q, k, v, out, lse in calls:
-        ref_o, ref_l = dilattn.fwd(q, k, v, PATS, True)
+    for q, k, v, out, lse, pats in calls:
+        ref_o, ref_l = dilattn.fwd(q, k, v, pats, True)
         torch.cuda.synchronize()
         check_close(to_f64(out), to_f64(ref_o), "bf16", "out vs dilattn_fwd")
         check_lse(to_f64(lse), to_f64(ref_l), 2e-2, "lse vs dilattn_fwd")

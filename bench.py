@@ -2,11 +2,13 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step is the whole hot path on one batch: dilattn_fwd (tile kernel +
-merge) then dilattn_bwd (preprocess + tile kernel + convert) on B=1,
-N=32768, H=12, d=64 bf16 inputs with patterns w = 2048..32768,
-r = 1, 2, 4, 6, 12, causal. Effective FLOPs count only the nonzero pairs of
-the causal sparse mask: 4 d per pair forward, 10 d backward.
+One step is the whole hot path on one batch: dilattn_fwd_train (tile kernel
+with the cross-pattern merge fused into the r = 1 pattern's tiles; out and its
+rounding residual) then dilattn_bwd (preprocess + tile kernel, fp32
+gradients) on B=1, N=32768, H=12, d=64
+bf16 inputs with patterns w = 2048..32768, r = 1, 2, 4, 6, 12, causal.
+Effective FLOPs count only the nonzero pairs of the causal sparse mask: 4 d
+per pair forward, 10 d backward.
 
 Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush
 (a 256 MB device write, outside the step's events) and timed with CUDA
@@ -17,21 +19,34 @@ the library's trace hook for the roofline line. e2e repeats the step through
 the public API with the step's inputs copied from pinned host memory and the
 results copied back inside the timed region; copy-in, compute and copy-out of
 consecutive steps overlap on three streams (two device buffer sets), as a
-training loop with a prefetching data loader would run them.
+training loop with a prefetching data loader would run them. Clocks are
+sampled through NVML every few milliseconds during the timed steps.
 
---impl reference times the float64 CPU oracle instead (rank 0 only), each
-step a bounded sample of the same workload: the first N' positions of head 0.
+The JSON detail adds the other workloads the metric is quoted on: the
+training step at B = 4, N = 32768 (forward + backward), the length sweep
+N = 8K .. 1M (forward + backward), the wide d = 128 forward, and the N = 8K
+step replayed back to back from a CUDA graph.
+
+cpu_baseline: the float64 CPU oracle on the whole LongNet-base layer, one
+worker process per (batch, head) slice, one BLAS thread each, on the host's
+cores, plus the one-core figures.
+
+--impl reference times that oracle instead (rank 0 only), each step a bounded
+sample of the same workload: every head, positions [0, N') with N' sized so
+that the run takes a few minutes.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
 import json
+import multiprocessing as mp
 import os
 import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -49,6 +64,9 @@ PEAK_FALLBACK = {"bf16_tflops": 1590.0, "hbm_gbs": 6650.0}
 KERNEL_SOURCES = {"fwd_tile_kernel": ("common.cuh", "fwd_tc.cuh"),
                   "bwd_tile_kernel": ("common.cuh", "bwd_tc.cuh")}
 NAMES = ("q", "k", "v", "dout")
+# kernels of the library launched per step of a family with an r = 1 pattern:
+# fwd_tile_kernel, bwd_prep_kernel, bwd_tile_kernel
+LAUNCHES_PER_STEP = 3
 
 
 def kernel_source_hash(kernel: str) -> str:
@@ -84,7 +102,69 @@ def load_traffic(kernel: str, workload: str):
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
+REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+def _summarise(rows, all_rows=None):
+    """rows: (sm_mhz, max_mhz, power_w, set of reasons) taken in the timed region."""
+    all_rows = all_rows if all_rows is not None else rows
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    return {"sm_mhz": statistics.median(r[0] for r in rows),
+            "sm_max_mhz": max(r[1] for r in all_rows),
+            "reasons": sorted(set().union(*[r[3] for r in rows])),
+            "samples": len(rows), "power_w_max": max(r[2] for r in all_rows)}
+
+
+class NvmlClockSampler:
+    """SM clock, power and throttle reasons read through NVML by a background
+    thread every `interval` seconds, from start() to stop()."""
+
+    def __init__(self, gpu_index: str, interval: float = 0.002):
+        self.gpu = int(gpu_index)
+        self.interval = interval
+        self.rows = []
+        self.source = "nvml"
+
+    def start(self):
+        import pynvml
+        pynvml.nvmlInit()
+        self.nv = pynvml
+        self.h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.bits = {"sw_power_cap": pynvml.nvmlClocksThrottleReasonSwPowerCap,
+                     "hw_slowdown": pynvml.nvmlClocksThrottleReasonHwSlowdown,
+                     "hw_thermal_slowdown": pynvml.nvmlClocksThrottleReasonHwThermalSlowdown,
+                     "sw_thermal_slowdown": pynvml.nvmlClocksThrottleReasonSwThermalSlowdown}
+        self.stop_ev = threading.Event()
+        self.sample()  # one sample before the thread starts, so even a short region has one
+        self.th = threading.Thread(target=self._loop, daemon=True)
+        self.th.start()
+
+    def sample(self):
+        nv, h = self.nv, self.h
+        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        self.rows.append((sm, self.max_mhz, pw, {n for n, b in self.bits.items() if rs & b}))
+
+    def _loop(self):
+        while not self.stop_ev.is_set():
+            self.sample()
+            time.sleep(self.interval)
+
+    def stop(self):
+        self.stop_ev.set()
+        self.th.join(timeout=5)
+        self.sample()
+        self.nv.nvmlShutdown()
+        rec = _summarise(self.rows)
+        rec["source"] = "nvml, every 2 ms"
+        return rec
+
+
 class ClockSampler:
+    """nvidia-smi -lms 50 in the background; only samples taken after start() count."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -138,90 +218,181 @@ class ClockSampler:
                 if len(parts) < 9:
                     continue
                 try:
-                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+                    rows.append((float(parts[1]), float(parts[2]), float(parts[3]),
+                                 {REASONS[j] for j, v in enumerate(parts[5:9]) if v == "Active"}))
                 except ValueError:
                     continue
         os.unlink(self.path)
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         loaded = [r for r in rows if r[2] > 250.0] or rows
-        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3]) if v == "Active"})
-        return {"sm_mhz": statistics.median(r[0] for r in loaded),
-                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
-                "samples": len(loaded), "power_w_max": max(r[2] for r in rows)}
+        rec = _summarise(loaded, rows)
+        rec["source"] = "nvidia-smi, every 50 ms"
+        return rec
 
 
-# ---------------------------------------------------------------------------
-# CPU oracle legs
-# ---------------------------------------------------------------------------
-def blas_threads() -> int:
+def make_clock_sampler(gpu_index: str):
     try:
-        import threadpoolctl
-        info = threadpoolctl.threadpool_info()
-        return max([i.get("num_threads", 1) for i in info] or [1])
+        import pynvml
+        pynvml.nvmlInit()
+        pynvml.nvmlShutdown()
+        return NvmlClockSampler(gpu_index)
     except Exception:
+        return ClockSampler(gpu_index)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs: one worker process per (batch, head) slice
+# ---------------------------------------------------------------------------
+def usable_cpus() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
         return os.cpu_count() or 1
 
 
-def oracle_sample(wl, n_prefix: int):
-    """The oracle forward + backward on head 0 of the first n_prefix positions.
-
-    Returns (seconds, effective FLOPs of the sample)."""
+def _oracle_task(args):
+    """Worker: the oracle forward (+ backward) of one slice; returns compute seconds."""
+    q, k, v, do, h, patterns, causal = args
     import oracle
-    inp = make_inputs(1, n_prefix, 1, wl.d, wl.seed, wl.dtype, NAMES)
     t0 = time.perf_counter()
-    out, lse = oracle.fwd(inp["q"], inp["k"], inp["v"], wl.patterns, wl.causal)
-    oracle.bwd(inp["q"], inp["k"], inp["v"], inp["dout"], wl.patterns, wl.causal, out=out, lse=lse)
-    dt = time.perf_counter() - t0
-    work = (flops.fwd_flops(1, n_prefix, 1, wl.d, wl.patterns, wl.causal)
-            + flops.bwd_flops(1, n_prefix, 1, wl.d, wl.patterns, wl.causal))
-    return dt, work
+    out, lse = oracle.fwd_head(q, k, v, h, patterns, causal)
+    if do is not None:
+        oracle.bwd_head(q, k, v, do, h, patterns, causal, out, lse)
+    return time.perf_counter() - t0
+
+
+def _noop(_):
+    return 0
+
+
+class OraclePool:
+    """Spawn-started workers with one BLAS thread each (never forked: the parent
+    may hold a CUDA context)."""
+
+    def __init__(self, nproc: int):
+        keys = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+        old = {k_: os.environ.get(k_) for k_ in keys}
+        for k_ in keys:
+            os.environ[k_] = "1"
+        try:
+            self.pool = mp.get_context("spawn").Pool(nproc)
+        finally:
+            for k_, v_ in old.items():
+                if v_ is None:
+                    os.environ.pop(k_, None)
+                else:
+                    os.environ[k_] = v_
+        self.nproc = nproc
+        self.pool.map(_noop, range(nproc))  # workers started and warm before any timing
+        self.pool.map(_oracle_task, [_tiny_task()] * nproc)  # oracle and numpy imported
+
+    def run(self, wl, n_prefix: int, with_bwd: bool, seed: int = 0):
+        """Oracle over every (batch, head) slice of positions [0, n_prefix).
+
+        Returns (wall seconds, sum of per-slice compute seconds, effective FLOPs)."""
+        names = NAMES if with_bwd else NAMES[:3]
+        inp = make_inputs(wl.B, n_prefix, wl.H, wl.d, seed, wl.dtype, names)
+        tasks = [(inp["q"][b, :, h], inp["k"][b, :, h], inp["v"][b, :, h],
+                  inp["dout"][b, :, h] if with_bwd else None, h,
+                  tuple(map(tuple, wl.patterns)), wl.causal)
+                 for b in range(wl.B) for h in range(wl.H)]
+        t0 = time.perf_counter()
+        secs = self.pool.map(_oracle_task, tasks, chunksize=1)
+        wall = time.perf_counter() - t0
+        work = flops.fwd_flops(wl.B, n_prefix, wl.H, wl.d, wl.patterns, wl.causal)
+        if with_bwd:
+            work += flops.bwd_flops(wl.B, n_prefix, wl.H, wl.d, wl.patterns, wl.causal)
+        return wall, sum(secs), work
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+def _tiny_task():
+    import numpy as np
+    z = np.zeros((4, 8))
+    return (z, z, z, z, 0, ((4, 1),), True)
+
+
+def affinity_note() -> str:
+    try:
+        return ",".join(str(c) for c in sorted(os.sched_getaffinity(0)))
+    except AttributeError:
+        return "n/a"
 
 
 def cpu_baseline(wl):
-    dt, work = oracle_sample(wl, wl.N)
-    return {"value": work / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-            "sample": f"float64 oracle fwd+bwd, batch 0 head 0 of {wl.name} (N={wl.N}, all "
-                      f"{len(wl.patterns)} patterns): {work:.3e} effective FLOP in {dt:.2f} s"}
+    """The oracle on the whole workload over its (batch, head) slices, one process per
+    core, plus one-core figures (a slice's own compute time, and the tiny fp32 case)."""
+    import threadpoolctl
+
+    import oracle
+    nslices = wl.B * wl.H
+    nproc = max(1, min(nslices, usable_cpus()))
+    pool = OraclePool(nproc)
+    try:
+        wall, cpu_s, work = pool.run(wl, wl.N, wl.backward, wl.seed)
+    finally:
+        pool.close()
+    tiny = WORKLOADS["tiny_f32"]
+    ti = make_inputs(tiny.B, tiny.N, tiny.H, tiny.d, tiny.seed, tiny.dtype)
+    with threadpoolctl.threadpool_limits(1):
+        t0 = time.perf_counter()
+        oracle.fwd(ti["q"], ti["k"], ti["v"], tiny.patterns, tiny.causal)
+        t_tiny = time.perf_counter() - t0
+    tiny_work = flops.fwd_flops(tiny.B, tiny.N, tiny.H, tiny.d, tiny.patterns, tiny.causal)
+    what = "fwd+bwd" if wl.backward else "fwd"
+    return {"value": work / wall / 1e12, "unit": UNIT, "cores": nproc, "kind": "oracle",
+            "sample": f"float64 oracle {what} of all {nslices} (batch, head) slices of {wl.name} "
+                      f"(the whole workload), one spawn-started process per slice, {nproc} at "
+                      f"a time, one BLAS thread each: {work:.3e} effective FLOP in {wall:.2f} s",
+            "os_cpu_count": os.cpu_count(), "affinity": affinity_note(),
+            "one_core": {"per_slice_tflops": work / cpu_s / 1e12,
+                         "note": f"{wl.name} {what}: the slices' own compute seconds, each on one "
+                                 f"core ({cpu_s:.2f} s in all)",
+                         "tiny_f32_fwd_tflops": tiny_work / t_tiny / 1e12,
+                         "tiny_f32_fwd_s": t_tiny}}
 
 
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
     wl = WORKLOADS[args.workload]
-    # size each step so that warm-up + timed steps take about two minutes
-    budget_s = 120.0 / max(1, args.steps + args.warmup)
-    cal_n = min(wl.N, 4096)
-    dt, _ = oracle_sample(wl, cal_n)
-    n_prefix = int(min(wl.N, max(2048, cal_n * budget_s / max(dt, 1e-3))))
-    n_prefix = max(2048, (n_prefix // 2048) * 2048)
-    for _ in range(args.warmup):
-        oracle_sample(wl, n_prefix)
-    tot_t, tot_w = 0.0, 0
-    for _ in range(args.steps):
-        dt, w = oracle_sample(wl, n_prefix)
-        tot_t += dt
-        tot_w += w
+    nproc = max(1, min(wl.B * wl.H, usable_cpus()))
+    pool = OraclePool(nproc)
+    try:
+        # size each step so that warm-up + timed steps take about three minutes
+        budget_s = 180.0 / max(1, args.steps + args.warmup)
+        cal_n = min(wl.N, 4096)
+        wall, _, _ = pool.run(wl, cal_n, wl.backward, wl.seed)
+        n_prefix = int(min(wl.N, max(2048, cal_n * budget_s / max(wall, 1e-3))))
+        n_prefix = max(2048, (n_prefix // 2048) * 2048)
+        for _ in range(args.warmup):
+            pool.run(wl, n_prefix, wl.backward, wl.seed)
+        tot_t, tot_w = 0.0, 0
+        for _ in range(args.steps):
+            wall, _, w = pool.run(wl, n_prefix, wl.backward, wl.seed)
+            tot_t += wall
+            tot_w += w
+    finally:
+        pool.close()
     value = tot_w / tot_t / 1e12
-    sample = (f"float64 oracle fwd+bwd on head 0, positions [0, {n_prefix}) of {wl.name} "
-              f"(same patterns), one sample per step")
+    what = "fwd+bwd" if wl.backward else "fwd"
+    sample = (f"float64 oracle {what} of every (batch, head) slice, positions [0, {n_prefix}) of "
+              f"{wl.name} (same patterns), one spawn-started process per slice on {nproc} cores")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
             "config": {"workload": wl.name, "B": wl.B, "N": wl.N, "H": wl.H, "d": wl.d,
                        "patterns": [list(p) for p in wl.patterns], "causal": wl.causal},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
-                             "kind": "oracle", "sample": sample},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nproc, "kind": "oracle",
+                             "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-# ---------------------------------------------------------------------------
-# GPU leg
-# ---------------------------------------------------------------------------
 # ---------------------------------------------------------------------------
 # multi-rank host logic (one process per GPU; also run with gloo on CPU in tests)
 # ---------------------------------------------------------------------------
@@ -246,79 +417,151 @@ def job_tflops(world: int, work_per_rank: float, ms: float, calls: int = 1) -> f
     return world * work_per_rank * calls / (ms * 1e-3) / 1e12
 
 
-SWEEP = ("sweep_8192", "sweep_131072", "sweep_1048576")  # the length sweep, fwd + bwd
-WIDE = "wide_128k"                                         # d = 128, forward
+# ---------------------------------------------------------------------------
+# GPU detail: the other workloads of the metric
+# ---------------------------------------------------------------------------
+SWEEP = ("sweep_8192", "sweep_32768", "sweep_131072", "sweep_262144", "sweep_1048576")
+TRAIN = "train_b4_32k"                                      # B = 4 training step, fwd + bwd
+WIDE = "wide_128k"                                          # d = 128, forward
 
 
-def sweep_detail(dilattn, dev, steps: int = 3, warmup: int = 2):
-    """Tile-kernel and whole-call times for the length sweep (N = 8K, 128K, 1M; fwd + bwd)
-    and the wide d = 128 forward, each on i.i.d. N(0, 1) bf16 inputs drawn on the device
-    (the kernels' cost does not depend on the values), L2 flushed before every call."""
+def time_workload(dilattn, dev, name: str, flush_buf, peak: float, steps: int = 3,
+                  warmup: int = 2):
+    """Whole-call and tile-kernel times of one workload on i.i.d. N(0, 1) bf16 inputs
+    drawn on the device (the kernels' cost does not depend on the values), L2
+    flushed before every call; medians of `steps` timed calls after `warmup`."""
     import torch
 
+    wl = WORKLOADS[name]
+    B, N, H, d, pats = wl.B, wl.N, wl.H, wl.d, wl.patterns
     gen = torch.Generator(device=dev)
     gen.manual_seed(0)
-    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    q, k, v, do = (torch.randn((B, N, H, d), generator=gen, device=dev, dtype=torch.float32)
+                   .to(torch.bfloat16) for _ in range(4))
+    with_bwd = wl.backward and d == 64
+    ws_b = torch.empty(max(dilattn.bwd_workspace_size(B, N, H, d), 256), dtype=torch.uint8,
+                       device=dev) if with_bwd else None
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    res = []
-    for name in SWEEP + (WIDE,):
-        wl = WORKLOADS[name]
-        B, N, H, d, pats = wl.B, wl.N, wl.H, wl.d, wl.patterns
-        t = [torch.randn((B, N, H, d), generator=gen, device=dev, dtype=torch.float32)
-             .to(torch.bfloat16) for _ in range(4)]
-        q, k, v, do = t
-        ws_f = torch.empty(dilattn.fwd_workspace_size(B, N, H, d, pats), dtype=torch.uint8,
-                           device=dev)
-        with_bwd = wl.backward and d == 64
-        tiles = [ev() for _ in range(4)]
-        for e in tiles:
-            e.record()
-        ftile, btile, fwhole, bwhole = [], [], [], []
-        for i in range(warmup + steps):
-            a, b, c = ev(), ev(), ev()
-            flush_buf.fill_(1)
-            a.record()
-            dilattn.set_trace_events(tiles[0], tiles[1])
-            out, lse = dilattn.fwd(q, k, v, pats, wl.causal, workspace=ws_f)
-            b.record()
-            if with_bwd:
-                dilattn.set_trace_events(tiles[2], tiles[3])
-                dilattn.bwd(q, k, v, out, lse, do, pats, wl.causal, fwd_workspace=ws_f)
-            c.record()
-            dilattn.set_trace_events(None, None)
-            torch.cuda.synchronize()
-            if i >= warmup:
-                ftile.append(tiles[0].elapsed_time(tiles[1]))
-                fwhole.append(a.elapsed_time(b))
-                if with_bwd:
-                    btile.append(tiles[2].elapsed_time(tiles[3]))
-                    bwhole.append(b.elapsed_time(c))
-        fw = flops.fwd_flops(B, N, H, d, pats, wl.causal)
-        ent = {"workload": name, "B": B, "N": N, "H": H, "d": d,
-               "fwd_tile_ms": statistics.median(ftile), "fwd_ms": statistics.median(fwhole),
-               "fwd_tile_tflops": fw / statistics.median(ftile) / 1e9,
-               "fwd_tflops": fw / statistics.median(fwhole) / 1e9}
+    tiles = [ev() for _ in range(4)]
+    for e in tiles:
+        e.record()
+    ftile, btile, fwhole, bwhole = [], [], [], []
+    for i in range(warmup + steps):
+        a, b, c = ev(), ev(), ev()
+        flush_buf.fill_(1)
+        a.record()
+        dilattn.set_trace_events(tiles[0], tiles[1])
         if with_bwd:
-            bw = flops.bwd_flops(B, N, H, d, pats, wl.causal)
-            ent.update({"bwd_tile_ms": statistics.median(btile), "bwd_ms": statistics.median(bwhole),
-                        "bwd_tile_tflops": bw / statistics.median(btile) / 1e9,
-                        "step_tflops": (fw + bw) / (statistics.median(fwhole)
-                                                    + statistics.median(bwhole)) / 1e9,
-                        "tokens_per_s": B * N / ((statistics.median(fwhole)
-                                                  + statistics.median(bwhole)) * 1e-3)})
-        res.append(ent)
-        del q, k, v, do, t, ws_f
-        torch.cuda.empty_cache()
-    if dilattn.device_error() != 0:
-        raise RuntimeError("a kernel reported a device-side error in the length sweep")
-    return res
+            out, lse, res = dilattn.fwd_train(q, k, v, pats, wl.causal)
+        else:
+            out, lse = dilattn.fwd(q, k, v, pats, wl.causal)
+        b.record()
+        if with_bwd:
+            dilattn.set_trace_events(tiles[2], tiles[3])
+            dilattn.bwd(q, k, v, out, lse, do, pats, wl.causal, out_res=res, workspace=ws_b)
+        c.record()
+        dilattn.set_trace_events(None, None)
+        torch.cuda.synchronize()
+        if i >= warmup:
+            ftile.append(tiles[0].elapsed_time(tiles[1]))
+            fwhole.append(a.elapsed_time(b))
+            if with_bwd:
+                btile.append(tiles[2].elapsed_time(tiles[3]))
+                bwhole.append(b.elapsed_time(c))
+    fw = flops.fwd_flops(B, N, H, d, pats, wl.causal)
+    fm = statistics.median(fwhole)
+    ent = {"workload": name, "B": B, "N": N, "H": H, "d": d, "npat": len(pats),
+           "fwd_ms": fm, "fwd_tflops": fw / fm / 1e9, "fwd_frac_of_peak": fw / fm / 1e9 / peak,
+           "fwd_tokens_per_s": B * N / (fm * 1e-3),
+           "fwd_tile_ms": statistics.median(ftile),
+           "fwd_tile_tflops": fw / statistics.median(ftile) / 1e9}
+    if with_bwd:
+        bw = flops.bwd_flops(B, N, H, d, pats, wl.causal)
+        bm = statistics.median(bwhole)
+        ent.update({"bwd_ms": bm, "bwd_tflops": bw / bm / 1e9,
+                    "bwd_frac_of_peak": bw / bm / 1e9 / peak,
+                    "bwd_tokens_per_s": B * N / (bm * 1e-3),
+                    "bwd_tile_ms": statistics.median(btile),
+                    "bwd_tile_tflops": bw / statistics.median(btile) / 1e9,
+                    "step_tflops": (fw + bw) / (fm + bm) / 1e9,
+                    "step_frac_of_peak": (fw + bw) / (fm + bm) / 1e9 / peak,
+                    "tokens_per_s": B * N / ((fm + bm) * 1e-3)})
+    del q, k, v, do, ws_b
+    torch.cuda.empty_cache()
+    return ent
 
 
-def e2e_pipelined(dilattn, host, dev, pats, causal, ws_f, ws_b, K: int, W: int):
+def graph_step(dilattn, dev, name: str = "sweep_8192", replays: int = 50):
+    """The N = 8192 step captured once in a CUDA graph and replayed back to back,
+    without L2 flushes: the launch-bound regime. The training step
+    (dilattn_fwd_train + dilattn_bwd; the forward's pooled scratch becomes an
+    allocation node of the graph) when the capture takes it, else the forward
+    alone through dilattn_fwd_noalloc (scratch in the library's fixed array)."""
+    try:
+        return _graph_step(dilattn, dev, name, replays, train=True)
+    except Exception as e:  # noqa: BLE001 (reported in the JSON detail)
+        import torch
+        torch.cuda.synchronize()
+        ent = _graph_step(dilattn, dev, name, replays, train=False)
+        ent["training_step_capture"] = f"not taken: {type(e).__name__}: {e}"[:300]
+        return ent
+
+
+def _graph_step(dilattn, dev, name, replays, train):
+    import torch
+
+    wl = WORKLOADS[name]
+    B, N, H, d, pats = wl.B, wl.N, wl.H, wl.d, wl.patterns
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    q, k, v, do = (torch.randn((B, N, H, d), generator=gen, device=dev, dtype=torch.float32)
+                   .to(torch.bfloat16) for _ in range(4))
+    out, res = torch.empty_like(q), torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty((B, N, H, d), dtype=torch.float32, device=dev) for _ in range(3))
+    ws_b = torch.empty(dilattn.bwd_workspace_size(B, N, H, d), dtype=torch.uint8, device=dev)
+    s = torch.cuda.Stream(dev)
+
+    def body():
+        if train:
+            dilattn.fwd_train(q, k, v, pats, wl.causal, out=out, lse=lse, out_res=res, stream=s)
+            dilattn.bwd(q, k, v, out, lse, do, pats, wl.causal, out_res=res, dq=dq, dk=dk, dv=dv,
+                        workspace=ws_b, stream=s)
+        else:
+            dilattn.fwd_noalloc(q, k, v, pats, wl.causal, out=out, lse=lse, stream=s)
+
+    with torch.cuda.stream(s):
+        for _ in range(3):  # the first call looks up the fixed array, outside the capture
+            body()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        body()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(replays):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / replays
+    work = flops.fwd_flops(B, N, H, d, pats, wl.causal)
+    if train:
+        work += flops.bwd_flops(B, N, H, d, pats, wl.causal)
+    del g
+    return {"workload": name, "replays": replays,
+            "step": "dilattn_fwd_train + dilattn_bwd" if train else "dilattn_fwd_noalloc",
+            "ms_per_step": ms, "tflops": work / ms / 1e9, "tokens_per_s": B * N / (ms * 1e-3),
+            "l2": "not flushed (back-to-back replays)"}
+
+
+def e2e_pipelined(dilattn, host, dev, pats, causal, ws_b, K: int, W: int):
     """K training steps through the public API, each with its own copies.
 
-    Step i copies q, k, v, dout in from pinned host memory, runs dilattn.fwd and
-    dilattn.bwd, and copies out, lse, dq, dk, dv back to pinned host memory.
+    Step i copies q, k, v, dout in from pinned host memory, runs dilattn.fwd_train
+    and dilattn.bwd, and copies out, lse, dq, dk, dv back to pinned host memory.
     Copy-in, compute and copy-out run on three streams with two device buffer
     sets, so step i + 1's inputs cross PCIe while step i computes and step
     i - 1's results cross back (PCIe is full duplex); a buffer set is reused
@@ -330,10 +573,12 @@ def e2e_pipelined(dilattn, host, dev, pats, causal, ws_f, ws_b, K: int, W: int):
     B, N, H, _ = shp
     s_in, s_c, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     din = [{n: torch.empty(shp, dtype=bf, device=dev) for n in NAMES} for _ in range(2)]
-    dres = [{n: torch.empty(shp, dtype=bf, device=dev) for n in ("out", "dq", "dk", "dv")}
-            for _ in range(2)]
+    dres = [{"out": torch.empty(shp, dtype=bf, device=dev)} for _ in range(2)]
     for r_ in dres:
         r_["lse"] = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        for n in ("dq", "dk", "dv"):
+            r_[n] = torch.empty(shp, dtype=torch.float32, device=dev)
+    res = [torch.empty(shp, dtype=bf, device=dev) for _ in range(2)]  # stays on the device
     hres = [{n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in r_.items()}
             for r_ in dres]
     h2d = sum(host[n].numel() * host[n].element_size() for n in NAMES)
@@ -355,10 +600,10 @@ def e2e_pipelined(dilattn, host, dev, pats, causal, ws_f, ws_b, K: int, W: int):
             if res_free[b] is not None:
                 s_c.wait_event(res_free[b])  # step i - 2's results have left the device
             x, r_ = din[b], dres[b]
-            dilattn.fwd(x["q"], x["k"], x["v"], pats, causal, out=r_["out"], lse=r_["lse"],
-                        workspace=ws_f)
+            dilattn.fwd_train(x["q"], x["k"], x["v"], pats, causal, out=r_["out"],
+                              lse=r_["lse"], out_res=res[b])
             dilattn.bwd(x["q"], x["k"], x["v"], r_["out"], r_["lse"], x["dout"], pats, causal,
-                        dq=r_["dq"], dk=r_["dk"], dv=r_["dv"], workspace=ws_b, fwd_workspace=ws_f)
+                        out_res=res[b], dq=r_["dq"], dk=r_["dk"], dv=r_["dv"], workspace=ws_b)
             e_c = torch.cuda.Event()
             e_c.record(s_c)
             in_free[b] = e_c
@@ -404,28 +649,29 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     host = {n: torch.from_numpy(np.ascontiguousarray(inp[n + "_bits"]).view(np.int16))
             .view(torch.bfloat16).pin_memory() for n in NAMES}
     q, k, v, do = (host[n].to(dev) for n in NAMES)
-    out = torch.empty_like(q)
+    out, res = torch.empty_like(q), torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
-    ws_f = torch.empty(dilattn.fwd_workspace_size(B, N, H, d, pats), dtype=torch.uint8, device=dev)
-    ws_b = torch.empty(dilattn.bwd_workspace_size(B, N, H, d, pats), dtype=torch.uint8, device=dev)
+    dq, dk, dv = (torch.empty((B, N, H, d), dtype=torch.float32, device=dev) for _ in range(3))
+    ws_b = torch.empty(dilattn.bwd_workspace_size(B, N, H, d), dtype=torch.uint8, device=dev)
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(trace=None):
+    def step(trace=None, fwd_ev=None):
         if trace is not None:
             dilattn.set_trace_events(trace[0], trace[1])
-        dilattn.fwd(q, k, v, pats, causal, out=out, lse=lse, workspace=ws_f)
+        dilattn.fwd_train(q, k, v, pats, causal, out=out, lse=lse, out_res=res)
+        if fwd_ev is not None:
+            fwd_ev.record(stream)
         if trace is not None:
             dilattn.set_trace_events(trace[2], trace[3])
-        dilattn.bwd(q, k, v, out, lse, do, pats, causal, dq=dq, dk=dk, dv=dv, workspace=ws_b,
-                    fwd_workspace=ws_f)
+        dilattn.bwd(q, k, v, out, lse, do, pats, causal, out_res=res, dq=dq, dk=dk, dv=dv,
+                    workspace=ws_b)
         if trace is not None:
             dilattn.set_trace_events(None, None)
 
     K, W = args.steps, args.warmup
     ev = lambda: torch.cuda.Event(enable_timing=True)
-    step_ev = [(ev(), ev()) for _ in range(K)]
+    step_ev = [(ev(), ev(), ev()) for _ in range(K)]   # start, forward done, step done
     tile_ev = [tuple(ev() for _ in range(4)) for _ in range(K)]
     for tev in tile_ev:  # create the underlying CUDA events before handing them to the library
         for e in tev:
@@ -439,7 +685,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         raise RuntimeError("a kernel reported a device-side error during warm-up")
 
     gpu_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank]
-    sampler = ClockSampler(gpu_index)
+    sampler = make_clock_sampler(gpu_index)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -447,13 +693,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     for i in range(K):
         flush_buf.fill_(1)
         step_ev[i][0].record(stream)
-        step(tile_ev[i])
-        step_ev[i][1].record(stream)
+        step(tile_ev[i], step_ev[i][1])
+        step_ev[i][2].record(stream)
     torch.cuda.synchronize()
+    clocks = sampler.stop()
     if world > 1:
         dist.barrier()
-    clocks = sampler.stop()
-    step_ms = sum(a.elapsed_time(b) for a, b in step_ev)
+    step_ms = sum(a.elapsed_time(c) for a, _, c in step_ev)
+    fwd_ms = sum(a.elapsed_time(b) for a, b, _ in step_ev) / K
+    bwd_ms = sum(b.elapsed_time(c) for _, b, c in step_ev) / K
     fwd_tile_ms = sum(t[0].elapsed_time(t[1]) for t in tile_ev) / K
     bwd_tile_ms = sum(t[2].elapsed_time(t[3]) for t in tile_ev) / K
     step_ms = max_over_ranks(step_ms, world, dev)
@@ -461,7 +709,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     # e2e through the public API: every step copies its inputs in from pinned
     # host memory and its results back out, inside the timed region
-    e2e_total_ms, h2d, d2h = e2e_pipelined(dilattn, host, dev, pats, causal, ws_f, ws_b, K, W)
+    e2e_total_ms, h2d, d2h = e2e_pipelined(dilattn, host, dev, pats, causal, ws_b, K, W)
     if world > 1:
         dist.barrier()
     e2e_ms = max_over_ranks(e2e_total_ms, world, dev)
@@ -478,39 +726,53 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     fwd_tile_tf = fwd_work / (fwd_tile_ms * 1e-3) / 1e12
     bwd_tile_tf = bwd_work / (bwd_tile_ms * 1e-3) / 1e12
     if bwd_tile_ms >= fwd_tile_ms:
-        dom, dom_tf, dom_work = "bwd_tile_kernel", bwd_tile_tf, bwd_work
+        dom, dom_tf = "bwd_tile_kernel", bwd_tile_tf
     else:
-        dom, dom_tf, dom_work = "fwd_tile_kernel", fwd_tile_tf, fwd_work
+        dom, dom_tf = "fwd_tile_kernel", fwd_tile_tf
+    fwd_tf = fwd_work / (fwd_ms * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "B": B, "N": N, "H": H, "d": d,
                    "patterns": [list(p) for p in pats], "causal": causal,
-                   "step": "dilattn_fwd + dilattn_bwd",
+                   "step": "dilattn_fwd_train + dilattn_bwd (fp32 gradients)",
                    "l2": "flushed between timed steps (256 MB device write outside the events)",
                    "parallelism": f"independent batch per GPU x{world}"},
         "tokens_per_s": world * B * N / (ms_per_step * 1e-3),
         "frac_of_bf16_peak": value / world / peak,
         "detail": {
             "fwd_effective_flop": fwd_work, "bwd_effective_flop": bwd_work,
+            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+            "fwd_tflops": fwd_tf, "bwd_tflops": bwd_work / (bwd_ms * 1e-3) / 1e12,
+            "fwd_tokens_per_s": B * N / (fwd_ms * 1e-3),
+            "bwd_tokens_per_s": B * N / (bwd_ms * 1e-3),
             "fwd_tile_ms": fwd_tile_ms, "bwd_tile_ms": bwd_tile_ms,
             "fwd_tile_tflops": fwd_tile_tf, "bwd_tile_tflops": bwd_tile_tf,
-            "fwd_tokens_per_s": B * N / (fwd_tile_ms * 1e-3),
             "peak_source": peak_src,
         },
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tf, "peak": peak,
                      "unit": "TFLOP/s", "frac": dom_tf / peak,
                      "peak_note": f"bf16_tflops (burst) of {peak_src} peaks",
                      "traffic": load_traffic(dom, wl.name)},
+        "roofline_fwd": {"bound": "tensor", "kernel": "dilattn_fwd_train (whole call)",
+                         "achieved": fwd_tf, "peak": peak, "unit": "TFLOP/s",
+                         "frac": fwd_tf / peak,
+                         "traffic": load_traffic("fwd_tile_kernel", wl.name)},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / K,
                 "overlap": "copy-in, compute, copy-out of consecutive steps on three streams"},
-        "gpu_launches": 5 * K,
+        "gpu_launches": LAUNCHES_PER_STEP * K,
         "clocks": clocks,
     }
     if world == 1 and not args.no_sweep:
-        line["detail"]["length_sweep"] = sweep_detail(dilattn, dev)
+        det = line["detail"]
+        det["training_step_b4"] = time_workload(dilattn, dev, TRAIN, flush_buf, peak)
+        det["length_sweep"] = [time_workload(dilattn, dev, n, flush_buf, peak) for n in SWEEP]
+        det["wide_d128"] = time_workload(dilattn, dev, WIDE, flush_buf, peak)
+        det["graph_8k"] = graph_step(dilattn, dev)
+        if dilattn.device_error() != 0:
+            raise RuntimeError("a kernel reported a device-side error in the detail runs")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(wl)
     if rank == 0:
@@ -529,7 +791,7 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true",
-                    help="skip the length sweep (N = 8K, 128K, 1M) and the wide d = 128 forward")
+                    help="skip the detail runs (B = 4 step, length sweep, wide d = 128, graph)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -23,15 +23,18 @@
  *   q, k, v, out, dout, dq, dk, dv : [B][N][H][d]
  *   lse                            : [B][H][N] float32, natural log
  * Element types: the unsuffixed entry points take bfloat16 tensors (stored as
- * 16-bit words) and compute in fp32 with bf16 tensor-core products; the _f32
- * entry points take float32 tensors and compute in plain fp32.
+ * 16-bit words) and compute in fp32 with bf16 tensor-core products; their
+ * out is bf16 and the backward's gradients are fp32. The _f32 entry points
+ * take and return float32 tensors and compute in plain fp32.
  *
  * Ownership: every tensor pointer is a DEVICE pointer owned by the caller;
  * the library keeps no reference after the call returns. w and r are HOST
- * arrays of npat ints, read before the call returns. Workspaces are
- * caller-owned device memory of at least the size the matching
- * *_workspace_size function returns, 256-byte aligned; their contents on
- * entry do not matter and are garbage on return.
+ * arrays of npat ints, read before the call returns. The backward's
+ * workspace is caller-owned device memory of at least
+ * dilattn_bwd_workspace_size(...) bytes, 256-byte aligned; its contents on
+ * entry do not matter and are garbage on return. Library-owned device
+ * memory: one error word per device, the forward's scratch pool (below) and
+ * the fixed array of dilattn_fwd_noalloc.
  *
  * Asynchrony: every compute entry point validates its arguments, enqueues
  * its kernels on `stream` and returns; faults during execution surface at the
@@ -75,44 +78,69 @@ const char* dilattn_status_string(int status);
 const char* dilattn_last_error(void);
 
 /*
- * Forward. Writes out [B][N][H][d] bf16 and, unless lse is NULL,
- * lse [B][H][N] fp32. Workspace: fp32 per-pattern partial results
- * (one row of d + 1 floats per kept row of every pattern, segments padded to
- * whole 128-row tiles) followed by an fp32 copy of out; at least
- * dilattn_fwd_workspace_size(...) bytes. Keep the workspace untouched until
- * the matching dilattn_bwd if the backward should use that fp32 copy.
+ * Forward: merged dilated attention (the whole method of the preamble; the
+ * LongNet method description, gptget.net summary of arXiv 2307.02486,
+ * "方法详解" bullets 1-3, and the shared-denominator merge of the DarcStar
+ * commentary, third paragraph). Writes out [B][N][H][d] bf16 and, unless lse
+ * is NULL, lse [B][H][N] fp32.
+ *
+ * The merge runs inside the forward: when a pattern has r = 1 (it keeps every
+ * row), the tiles of that pattern finish each row, combining their own
+ * online softmax with the stored partial results (normalised O_i and lse_i,
+ * fp32) of the other patterns that keep the row, and write out and lse once;
+ * the r = 1 pattern itself stores no partial. Without an r = 1 pattern every
+ * pattern stores partials and a second kernel merges them. The partials live
+ * in scratch of dilattn_fwd_scratch_size(...) bytes, which dilattn_fwd takes
+ * stream-ordered from a memory pool the library creates per device on first
+ * use (cudaMallocFromPoolAsync / cudaFreeAsync on `stream`; freed blocks stay
+ * in the pool for the next call, so repeated calls map no new memory).
+ * Callers that must not allocate use dilattn_fwd_noalloc.
  */
-size_t dilattn_fwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
-                                  int npat);
+size_t dilattn_fwd_scratch_size(int B, int N, int H, int d, const int* w, const int* r,
+                                int npat);
 int dilattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
                 int B, int N, int H, int d, const int* w, const int* r, int npat, int causal,
-                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+                cudaStream_t stream);
+
+/*
+ * Forward for training: dilattn_fwd plus out_res [B][N][H][d] bf16, the
+ * rounding residual bf16(O - out) of each output element, written by the
+ * same fused epilogue. dilattn_bwd forms its row term D = rowsum(dout * O)
+ * from out + out_res, i.e. from O to about 16 significant bits: D taken from
+ * the bf16 out alone is off by sum_c dout_c (O_c - out_c), up to a few 1e-2,
+ * which moves dq and dk by up to about 1e-2. out_res must not be NULL nor
+ * overlap any other tensor argument.
+ */
+int dilattn_fwd_train(const void* q, const void* k, const void* v, void* out, void* out_res,
+                      float* lse, int B, int N, int H, int d, const int* w, const int* r, int npat,
+                      int causal, cudaStream_t stream);
 
 /*
  * Forward for callers that cannot allocate device memory: same arguments and
- * results as dilattn_fwd minus the workspace. Some callers have no way to
- * get scratch memory: a plugin handed only its input and output pointers by a
- * host framework, a server that reserves all device memory up front and
- * forbids later cudaMalloc calls, or code that must not risk the implicit
- * device synchronisation a cudaMalloc/cudaFree can bring. This entry point
+ * results as dilattn_fwd. Some callers have no way to get scratch memory: a
+ * plugin handed only its input and output pointers by a host framework, a
+ * server that reserves all device memory up front and forbids later
+ * allocations, or code that must not risk the implicit device
+ * synchronisation a cudaMalloc/cudaFree can bring. This entry point
  * allocates nothing, neither itself nor through any library: the forward's
- * per-pattern partial results go to a fixed array compiled into the library,
+ * scratch is a fixed array compiled into the library,
  * DILATTN_NOALLOC_SCRATCH_BYTES (64 MiB) large, which every device that
  * loads the library keeps reserved until the process exits. There is no
  * counterpart in the LongNet pages; it only changes where scratch lives.
  *
  * Limits and rules:
- *   - Problems whose dilattn_fwd_workspace_size(...) exceeds the array are
+ *   - Problems whose dilattn_fwd_scratch_size(...) exceeds the array are
  *     rejected with DILATTN_ERR_WORKSPACE (dilattn_last_error() gives the two
  *     sizes); nothing is launched.
  *   - The first call on each device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
  *     before any stream capture.
  *   - All calls on a device share the one array, and it keeps whatever the
- *     last call left there (this forward writes every scratch entry it later
- *     reads, so nothing needs to start at zero). Calls that can overlap on the
- *     GPU -- on different streams, or from different host threads -- race on
- *     the array; the caller must order them, e.g. on one stream.
+ *     last call left there; the forward clears the part that must start at
+ *     zero (its flags and ticket counter) itself, on `stream`. Calls that can
+ *     overlap on the GPU -- on different streams, or from different host
+ *     threads -- race on the array; the caller must order them, e.g. on one
+ *     stream.
  */
 #define DILATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -120,33 +148,66 @@ int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, 
                         int causal, cudaStream_t stream);
 
 /*
- * Backward of dilattn_fwd: given out and lse from the forward and the
- * output gradient dout (all device), writes dq, dk, dv [B][N][H][d] bf16, the
- * full derivative of sum(out * dout). The probabilities are recomputed from
- * the saved lse. Workspace: fp32 accumulators for dq, dk, dv, the row term
- * D = rowsum(dout * out) and the key-tile kernel's work counter, at least
- * dilattn_bwd_workspace_size(...) bytes. Calls that share a workspace must
- * not overlap on the GPU.
+ * Sequence-parallel forward, one rank's part (LongNet's distributed
+ * algorithm: the gptget.net summary of arXiv 2307.02486, "方法详解" bullet 5,
+ * and the abstract's second contribution). The sequence of N = L * world
+ * positions is split into world contiguous blocks of L; this rank holds
+ * block `rank` of q, k, v ([B][L][H][d] bf16) and writes out ([B][L][H][d])
+ * and lse ([B][H][L]) for its own rows, equal to the single-device
+ * dilattn_fwd on the whole sequence restricted to those rows.
  *
- * fwd_workspace: the workspace of the dilattn_fwd call that produced out and
- * lse, untouched since (fwd_workspace_bytes >= dilattn_fwd_workspace_size).
- * The backward then forms D from the forward's fp32 copy of out. It may be
- * NULL: D then comes from the bf16 out, the usual convention, whose rounding
- * (up to one bf16 ulp of out per element) moves dq and dk by up to about
- * 1e-2 more at rows whose exact gradient is near zero.
+ * A pattern with w <= L keeps its segments inside one block (L must be a
+ * multiple of w) and runs locally. A pattern with w > L spans
+ * min(w, N) / L ranks per segment (N a multiple of w unless w >= N; L a
+ * multiple of r; L / r a multiple of 128): every rank of the segment packs
+ * its kept rows of k and v (dilattn_pack_dilated: for head h the rows
+ * (h mod r) + m r of its block, [B][L/r][H][d]), the ranks all-gather them
+ * in rank order, and kg[i], vg[i] point to the gathered
+ * [ranks][B][L/r][H][d] buffers of this rank's segment. Only those dilated
+ * rows cross between ranks, never a full block. kg, vg may be NULL when no
+ * pattern spans ranks. Scratch as in dilattn_fwd.
  */
-size_t dilattn_bwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
-                                  int npat);
-int dilattn_bwd(const void* q, const void* k, const void* v, const void* out,
-                const float* lse, const void* dout, void* dq, void* dk, void* dv,
-                int B, int N, int H, int d, const int* w, const int* r, int npat, int causal,
-                const void* fwd_workspace, size_t fwd_workspace_bytes,
-                void* workspace, size_t workspace_bytes, cudaStream_t stream);
+int dilattn_fwd_seqpar(const void* q, const void* k, const void* v, void* out, float* lse,
+                       int B, int L, int H, int d, const int* w, const int* r, int npat,
+                       int causal, int rank, int world, const void* const* kg,
+                       const void* const* vg, cudaStream_t stream);
 
 /*
- * fp32 forward and backward (same semantics, float32 tensors, no workspace,
- * full fp32 FMA arithmetic without TF32). Meant for small problems: each
- * output row is computed by one thread.
+ * The rows a rank sends for a pattern of dilation r that spans ranks:
+ * buf[b][m][h][:] = x[b][(h mod r) + m r][h][:] for m < L / r (x and buf
+ * bf16, device; buf holds B * (L / r) * H * d elements; L a multiple of r).
+ */
+int dilattn_pack_dilated(const void* x, void* buf, int B, int L, int H, int d, int r,
+                         cudaStream_t stream);
+
+/*
+ * Backward of dilattn_fwd_train (the full derivative of the merged function:
+ * the merge weights depend on the scores and are differentiated, which
+ * equals the gradient of one softmax over the multiset union of the keys
+ * each row attends; DarcStar commentary, third paragraph). Given out,
+ * out_res and lse from that forward and the output gradient dout (bf16,
+ * [B][N][H][d]), writes the gradients of sum(O * dout): dq, dk, dv
+ * [B][N][H][d] FLOAT32, the precision they are accumulated in (a caller
+ * that keeps bf16 gradients rounds them). The probabilities are recomputed
+ * from the saved lse; the row term D = rowsum(dout * O) is formed from
+ * out + out_res. Workspace: D and the key-tile kernel's work counter,
+ * at least dilattn_bwd_workspace_size(B, N, H, d) bytes, 256-byte aligned;
+ * the workspace and dq, dk, dv must not overlap any input or each other.
+ * Calls that share a workspace or gradient buffers must not overlap on the
+ * GPU. d = 64 only (DILATTN_ERR_UNSUPPORTED otherwise; the fp32 entry point
+ * covers d = 128).
+ */
+size_t dilattn_bwd_workspace_size(int B, int N, int H, int d);
+int dilattn_bwd(const void* q, const void* k, const void* v, const void* out,
+                const void* out_res, const float* lse, const void* dout, float* dq, float* dk,
+                float* dv, int B, int N, int H, int d, const int* w, const int* r, int npat,
+                int causal, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * fp32 forward and backward: the same operation as dilattn_fwd / dilattn_bwd
+ * (same passages), float32 tensors, no workspace, full fp32 FMA arithmetic
+ * without TF32. Meant for small problems: each output row is computed by
+ * one thread.
  */
 int dilattn_fwd_f32(const float* q, const float* k, const float* v, float* out, float* lse,
                     int B, int N, int H, int d, const int* w, const int* r, int npat,
@@ -157,8 +218,10 @@ int dilattn_bwd_f32(const float* q, const float* k, const float* v, const float*
                     int causal, cudaStream_t stream);
 
 /*
- * Row selection, as the attention kernels see it: sig [H][N] (device,
- * uint32) receives bit i at (h, n) when pattern i keeps row n for head h.
+ * Row selection ("方法详解" bullets 1-3: segments of length w, every r-th row,
+ * offset h mod r per head), as the attention kernels see it: sig [H][N]
+ * (device, uint32) receives bit i at (h, n) when pattern i keeps row n for
+ * head h.
  * It enumerates kept rows with the same segment/offset code the attention
  * kernels use to address their tiles, so it checks that code bit for bit.
  */

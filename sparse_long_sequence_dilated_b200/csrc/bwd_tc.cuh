@@ -1,5 +1,5 @@
-// Backward kernels: preprocess (D = rowsum(dO * O) from the forward's fp32
-// copy of O when given, else from the bf16 O; zero the fp32 accumulators),
+// Backward kernels: preprocess (D = rowsum(dO * O) from the bf16 O the forward
+// returned; zero the fp32 accumulators),
 // the tcgen05 key-tile kernel, and the fp32 -> bf16 convert.
 //
 // The merged forward is one softmax over the multiset union of the keys the
@@ -38,9 +38,9 @@
 // dQ goes through a double-buffered TMEM accumulator; after each pair every
 // row warp stages its 32 x 32 block in a private shared-memory slab and adds
 // it to the fp32 accumulator with a TMA reduce-add. dK, dV are added the same
-// way once per unit (other patterns and tiles reach the same rows). The three
-// accumulators form one [3B][N][H][64] fp32 tensor read through the same
-// strided views as the inputs.
+// way once per unit (other patterns and tiles reach the same rows). The
+// gradients are fp32 [B][N][H][64] tensors, reached through the same strided
+// views as the inputs; they are the accumulators themselves.
 //
 // Warp roles (320 threads): warp 0 TMA producer (+ per-tile L and D rows and
 // an L2 prefetch of the next unit's key tile), warp 1 TMEM allocator and MMA
@@ -60,7 +60,9 @@ namespace dil {
 struct BwdParams {
   CUtensorMap tmq[kMaxPat], tmk[kMaxPat], tmv[kMaxPat], tmdo[kMaxPat];
   CUtensorMap tmq_t[kMaxPat], tmk_t[kMaxPat], tmv_t[kMaxPat], tmdo_t[kMaxPat];
-  CUtensorMap tmacc[kMaxPat], tmacc_t[kMaxPat];  // fp32 [3B][N][H][64]: dq, dk, dv; 32 x 32 boxes
+  // reduce-add targets, the fp32 gradients [B][N][H][64] (32 x 32 boxes)
+  CUtensorMap tmdq[kMaxPat], tmdk[kMaxPat], tmdv[kMaxPat];
+  CUtensorMap tmdq_t[kMaxPat], tmdk_t[kMaxPat], tmdv_t[kMaxPat];
   PatternGeom pat[kMaxPat];
   int npat, B, N, H, causal;
   float scale_log2;  // log2(e) / sqrt(d)
@@ -173,7 +175,7 @@ struct BwdUnit {
   PatternGeom g;
   SegInfo si;
   int u, t0, np;
-  const CUtensorMap *mq, *mk, *mv, *mdo, *macc;
+  const CUtensorMap *mq, *mk, *mv, *mdo, *mdq, *mdk, *mdv;
 };
 
 __device__ __forceinline__ bool bwd_unit(const BwdParams& p, long long uu, BwdUnit& U) {
@@ -205,7 +207,9 @@ __device__ __forceinline__ bool bwd_unit(const BwdParams& p, long long uu, BwdUn
   U.mk = tv ? &p.tmk_t[i] : &p.tmk[i];
   U.mv = tv ? &p.tmv_t[i] : &p.tmv[i];
   U.mdo = tv ? &p.tmdo_t[i] : &p.tmdo[i];
-  U.macc = tv ? &p.tmacc_t[i] : &p.tmacc[i];
+  U.mdq = tv ? &p.tmdq_t[i] : &p.tmdq[i];
+  U.mdk = tv ? &p.tmdk_t[i] : &p.tmdk[i];
+  U.mdv = tv ? &p.tmdv_t[i] : &p.tmdv[i];
   return true;
 }
 
@@ -553,7 +557,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       if (lane == 0) {
         int ph, m;
         view_coords(U.g, U.si, t * BM + q4 * 32, ph, m);
-        tma_reduce_add_5d(U.macc, slab, cg * 32, U.wu.h, ph, m, U.wu.b);
+        tma_reduce_add_5d(U.mdq, slab, cg * 32, U.wu.h, ph, m, U.wu.b);
         bulk_commit();
       }
       return true;
@@ -656,7 +660,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       }
       // dV, dK of the key tile: every MMA of the unit is complete (the last dQ
       // commit tracks them all). Rows past the segment are exact zeros (their
-      // P was forced to 0). dv and dk are batch slots 2B + b and B + b.
+      // P was forced to 0).
       {
         uint32_t rv[32], rk[32];
         tmem_ld32_sync(tl + C::TM_DV + cg * 32, rv);
@@ -674,7 +678,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_reduce_add_5d(U.macc, slab, cg * 32, U.wu.h, ph, m, 2 * p.B + U.wu.b);
+          tma_reduce_add_5d(U.mdv, slab, cg * 32, U.wu.h, ph, m, U.wu.b);
           bulk_commit();
           bulk_wait_read<0>();
         }
@@ -683,7 +687,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_reduce_add_5d(U.macc, slab, cg * 32, U.wu.h, ph, m, p.B + U.wu.b);
+          tma_reduce_add_5d(U.mdk, slab, cg * 32, U.wu.h, ph, m, U.wu.b);
           bulk_commit();
         }
       }
@@ -700,16 +704,17 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   }
 }
 
-// D = rowsum(dO * O) per (b, h, n) and zeroed fp32 accumulators; one warp per row.
+// D = rowsum(dO * O) per (b, h, n) from out + out_res (O to about 16
+// significant bits), and zeroed fp32 gradients; one warp per row.
 struct PrepParams {
   int B, N, H;
   const __nv_bfloat16* out;
-  const float* out_f32;  // the forward's fp32 copy of out, or null
+  const __nv_bfloat16* out_res;  // bf16(O - out) from the training forward
   const __nv_bfloat16* dout;
   float* drow;
-  float* dq_acc;
-  float* dk_acc;
-  float* dv_acc;
+  float* dq;
+  float* dk;
+  float* dv;
   int* counter;  // the key-tile kernel's unit counter
 };
 
@@ -719,39 +724,22 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(PrepParams p) {
   if (row == 0 && threadIdx.x == 0) *p.counter = 0;
   if (row >= (long long)p.B * p.N * p.H) return;
   const __nv_bfloat162 d = reinterpret_cast<const __nv_bfloat162*>(p.dout + row * 64)[lane];
-  float2 o;
-  if (p.out_f32 != nullptr) {
-    o = reinterpret_cast<const float2*>(p.out_f32 + row * 64)[lane];
-  } else {
-    const __nv_bfloat162 ob = reinterpret_cast<const __nv_bfloat162*>(p.out + row * 64)[lane];
-    o = make_float2(__low2float(ob), __high2float(ob));
-  }
-  float acc = o.x * __low2float(d) + o.y * __high2float(d);
+  const __nv_bfloat162 ob = reinterpret_cast<const __nv_bfloat162*>(p.out + row * 64)[lane];
+  const __nv_bfloat162 rb = reinterpret_cast<const __nv_bfloat162*>(p.out_res + row * 64)[lane];
+  const float o0 = __low2float(ob) + __low2float(rb), o1 = __high2float(ob) + __high2float(rb);
+  float acc = o0 * __low2float(d) + o1 * __high2float(d);
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
   const float2 z = make_float2(0.f, 0.f);
-  reinterpret_cast<float2*>(p.dq_acc + row * 64)[lane] = z;
-  reinterpret_cast<float2*>(p.dk_acc + row * 64)[lane] = z;
-  reinterpret_cast<float2*>(p.dv_acc + row * 64)[lane] = z;
+  reinterpret_cast<float2*>(p.dq + row * 64)[lane] = z;
+  reinterpret_cast<float2*>(p.dk + row * 64)[lane] = z;
+  reinterpret_cast<float2*>(p.dv + row * 64)[lane] = z;
   if (lane == 0) {
     const int h = (int)(row % p.H);
     const long long bn = row / p.H;
     const int n = (int)(bn % p.N);
     const int b = (int)(bn / p.N);
     p.drow[((long long)b * p.H + h) * p.N + n] = acc;
-  }
-}
-
-// fp32 accumulators -> bf16 gradients (round to nearest even).
-__global__ void __launch_bounds__(256) bwd_convert_kernel(long long n4, const float4* dq,
-                                                          const float4* dk, const float4* dv,
-                                                          uint2* gq, uint2* gk, uint2* gv) {
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
-       i += (long long)gridDim.x * blockDim.x) {
-    const float4 a = dq[i], b = dk[i], c = dv[i];
-    gq[i] = make_uint2(pack_bf16(a.x, a.y), pack_bf16(a.z, a.w));
-    gk[i] = make_uint2(pack_bf16(b.x, b.y), pack_bf16(b.z, b.w));
-    gv[i] = make_uint2(pack_bf16(c.x, c.y), pack_bf16(c.z, c.w));
   }
 }
 

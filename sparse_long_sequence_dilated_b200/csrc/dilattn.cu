@@ -80,6 +80,8 @@ struct DeviceState {
   bool arch_ok = false;
   int* err_word = nullptr;
   int num_sms = 0;
+  int dev = 0;
+  cudaMemPool_t pool = nullptr;  // the forward's scratch pool, created on first use
 };
 
 std::mutex g_mu;
@@ -91,6 +93,7 @@ int device_state(DeviceState** out) {
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceState& st = g_devices[dev];
+  st.dev = dev;
   if (!st.init) {
     int major = 0;
     e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
@@ -115,6 +118,29 @@ int device_state(DeviceState** out) {
   }
   if (!st.arch_ok) return DILATTN_ERR_UNSUPPORTED;
   *out = &st;
+  return DILATTN_OK;
+}
+
+// Stream-ordered memory pool of the device for the forward's scratch. Freed
+// blocks stay in the pool (release threshold: never), so after the first call
+// of a given size the forward maps no new memory.
+int scratch_pool(DeviceState* st, cudaMemPool_t* out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (st->pool == nullptr) {
+    cudaMemPoolProps props;
+    memset(&props, 0, sizeof(props));
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = st->dev;
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = cudaMemPoolCreate(&pool, &props);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+    uint64_t keep = ~0ull;
+    e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemPoolSetAttribute");
+    st->pool = pool;
+  }
+  *out = st->pool;
   return DILATTN_OK;
 }
 
@@ -197,10 +223,12 @@ int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CU
   return DILATTN_OK;
 }
 
-// 2-D view of the forward's fp32 partial outputs [rows][d] for TMA stores:
-// box 32 columns (128 bytes, 128-byte swizzle) x 128 rows.
-int partial_map(const float* ptr, long long rows, int d, CUtensorMap* out) {
-  MapKey key{ptr, (int)(rows >> 31), (int)(rows & 0x7fffffff), d, -1, -1, -1, 2, BM};
+// View of a gathered dilated buffer [ranks][B][rank_rows][H][d] bf16 whose
+// row j of head h is dilated row j of that head's segment: dims
+// {d, H, rank_rows, ranks, B}; a 128-row box never crosses a rank's block
+// (rank_rows is a multiple of 128).
+int gathered_map(const void* ptr, int B, int H, int d, int rank_rows, int ranks, CUtensorMap* out) {
+  MapKey key{ptr, B, rank_rows, H, d, -ranks, 2, 0, BM};
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -211,12 +239,14 @@ int partial_map(const float* ptr, long long rows, int d, CUtensorMap* out) {
   }
   int rc = get_encoder();
   if (rc != DILATTN_OK) return rc;
-  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)d * 4};
-  cuuint32_t box[2] = {32, (cuuint32_t)BM};
-  cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t rowb = (cuuint64_t)H * d * 2;
+  cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rank_rows, (cuuint64_t)ranks,
+                        (cuuint64_t)B};
+  cuuint64_t strides[4] = {(cuuint64_t)d * 2, rowb, rowb * rank_rows * B, rowb * rank_rows};
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)BM, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap m;
-  CUresult cr = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(ptr), dims,
+  CUresult cr = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -232,6 +262,17 @@ int partial_map(const float* ptr, long long rows, int d, CUtensorMap* out) {
   *out = m;
   return DILATTN_OK;
 }
+
+// One sequence-parallel rank's per-pattern inputs (see FwdParams): patterns
+// with kv_rows > 0 take K and V from the gathered buffers kg, vg.
+struct SeqParPlan {
+  int kv_rows[kMaxPat];
+  int kv_rank_rows[kMaxPat];
+  int ranks[kMaxPat];
+  int toff[kMaxPat];
+  const void* kg[kMaxPat];
+  const void* vg[kMaxPat];
+};
 
 // ------------------------------------------------------------------ validation
 int check_shape(int B, int N, int H, int d, const int* w, const int* r, int npat, int causal) {
@@ -256,8 +297,31 @@ bool overlaps(const void* a, size_t an, const void* b, size_t bn) {
   return x < y + bn && y < x + an;
 }
 
+// Pattern geometry and partial-buffer layout. Pattern `skip` (the merging
+// pattern, or -1) stores no partials and gets no rows. Returns the partial rows.
+// Argument checks shared by the forward entry points.
+int check_fwd_args(const void* q, const void* k, const void* v, const void* out, const float* lse,
+                   int B, int N, int H, int d, const int* w, const int* r, int npat, int causal) {
+  int rc = check_shape(B, N, H, d, w, r, npat, causal);
+  if (rc != DILATTN_OK) return rc;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return DILATTN_ERR_INVALID_ARG;
+  if (lse != nullptr && !aligned16(lse)) return DILATTN_ERR_INVALID_ARG;
+  const size_t tb = (size_t)B * N * H * d * 2;
+  if (overlaps(out, tb, q, tb) || overlaps(out, tb, k, tb) || overlaps(out, tb, v, tb))
+    return DILATTN_ERR_INVALID_ARG;
+  if (lse != nullptr) {
+    const size_t lb = (size_t)B * H * N * 4;
+    if (overlaps(lse, lb, q, tb) || overlaps(lse, lb, k, tb) || overlaps(lse, lb, v, tb) ||
+        overlaps(lse, lb, out, tb))
+      return DILATTN_ERR_INVALID_ARG;
+  }
+  if (d != 64 && d != 128) return DILATTN_ERR_UNSUPPORTED;
+  return DILATTN_OK;
+}
+
 long long make_geoms(int B, int N, int H, const int* w, const int* r, int npat,
-                     PatternGeom* geo) {
+                     PatternGeom* geo, int skip = -1) {
   long long rows = 0;
   for (int i = 0; i < npat; ++i) {
     PatternGeom& g = geo[i];
@@ -270,23 +334,38 @@ long long make_geoms(int B, int N, int H, const int* w, const int* r, int npat,
     g.pstride = g.ntiles * BM;
     g.nmod = N % r[i];
     g.part_base = rows;
-    rows += (long long)B * H * g.nseg * g.pstride;
+    if (i != skip) rows += (long long)B * H * g.nseg * g.pstride;
   }
   return rows;
+}
+
+// The merging pattern: one with r = 1 keeps every row of every head, so its
+// tiles can finish the merge of all patterns. The shortest such pattern is
+// taken (its tiles are the shortest, which keeps the end of the launch short).
+int pick_merger(const int* w, const int* r, int npat) {
+  int m = -1;
+  for (int i = 0; i < npat; ++i)
+    if (r[i] == 1 && (m < 0 || w[i] < w[m])) m = i;
+  return m;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
 // Longest-first unit order for the tile kernels (see Sched).
-long long make_schedule(const PatternGeom* pat, int npat, int B, int H, Sched& sc) {
-  std::vector<int> order(npat);
-  for (int i = 0; i < npat; ++i) order[i] = i;
+long long make_schedule(const PatternGeom* pat, int npat, int B, int H, Sched& sc,
+                        unsigned include = 0xffffffffu) {
+  std::vector<int> order;
+  for (int i = 0; i < npat; ++i)
+    if (include >> i & 1u) order.push_back(i);
+  const int nsel = (int)order.size();
+  memset(&sc, 0, sizeof(sc));
+  if (nsel == 0) return 0;
   std::stable_sort(order.begin(), order.end(),
                    [&](int a, int b) { return pat[a].ntiles > pat[b].ntiles; });
   std::vector<int> vals;
   for (int i : order)
     if (vals.empty() || vals.back() != pat[i].ntiles) vals.push_back(pat[i].ntiles);
-  for (int i = 0; i < npat; ++i) sc.order[i] = order[i];
+  for (int i = 0; i < nsel; ++i) sc.order[i] = order[i];
   sc.nband = (int)vals.size();
   sc.start[0] = 0;
   for (int j = 0; j < sc.nband; ++j) {
@@ -294,7 +373,7 @@ long long make_schedule(const PatternGeom* pat, int npat, int B, int H, Sched& s
     sc.nt[j] = vals[j];
     int act = 0;
     long long per = 0;
-    for (int a = 0; a < npat; ++a) {
+    for (int a = 0; a < nsel; ++a) {
       if (pat[order[a]].ntiles >= vals[j]) {
         ++act;
         per += (long long)pat[order[a]].nseg * B * H;
@@ -308,16 +387,30 @@ long long make_schedule(const PatternGeom* pat, int npat, int B, int H, Sched& s
   return sc.start[sc.nband];
 }
 
-// The fp32 copy of out inside a forward workspace of `rows` partial rows.
-float* fwd_out_f32(void* ws, long long rows, int d) {
-  return reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + align256((size_t)rows * d * 4) +
-                                  align256((size_t)rows * 4));
+// Forward scratch: [rows][d] fp32 partial outputs, [rows] fp32 partial lse,
+// one flag per 128-row block of partials, and the ticket counter.
+struct FwdScratch {
+  size_t o_bytes, lse_bytes, flag_bytes;
+  size_t total() const { return o_bytes + lse_bytes + flag_bytes; }
+};
+FwdScratch fwd_scratch_layout(long long rows, int d) {
+  FwdScratch f;
+  f.o_bytes = align256((size_t)rows * d * 4);
+  f.lse_bytes = align256((size_t)rows * 4);
+  f.flag_bytes = align256((size_t)(rows / BM + 1) * 4 + 4);  // flags, then the counter
+  return f;
+}
+
+size_t fwd_scratch_bytes(int B, int N, int H, int d, const int* w, const int* r, int npat) {
+  PatternGeom geo[kMaxPat];
+  const long long rows = make_geoms(B, N, H, w, r, npat, geo, pick_merger(w, r, npat));
+  return fwd_scratch_layout(rows, d).total();
 }
 
 template <int D>
-int launch_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N,
-               int H, const int* w, const int* r, int npat, int causal, void* ws,
-               DeviceState* st, cudaStream_t stream) {
+int launch_fwd(const void* q, const void* k, const void* v, void* out, void* out_res, float* lse,
+               int B, int N, int H, const int* w, const int* r, int npat, int causal, void* ws,
+               DeviceState* st, cudaStream_t stream, const SeqParPlan* sp = nullptr) {
   static_assert(sizeof(FwdParams) < 32000, "kernel parameter block too large");
   FwdParams p;
   memset(&p, 0, sizeof(p));
@@ -327,14 +420,18 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   p.H = H;
   p.causal = causal;
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
-  const long long rows = make_geoms(B, N, H, w, r, npat, p.pat);
-  p.part_o = reinterpret_cast<float*>(ws);
-  p.part_lse = reinterpret_cast<float*>((char*)ws + align256((size_t)rows * D * 4));
+  p.merger = pick_merger(w, r, npat);
+  const long long rows = make_geoms(B, N, H, w, r, npat, p.pat, p.merger);
+  const FwdScratch lay = fwd_scratch_layout(rows, D);
+  char* wsb = reinterpret_cast<char*>(ws);
+  p.part_o = reinterpret_cast<float*>(wsb);
+  p.part_lse = reinterpret_cast<float*>(wsb + lay.o_bytes);
+  p.flags = reinterpret_cast<int*>(wsb + lay.o_bytes + lay.lse_bytes);
+  p.counter = p.flags + rows / BM + 1;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.out_res = reinterpret_cast<__nv_bfloat16*>(out_res);
+  p.lse = lse;
   p.err = ErrCtx{st->err_word, next_tag()};
-  {
-    int rc = partial_map(p.part_o, rows, D, &p.tm_po);
-    if (rc != DILATTN_OK) return rc;
-  }
   for (int i = 0; i < npat; ++i) {
     const void* src[3] = {q, k, v};
     CUtensorMap* dst[3] = {&p.tmq[i], &p.tmk[i], &p.tmv[i]};
@@ -344,17 +441,35 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
       if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j]);
       if (rc != DILATTN_OK) return rc;
     }
+    if (sp != nullptr && sp->kv_rows[i] > 0) {
+      p.kv_rows[i] = sp->kv_rows[i];
+      p.kv_rank_rows[i] = sp->kv_rank_rows[i];
+      p.toff[i] = sp->toff[i];
+      int rc = gathered_map(sp->kg[i], B, H, D, sp->kv_rank_rows[i], sp->ranks[i], &p.tmk[i]);
+      if (rc == DILATTN_OK)
+        rc = gathered_map(sp->vg[i], B, H, D, sp->kv_rank_rows[i], sp->ranks[i], &p.tmv[i]);
+      if (rc != DILATTN_OK) return rc;
+    }
   }
-  const long long units = make_schedule(p.pat, npat, B, H, p.sched);
+  const unsigned all = (1u << npat) - 1u;
+  const unsigned mbit = p.merger >= 0 ? (1u << p.merger) : 0u;
+  p.units_p = make_schedule(p.pat, npat, B, H, p.sched, all & ~mbit);
+  const long long units_m = mbit ? make_schedule(p.pat, npat, B, H, p.sched_m, mbit) : 0;
+  const long long units = p.units_p + units_m;
   if (units > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
+  cudaError_t e = cudaMemsetAsync(p.flags, 0, lay.flag_bytes, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   int rc = trace_mark(g_trace_begin, stream);
   if (rc != DILATTN_OK) return rc;
-  fwd_tile_kernel<D><<<(unsigned)units, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM_BYTES, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  if (units > 0)
+    fwd_tile_kernel<D><<<(unsigned)units, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM_BYTES, stream>>>(p);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd_tile_kernel launch");
   rc = trace_mark(g_trace_end, stream);
   if (rc != DILATTN_OK) return rc;
+  if (p.merger >= 0) return DILATTN_OK;
 
+  // No pattern keeps every row: a separate pass merges the partials.
   MergeParams mp;
   memset(&mp, 0, sizeof(mp));
   memcpy(mp.pat, p.pat, sizeof(mp.pat));
@@ -365,7 +480,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   mp.part_o = p.part_o;
   mp.part_lse = p.part_lse;
   mp.out = reinterpret_cast<__nv_bfloat16*>(out);
-  mp.out_f32 = fwd_out_f32(ws, rows, D);
+  mp.out_res = reinterpret_cast<__nv_bfloat16*>(out_res);
   mp.lse = lse;
   const long long total_rows = (long long)B * N * H;
   constexpr int rows_per_block = 256 / DILATTN_MERGE_TPR;
@@ -376,9 +491,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, float* ls
   return DILATTN_OK;
 }
 
-int launch_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
-               const void* dout, void* dq, void* dk, void* dv, int B, int N, int H,
-               const int* w, const int* r, int npat, int causal, const float* out_f32, void* ws,
+int launch_bwd(const void* q, const void* k, const void* v, const void* out, const void* out_res,
+               const float* lse, const void* dout, float* dq, float* dk, float* dv, int B, int N,
+               int H,
+               const int* w, const int* r, int npat, int causal, void* ws,
                DeviceState* st, cudaStream_t stream) {
   constexpr int D = 64;
   static_assert(sizeof(BwdParams) < 32000, "kernel parameter block too large");
@@ -392,16 +508,12 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   p.tau = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   make_geoms(B, N, H, w, r, npat, p.pat);
-  // [3B][N][H][64] fp32: dq for batches 0..B-1, then dk, then dv (B*N*H*64*4
-  // is a multiple of 256, so the three align256 blocks are adjacent)
-  const size_t tbytes = align256((size_t)B * N * H * D * 4);
+  // workspace: D [B][H][N] fp32, then 256 bytes for the key-tile kernel's unit counter
   char* wsb = reinterpret_cast<char*>(ws);
-  float* dq_acc = reinterpret_cast<float*>(wsb);
-  float* dk_acc = reinterpret_cast<float*>(wsb + tbytes);
-  float* dv_acc = reinterpret_cast<float*>(wsb + 2 * tbytes);
-  float* drow = reinterpret_cast<float*>(wsb + 3 * tbytes);
+  float* drow = reinterpret_cast<float*>(wsb);
   p.drow = drow;
   p.lse = lse;
+  p.counter = reinterpret_cast<int*>(wsb + align256((size_t)B * H * N * 4));
   p.err = ErrCtx{st->err_word, next_tag()};
   for (int i = 0; i < npat; ++i) {
     const void* src[4] = {q, k, v, dout};
@@ -413,9 +525,14 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
       if (rc != DILATTN_OK) return rc;
     }
     // reduce-add targets: one row warp adds a 32-row x 32-column block
-    int rc = strided_map(dq_acc, 3 * B, N, H, D, r[i], 0, &p.tmacc[i], 1, 32);
-    if (rc == DILATTN_OK) rc = strided_map(dq_acc, 3 * B, N, H, D, r[i], 1, &p.tmacc_t[i], 1, 32);
-    if (rc != DILATTN_OK) return rc;
+    const float* grad[3] = {dq, dk, dv};
+    CUtensorMap* gm[3] = {&p.tmdq[i], &p.tmdk[i], &p.tmdv[i]};
+    CUtensorMap* gm_t[3] = {&p.tmdq_t[i], &p.tmdk_t[i], &p.tmdv_t[i]};
+    for (int j = 0; j < 3; ++j) {
+      int rc = strided_map(grad[j], B, N, H, D, r[i], 0, gm[j], 1, 32);
+      if (rc == DILATTN_OK) rc = strided_map(grad[j], B, N, H, D, r[i], 1, gm_t[j], 1, 32);
+      if (rc != DILATTN_OK) return rc;
+    }
   }
   // group-major unit order: patterns by tile count (descending, stable), then
   // (segment, batch, head) groups, then key tiles
@@ -434,19 +551,18 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   const long long units = p.gstart[npat];
   if (units > 0x7fffffffLL) return DILATTN_ERR_UNSUPPORTED;
   const long long rows = (long long)B * N * H;
-  p.counter = reinterpret_cast<int*>(wsb + 3 * tbytes + align256((size_t)B * H * N * 4));
 
   PrepParams pp;
   pp.B = B;
   pp.N = N;
   pp.H = H;
   pp.out = reinterpret_cast<const __nv_bfloat16*>(out);
-  pp.out_f32 = out_f32;
+  pp.out_res = reinterpret_cast<const __nv_bfloat16*>(out_res);
   pp.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
   pp.drow = drow;
-  pp.dq_acc = dq_acc;
-  pp.dk_acc = dk_acc;
-  pp.dv_acc = dv_acc;
+  pp.dq = dq;
+  pp.dk = dk;
+  pp.dv = dv;
   pp.counter = p.counter;
   bwd_prep_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>(pp);
   cudaError_t e = cudaGetLastError();
@@ -460,17 +576,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
     bwd_tile_kernel<<<(unsigned)grid, BwdCfg::THREADS, BwdCfg::SMEM_BYTES, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "bwd_tile_kernel launch");
-  rc = trace_mark(g_trace_end, stream);
-  if (rc != DILATTN_OK) return rc;
-  const long long n4 = rows * D / 4;
-  const long long cblocks = std::min<long long>((n4 + 255) / 256, (long long)st->num_sms * 16);
-  bwd_convert_kernel<<<(unsigned)cblocks, 256, 0, stream>>>(
-      n4, reinterpret_cast<const float4*>(dq_acc), reinterpret_cast<const float4*>(dk_acc),
-      reinterpret_cast<const float4*>(dv_acc), reinterpret_cast<uint2*>(dq),
-      reinterpret_cast<uint2*>(dk), reinterpret_cast<uint2*>(dv));
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return cuda_fail(e, "bwd_convert_kernel launch");
-  return DILATTN_OK;
+  return trace_mark(g_trace_end, stream);
 }
 
 RowParams make_row_params(int B, int N, int H, int d, const int* w, const int* r, int npat,
@@ -508,94 +614,105 @@ const char* dilattn_status_string(int status) {
 
 const char* dilattn_last_error(void) { return g_last_error; }
 
-size_t dilattn_fwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
-                                  int npat) {
+size_t dilattn_fwd_scratch_size(int B, int N, int H, int d, const int* w, const int* r,
+                                int npat) {
   if (check_shape(B, N, H, d, w, r, npat, 1) != DILATTN_OK) return 0;
-  PatternGeom geo[kMaxPat];
-  const long long rows = make_geoms(B, N, H, w, r, npat, geo);
-  return align256((size_t)rows * d * 4) + align256((size_t)rows * 4) +
-         align256((size_t)B * N * H * d * 4);
+  return fwd_scratch_bytes(B, N, H, d, w, r, npat);
 }
 
-int dilattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N,
-                int H, int d, const int* w, const int* r, int npat, int causal, void* workspace,
-                size_t workspace_bytes, cudaStream_t stream) {
-  int rc = check_shape(B, N, H, d, w, r, npat, causal);
+}  // extern "C"
+
+namespace dil {
+namespace {
+// dilattn_fwd and dilattn_fwd_train: scratch from the library's pool.
+int fwd_pooled(const void* q, const void* k, const void* v, void* out, void* out_res, float* lse,
+               int B, int N, int H, int d, const int* w, const int* r, int npat, int causal,
+               cudaStream_t stream) {
+  int rc = check_fwd_args(q, k, v, out, lse, B, N, H, d, w, r, npat, causal);
   if (rc != DILATTN_OK) return rc;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-    return DILATTN_ERR_INVALID_ARG;
-  if (lse != nullptr && !aligned16(lse)) return DILATTN_ERR_INVALID_ARG;
-  const size_t tb = (size_t)B * N * H * d * 2;
-  if (overlaps(out, tb, q, tb) || overlaps(out, tb, k, tb) || overlaps(out, tb, v, tb))
-    return DILATTN_ERR_INVALID_ARG;
-  if (lse != nullptr) {
-    const size_t lb = (size_t)B * H * N * 4;
-    if (overlaps(lse, lb, q, tb) || overlaps(lse, lb, k, tb) || overlaps(lse, lb, v, tb) ||
-        overlaps(lse, lb, out, tb))
+  if (out_res != nullptr) {
+    const size_t tb = (size_t)B * N * H * d * 2;
+    if (!aligned16(out_res) || overlaps(out_res, tb, q, tb) || overlaps(out_res, tb, k, tb) ||
+        overlaps(out_res, tb, v, tb) || overlaps(out_res, tb, out, tb) ||
+        (lse != nullptr && overlaps(out_res, tb, lse, (size_t)B * H * N * 4)))
       return DILATTN_ERR_INVALID_ARG;
   }
-  if (d != 64 && d != 128) return DILATTN_ERR_UNSUPPORTED;
-  const size_t need = dilattn_fwd_workspace_size(B, N, H, d, w, r, npat);
-  if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0 ||
-      workspace_bytes < need)
-    return DILATTN_ERR_WORKSPACE;
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != DILATTN_OK) return rc;
-  if (d == 64)
-    return launch_fwd<64>(q, k, v, out, lse, B, N, H, w, r, npat, causal, workspace, st, stream);
-  return launch_fwd<128>(q, k, v, out, lse, B, N, H, w, r, npat, causal, workspace, st, stream);
+  cudaMemPool_t pool = nullptr;
+  rc = scratch_pool(st, &pool);
+  if (rc != DILATTN_OK) return rc;
+  const size_t need = fwd_scratch_bytes(B, N, H, d, w, r, npat);
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&scratch, need, pool, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync (forward scratch)");
+  rc = d == 64 ? launch_fwd<64>(q, k, v, out, out_res, lse, B, N, H, w, r, npat, causal, scratch,
+                                st, stream)
+               : launch_fwd<128>(q, k, v, out, out_res, lse, B, N, H, w, r, npat, causal, scratch,
+                                 st, stream);
+  e = cudaFreeAsync(scratch, stream);  // stream-ordered: after the kernels that use it
+  if (rc == DILATTN_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync (forward scratch)");
+  return rc;
 }
+}  // namespace
+}  // namespace dil
 
-size_t dilattn_bwd_workspace_size(int B, int N, int H, int d, const int* w, const int* r,
-                                  int npat) {
-  if (check_shape(B, N, H, d, w, r, npat, 1) != DILATTN_OK) return 0;
-  const size_t t = (size_t)B * N * H * d * 4;
-  return 3 * align256(t) + align256((size_t)B * H * N * 4) + 256;  // + the unit counter
-}
+extern "C" {
 
-int dilattn_bwd(const void* q, const void* k, const void* v, const void* out, const float* lse,
-                const void* dout, void* dq, void* dk, void* dv, int B, int N, int H, int d,
-                const int* w, const int* r, int npat, int causal, const void* fwd_workspace,
-                size_t fwd_workspace_bytes, void* workspace, size_t workspace_bytes,
+int dilattn_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int N,
+                int H, int d, const int* w, const int* r, int npat, int causal,
                 cudaStream_t stream) {
+  return fwd_pooled(q, k, v, out, nullptr, lse, B, N, H, d, w, r, npat, causal, stream);
+}
+
+int dilattn_fwd_train(const void* q, const void* k, const void* v, void* out, void* out_res,
+                      float* lse, int B, int N, int H, int d, const int* w, const int* r, int npat,
+                      int causal, cudaStream_t stream) {
+  if (out_res == nullptr) return DILATTN_ERR_INVALID_ARG;
+  return fwd_pooled(q, k, v, out, out_res, lse, B, N, H, d, w, r, npat, causal, stream);
+}
+
+size_t dilattn_bwd_workspace_size(int B, int N, int H, int d) {
+  if (B < 1 || N < 1 || H < 1 || d < 1 || (double)B * N * H * d >= 1099511627776.0) return 0;
+  return align256((size_t)B * H * N * 4) + 256;  // D, then the unit counter
+}
+
+int dilattn_bwd(const void* q, const void* k, const void* v, const void* out,
+                const void* out_res, const float* lse, const void* dout, float* dq, float* dk,
+                float* dv, int B, int N, int H, int d, const int* w, const int* r, int npat,
+                int causal, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   int rc = check_shape(B, N, H, d, w, r, npat, causal);
   if (rc != DILATTN_OK) return rc;
-  const void* ins[6] = {q, k, v, out, lse, dout};
+  const void* ins[7] = {q, k, v, out, lse, dout, out_res};
   for (const void* x : ins)
     if (!aligned16(x)) return DILATTN_ERR_INVALID_ARG;
   if (!aligned16(dq) || !aligned16(dk) || !aligned16(dv)) return DILATTN_ERR_INVALID_ARG;
-  const size_t tb = (size_t)B * N * H * d * 2;
+  const size_t tb = (size_t)B * N * H * d * 2;  // a bf16 input
+  const size_t gb = 2 * tb;                     // an fp32 gradient
   const size_t lb = (size_t)B * H * N * 4;
   void* outs[3] = {dq, dk, dv};
   for (void* o : outs)
-    for (int j = 0; j < 6; ++j)
-      if (overlaps(o, tb, ins[j], j == 4 ? lb : tb)) return DILATTN_ERR_INVALID_ARG;
-  if (overlaps(dq, tb, dk, tb) || overlaps(dq, tb, dv, tb) || overlaps(dk, tb, dv, tb))
+    for (int j = 0; j < 7; ++j)
+      if (overlaps(o, gb, ins[j], j == 4 ? lb : tb)) return DILATTN_ERR_INVALID_ARG;
+  if (overlaps(dq, gb, dk, gb) || overlaps(dq, gb, dv, gb) || overlaps(dk, gb, dv, gb))
     return DILATTN_ERR_INVALID_ARG;
   if (d != 64) {
     snprintf(g_last_error, sizeof(g_last_error), "bf16 backward is built for d = 64");
     return DILATTN_ERR_UNSUPPORTED;
   }
-  const size_t need = dilattn_bwd_workspace_size(B, N, H, d, w, r, npat);
+  const size_t need = dilattn_bwd_workspace_size(B, N, H, d);
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0 ||
       workspace_bytes < need)
     return DILATTN_ERR_WORKSPACE;
+  for (int j = 0; j < 7; ++j)
+    if (overlaps(workspace, need, ins[j], j == 4 ? lb : tb)) return DILATTN_ERR_INVALID_ARG;
+  for (void* o : outs)
+    if (overlaps(workspace, need, o, gb)) return DILATTN_ERR_INVALID_ARG;
   DeviceState* st = nullptr;
   rc = device_state(&st);
   if (rc != DILATTN_OK) return rc;
-  const float* out_f32 = nullptr;
-  if (fwd_workspace != nullptr) {
-    if ((reinterpret_cast<uintptr_t>(fwd_workspace) & 255) != 0 ||
-        fwd_workspace_bytes < dilattn_fwd_workspace_size(B, N, H, d, w, r, npat))
-      return DILATTN_ERR_WORKSPACE;
-    PatternGeom geo[kMaxPat];
-    const long long rows = make_geoms(B, N, H, w, r, npat, geo);
-    out_f32 = fwd_out_f32(const_cast<void*>(fwd_workspace), rows, d);
-    if (overlaps(fwd_workspace, fwd_workspace_bytes, workspace, workspace_bytes))
-      return DILATTN_ERR_INVALID_ARG;
-  }
-  return launch_bwd(q, k, v, out, lse, dout, dq, dk, dv, B, N, H, w, r, npat, causal, out_f32,
+  return launch_bwd(q, k, v, out, out_res, lse, dout, dq, dk, dv, B, N, H, w, r, npat, causal,
                     workspace, st, stream);
 }
 
@@ -687,6 +804,76 @@ int dilattn_selection(uint32_t* sig, int N, int H, const int* w, const int* r, i
   return DILATTN_OK;
 }
 
+int dilattn_pack_dilated(const void* x, void* buf, int B, int L, int H, int d, int r,
+                         cudaStream_t stream) {
+  if (B < 1 || L < 1 || H < 1 || r < 1 || L % r != 0 || (d != 64 && d != 128))
+    return DILATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(buf)) return DILATTN_ERR_INVALID_ARG;
+  const size_t bytes = (size_t)B * L * H * d * 2;
+  if (overlaps(x, bytes, buf, bytes / r)) return DILATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  int rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  const long long n16 = (long long)B * (L / r) * H * (d / 8);  // 16-byte pieces
+  const long long blocks = std::min<long long>((n16 + 255) / 256, (long long)st->num_sms * 32);
+  pack_dilated_kernel<<<(unsigned)blocks, 256, 0, stream>>>(
+      reinterpret_cast<const uint4*>(x), reinterpret_cast<uint4*>(buf), B, L, H, d / 8, r);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pack_dilated_kernel launch");
+  return DILATTN_OK;
+}
+
+int dilattn_fwd_seqpar(const void* q, const void* k, const void* v, void* out, float* lse, int B,
+                       int L, int H, int d, const int* w, const int* r, int npat, int causal,
+                       int rank, int world, const void* const* kg, const void* const* vg,
+                       cudaStream_t stream) {
+  int rc = check_fwd_args(q, k, v, out, lse, B, L, H, d, w, r, npat, causal);
+  if (rc != DILATTN_OK) return rc;
+  if (world < 1 || rank < 0 || rank >= world || (long long)L * world > 0x7fffffffLL)
+    return DILATTN_ERR_INVALID_ARG;
+  const long long N = (long long)L * world;
+  SeqParPlan sp;
+  memset(&sp, 0, sizeof(sp));
+  int wl[kMaxPat];
+  for (int i = 0; i < npat; ++i) {
+    if (w[i] <= L) {  // every segment lies in one rank's block
+      if (L % w[i] != 0) return DILATTN_ERR_INVALID_ARG;
+      wl[i] = w[i];
+      continue;
+    }
+    const long long span = std::min<long long>(w[i], N);  // a segment spans span / L ranks
+    if (span % L != 0 || (w[i] < N && N % w[i] != 0) || L % r[i] != 0 || (L / r[i]) % BM != 0)
+      return DILATTN_ERR_INVALID_ARG;
+    if (kg == nullptr || vg == nullptr || !aligned16(kg[i]) || !aligned16(vg[i]))
+      return DILATTN_ERR_INVALID_ARG;
+    wl[i] = L;  // this rank's kept rows: offset h mod r, stride r, over its whole block
+    sp.ranks[i] = (int)(span / L);
+    sp.kv_rank_rows[i] = L / r[i];
+    sp.kv_rows[i] = sp.ranks[i] * sp.kv_rank_rows[i];
+    sp.toff[i] = (rank % sp.ranks[i]) * (sp.kv_rank_rows[i] / BM);
+    sp.kg[i] = kg[i];
+    sp.vg[i] = vg[i];
+  }
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  cudaMemPool_t pool = nullptr;
+  rc = scratch_pool(st, &pool);
+  if (rc != DILATTN_OK) return rc;
+  const size_t need = fwd_scratch_bytes(B, L, H, d, wl, r, npat);
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&scratch, need, pool, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync (forward scratch)");
+  rc = d == 64
+      ? launch_fwd<64>(q, k, v, out, nullptr, lse, B, L, H, wl, r, npat, causal, scratch, st,
+                       stream, &sp)
+      : launch_fwd<128>(q, k, v, out, nullptr, lse, B, L, H, wl, r, npat, causal, scratch, st,
+                        stream, &sp);
+  e = cudaFreeAsync(scratch, stream);
+  if (rc == DILATTN_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync (forward scratch)");
+  return rc;
+}
+
 int dilattn_set_trace_events(cudaEvent_t tile_begin, cudaEvent_t tile_end) {
   if ((tile_begin == nullptr) != (tile_end == nullptr)) return DILATTN_ERR_INVALID_ARG;
   g_trace_begin = tile_begin;
@@ -760,26 +947,13 @@ int noalloc_scratch(void** out) {
 extern "C" int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
                                    float* lse, int B, int N, int H, int d, const int* w,
                                    const int* r, int npat, int causal, cudaStream_t stream) {
-  int rc = check_shape(B, N, H, d, w, r, npat, causal);
+  int rc = check_fwd_args(q, k, v, out, lse, B, N, H, d, w, r, npat, causal);
   if (rc != DILATTN_OK) return rc;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-    return DILATTN_ERR_INVALID_ARG;
-  if (lse != nullptr && !aligned16(lse)) return DILATTN_ERR_INVALID_ARG;
-  const size_t tb = (size_t)B * N * H * d * 2;
-  if (overlaps(out, tb, q, tb) || overlaps(out, tb, k, tb) || overlaps(out, tb, v, tb))
-    return DILATTN_ERR_INVALID_ARG;
-  if (lse != nullptr) {
-    const size_t lb = (size_t)B * H * N * 4;
-    if (overlaps(lse, lb, q, tb) || overlaps(lse, lb, k, tb) || overlaps(lse, lb, v, tb) ||
-        overlaps(lse, lb, out, tb))
-      return DILATTN_ERR_INVALID_ARG;
-  }
-  if (d != 64 && d != 128) return DILATTN_ERR_UNSUPPORTED;
-  const size_t need = dilattn_fwd_workspace_size(B, N, H, d, w, r, npat);
+  const size_t need = fwd_scratch_bytes(B, N, H, d, w, r, npat);
   if (need > (size_t)DILATTN_NOALLOC_SCRATCH_BYTES) {
     snprintf(g_last_error, sizeof(g_last_error),
              "dilattn_fwd_noalloc: this problem needs %zu bytes of scratch; the built-in "
-             "scratch holds %zu bytes (use dilattn_fwd with a workspace)",
+             "scratch holds %zu bytes (use dilattn_fwd)",
              need, (size_t)DILATTN_NOALLOC_SCRATCH_BYTES);
     return DILATTN_ERR_WORKSPACE;
   }
@@ -790,6 +964,8 @@ extern "C" int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, 
   rc = noalloc_scratch(&scratch);
   if (rc != DILATTN_OK) return rc;
   if (d == 64)
-    return launch_fwd<64>(q, k, v, out, lse, B, N, H, w, r, npat, causal, scratch, st, stream);
-  return launch_fwd<128>(q, k, v, out, lse, B, N, H, w, r, npat, causal, scratch, st, stream);
+    return launch_fwd<64>(q, k, v, out, nullptr, lse, B, N, H, w, r, npat, causal, scratch, st,
+                          stream);
+  return launch_fwd<128>(q, k, v, out, nullptr, lse, B, N, H, w, r, npat, causal, scratch, st,
+                         stream);
 }

@@ -48,15 +48,76 @@ struct FwdParams {
   CUtensorMap tmq_t[kMaxPat]; // phases [0, N mod r), floor(N/r) + 1 rows
   CUtensorMap tmk_t[kMaxPat];
   CUtensorMap tmv_t[kMaxPat];
-  CUtensorMap tm_po;          // partial outputs [rows][D] fp32, box 32 x 128 (128-byte swizzle)
   PatternGeom pat[kMaxPat];
   int npat, B, N, H, causal;
   float scale_log2;  // log2(e) / sqrt(d)
-  Sched sched;
-  float* part_o;    // [rows][D]
-  float* part_lse;  // [rows] natural-log lse of each pattern's partial
+  Sched sched;       // tiles of every pattern that stores partials, longest first
+  Sched sched_m;     // tiles of the merging pattern (r = 1), longest first, after those
+  long long units_p; // units of `sched`
+  int merger;        // index of the merging pattern, or -1 (a separate merge kernel combines)
+  int* counter;      // ticket counter: the order in which CTAs take units (zero at launch)
+  int* flags;        // one per 128-row block of partial rows: nonzero once the block is stored
+  float* part_o;     // [rows][D] normalised per-pattern outputs
+  float* part_lse;   // [rows] natural-log lse of each pattern's partial
+  __nv_bfloat16* out;      // [B][N][H][D]
+  __nv_bfloat16* out_res;  // [B][N][H][D] bf16(O - out), the rounding residual; may be null
+  float* lse;              // [B][H][N], may be null
+  // Sequence-parallel rank (LongNet's distributed algorithm): for a pattern
+  // whose segments span several ranks, K and V come from a gathered buffer
+  // [ranks][B][kv_rank_rows][H][D] of every rank's dilated rows of the
+  // segment (kv_rows = ranks * kv_rank_rows rows per head, a multiple of 128),
+  // and this rank's query tiles start at key tile toff of that sequence.
+  int kv_rows[kMaxPat];       // 0: K and V from the strided views of k, v
+  int kv_rank_rows[kMaxPat];
+  int toff[kMaxPat];
   ErrCtx err;  // device error word and this launch's tag
 };
+
+// Acquire load of a flag word (gpu scope).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait for a partial block's flag, same limits as mbar_wait.
+__device__ __forceinline__ bool wait_flag(const int* f, volatile int* abort, const ErrCtx& err) {
+  if (ld_acquire_gpu(f) != 0) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(128);
+    if (ld_acquire_gpu(f) != 0) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (err.raised()) {
+        *abort = 1;
+        return false;
+      }
+      if (globaltimer_ns() - t0 > 4000000000ull) {
+        err.raise(kErrWaitTimeout);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Partial row of position n in pattern g for head h of slice bh (= b * H + h),
+// if g keeps n: segment n / w, kept iff (n - start - h mod r) is a
+// non-negative multiple of r.
+__device__ __forceinline__ bool partial_row(const PatternGeom& g, int n, int h, int bh,
+                                            long long& pr) {
+  const uint32_t seg = (uint32_t)n / (uint32_t)g.w;
+  const int rel = n - (int)(seg * (uint32_t)g.w) - h % g.r;
+  if (rel < 0) return false;
+  const uint32_t v = (uint32_t)rel / (uint32_t)g.r;
+  if ((int)(v * (uint32_t)g.r) != rel) return false;
+  pr = g.part_base + ((long long)bh * g.nseg + seg) * g.pstride + v;
+  return true;
+}
 
 template <int D>
 struct FwdCfg {
@@ -78,6 +139,77 @@ struct FwdCfg {
   static constexpr int THREADS = 64 + 32 * SM_WARPS;
 };
 
+// Epilogue of a tile of the merging pattern (r = 1, so it keeps every row):
+// the tile's own online softmax (O in TMEM relative to m_run, sum l_run, in
+// log2 units) is combined with the stored partials (O_i normalised, lse_i)
+// of every other pattern that keeps the row, weighting each by its share of
+// the shared denominator: O = sum_i Z_i O_i / sum_i Z_i, lse = log sum_i Z_i.
+// One thread per row; out is written once, in bf16 (and, for training, the
+// bf16 rounding residual of out, so that the backward's D = dO . O keeps
+// fp32-grade accuracy).
+template <int D>
+__device__ __forceinline__ void merge_epilogue(const FwdParams& p, const TileUnit& wu,
+                                               const SegInfo& si, int vq, uint32_t tl_o,
+                                               float m_run, float l_run,
+                                               volatile int* abort_flag) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  float acc[D];
+#pragma unroll
+  for (int c4 = 0; c4 < D / 32; ++c4) {
+    uint32_t r[32];
+    tmem_ld32_sync(tl_o + c4 * 32, r);  // warp-collective: every lane loads
+#pragma unroll
+    for (int c = 0; c < 32; ++c) acc[c4 * 32 + c] = __uint_as_float(r[c]);
+  }
+  if (vq >= si.n) return;
+  const int n = (int)si.start + vq;  // r = 1, offset 0
+  const int bh = wu.b * p.H + wu.h;
+  const float own = m_run + __log2f(l_run);
+  float M = own;
+  for (int i = 0; i < p.npat; ++i) {
+    long long pr;
+    if (i == p.merger || !partial_row(p.pat[i], n, wu.h, bh, pr)) continue;
+    if (!wait_flag(p.flags + (pr >> 7), abort_flag, p.err)) return;
+    M = fmaxf(M, __ldcg(p.part_lse + pr) * kLog2e);
+  }
+  float Z = ex2(own - M);
+  const float w_own = Z / l_run;
+#pragma unroll
+  for (int c = 0; c < D; ++c) acc[c] *= w_own;
+  for (int i = 0; i < p.npat; ++i) {
+    long long pr;
+    if (i == p.merger || !partial_row(p.pat[i], n, wu.h, bh, pr)) continue;
+    const float wi = ex2(__ldcg(p.part_lse + pr) * kLog2e - M);
+    Z += wi;
+    const float4* src = reinterpret_cast<const float4*>(p.part_o + pr * D);
+#pragma unroll
+    for (int e = 0; e < D / 4; ++e) {
+      const float4 x = __ldcg(src + e);
+      acc[4 * e] = fmaf(wi, x.x, acc[4 * e]);
+      acc[4 * e + 1] = fmaf(wi, x.y, acc[4 * e + 1]);
+      acc[4 * e + 2] = fmaf(wi, x.z, acc[4 * e + 2]);
+      acc[4 * e + 3] = fmaf(wi, x.w, acc[4 * e + 3]);
+    }
+  }
+  const float inv = 1.f / Z;
+  const long long o0 = (((long long)wu.b * p.N + n) * p.H + wu.h) * D;
+  uint4* dst = reinterpret_cast<uint4*>(p.out + o0);
+  uint4* rdst = p.out_res != nullptr ? reinterpret_cast<uint4*>(p.out_res + o0) : nullptr;
+#pragma unroll
+  for (int e = 0; e < D / 8; ++e) {
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float a = acc[8 * e + 2 * j] * inv, b = acc[8 * e + 2 * j + 1] * inv;
+      hi[j] = pack_bf16_rn(a, b);
+      lo[j] = pack_bf16_rn(a - __uint_as_float(hi[j] << 16), b - __uint_as_float(hi[j] & 0xffff0000u));
+    }
+    dst[e] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    if (rdst != nullptr) rdst[e] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+  if (p.lse != nullptr) p.lse[(long long)bh * p.N + n] = (M + __log2f(Z)) * 0.69314718055994531f;
+}
+
 template <int D>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     fwd_tile_kernel(const __grid_constant__ FwdParams p) {
@@ -87,11 +219,23 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   const uint32_t base = (raw_s + 1023u) & ~1023u;
   uint8_t* base_g = smem_raw + (base - raw_s);
 
-  const TileUnit wu = decode_unit(p.sched, p.pat, p.B, p.H, blockIdx.x);
+  // Units are taken in ticket order, not blockIdx order: every tile that
+  // stores partials has a smaller ticket than every merging tile, so a merging
+  // tile only ever waits for tiles that running CTAs already hold.
+  __shared__ int s_ticket;
+  if (threadIdx.x == 0) s_ticket = atomicAdd(p.counter, 1);
+  __syncthreads();
+  const long long ticket = s_ticket;
+  const TileUnit wu = ticket < p.units_p
+      ? decode_unit(p.sched, p.pat, p.B, p.H, ticket)
+      : decode_unit(p.sched_m, p.pat, p.B, p.H, ticket - p.units_p);
   const PatternGeom g = p.pat[wu.pat];
   const SegInfo si = seg_info(g, p.N, wu.h, wu.seg);
   if (wu.t * BM >= si.n) return;  // tile past the segment's kept rows (uniform exit)
-  const int nkv = p.causal ? (wu.t + 1) : (si.n + BN - 1) / BN;
+  const bool gathered = p.kv_rows[wu.pat] > 0;
+  const int kv_n = gathered ? p.kv_rows[wu.pat] : si.n;  // key rows of the segment
+  const int tq = wu.t + p.toff[wu.pat];                   // the query tile among the key tiles
+  const int nkv = p.causal ? (tq + 1) : (kv_n + BN - 1) / BN;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -109,7 +253,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   const uint32_t b_sfree = b_sfull + 8u;
   const uint32_t b_pfull = b_sfull + 16u;
   const uint32_t b_odone = b_sfull + 24u;
-  const uint32_t b_epi = b_sfull + 32u;  // the four softmax warps have staged their output rows
+  const uint32_t b_epi = b_sfull + 32u;  // the four softmax warps have stored their partial rows
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
 
@@ -137,8 +281,19 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
   view_coords(g, si, 0, phase0, m0);
   const bool tail_view = phase0 < g.nmod;
   const CUtensorMap* mq = tail_view ? &p.tmq_t[wu.pat] : &p.tmq[wu.pat];
-  const CUtensorMap* mk = tail_view ? &p.tmk_t[wu.pat] : &p.tmk[wu.pat];
-  const CUtensorMap* mv = tail_view ? &p.tmv_t[wu.pat] : &p.tmv[wu.pat];
+  const CUtensorMap* mk = tail_view && !gathered ? &p.tmk_t[wu.pat] : &p.tmk[wu.pat];
+  const CUtensorMap* mv = tail_view && !gathered ? &p.tmv_t[wu.pat] : &p.tmv[wu.pat];
+  // coordinates of key tile `it`: the strided view's (phase, row), or the
+  // gathered buffer's (row within a rank's block, rank)
+  auto kv_coords = [&](int it, int& c2, int& c3) {
+    if (gathered) {
+      const uint32_t j = (uint32_t)(it * BN), rr = (uint32_t)p.kv_rank_rows[wu.pat];
+      c3 = (int)(j / rr);
+      c2 = (int)(j - (uint32_t)c3 * rr);
+    } else {
+      view_coords(g, si, it * BN, c2, c3);
+    }
+  };
   if (warp == 0 && lane == 0) {
     prefetch_tmap(mq);
     prefetch_tmap(mk);
@@ -166,7 +321,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       for (int it = 0; it < nkv; ++it) {
         const int s = it % C::KST;
         if (!mbar_wait(b_kempty(s), ((it / C::KST) & 1) ^ 1, abort_flag, p.err)) break;
-        view_coords(g, si, it * BN, ph, m);
+        kv_coords(it, ph, m);
         mbar_arrive_expect_tx(b_kfull(s), C::KV_BYTES);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_5d(sK + s * C::KV_BYTES + c * C::CHUNK_BYTES, mk, b_kfull(s), c * 64, wu.h, ph,
@@ -186,7 +341,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       for (int it = 0; it < nkv; ++it) {
         const int s = it % C::VST;
         if (!mbar_wait(b_vempty(s), ((it / C::VST) & 1) ^ 1, abort_flag, p.err)) break;
-        view_coords(g, si, it * BN, ph, m);
+        kv_coords(it, ph, m);
         mbar_arrive_expect_tx(b_vfull(s), C::KV_BYTES);
         for (int c = 0; c < C::KCH; ++c)
           tma_load_5d(sV + s * C::KV_BYTES + c * C::CHUNK_BYTES, mv, b_vfull(s), c * 64, wu.h, ph,
@@ -280,13 +435,13 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       if (lane == 0) mbar_arrive(b_sfree);
 
       if (p.causal) {
-        if (it == wu.t) {
+        if (it == tq) {
 #pragma unroll
           for (int c = 0; c < BN; ++c)
             if (c > row) raw[c] = 0xff800000u;  // -inf
         }
       } else if (it == nkv - 1) {
-        const int lim = si.n - it * BN;
+        const int lim = kv_n - it * BN;
 #pragma unroll
         for (int c = 0; c < BN; ++c)
           if (c >= lim) raw[c] = 0xff800000u;
@@ -361,40 +516,39 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     }
     if (ok && warp_wait(b_odone, (nkv - 1) & 1, abort_flag, p.err)) {
       tc_fence_after();
-      // The tile's 128 partial rows are one contiguous block of the partial
-      // buffer (segments own whole tiles there; rows past the segment land in
-      // padding no one reads). O / l goes through the now idle K ring, staged
-      // as D/32 chunks of [128 rows][32 fp32] with 128-byte swizzle, and leaves
-      // by TMA stores.
-      const long long prow0 =
-          g.part_base + ((long long)(wu.b * p.H + wu.h) * g.nseg + wu.seg) * g.pstride +
-          (long long)wu.t * BM;
-      const float inv = 1.f / l_run;
-      uint8_t* stg = base_g + C::OFF_K;
+      if (wu.pat == p.merger) {
+        merge_epilogue<D>(p, wu, si, vq, tl + C::TM_O, m_run, l_run, abort_flag);
+      } else {
+        // The tile's 128 partial rows are one contiguous block of the partial
+        // buffer (segments own whole tiles there); each thread stores its row
+        // of O / l and its lse, then the block's flag is released.
+        const long long prow0 =
+            g.part_base + ((long long)(wu.b * p.H + wu.h) * g.nseg + wu.seg) * g.pstride +
+            (long long)wu.t * BM;
+        const float inv = 1.f / l_run;
+        float4* dst = reinterpret_cast<float4*>(p.part_o + (prow0 + row) * D);
 #pragma unroll
-      for (int c4 = 0; c4 < D / 32; ++c4) {
-        uint32_t r[32];
-        tmem_ld32_sync(tl + C::TM_O + c4 * 32, r);
-        uint8_t* rowp = stg + c4 * (BM * 128) + row * 128;
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          uint32_t r[32];
+          tmem_ld32_sync(tl + C::TM_O + c4 * 32, r);
+          if (vq < si.n) {
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          const float4 v = make_float4(__uint_as_float(r[4 * k]) * inv,
-                                       __uint_as_float(r[4 * k + 1]) * inv,
-                                       __uint_as_float(r[4 * k + 2]) * inv,
-                                       __uint_as_float(r[4 * k + 3]) * inv);
-          *reinterpret_cast<float4*>(rowp + ((k ^ (row & 7)) * 16)) = v;
+            for (int k = 0; k < 8; ++k)
+              dst[c4 * 8 + k] = make_float4(__uint_as_float(r[4 * k]) * inv,
+                                            __uint_as_float(r[4 * k + 1]) * inv,
+                                            __uint_as_float(r[4 * k + 2]) * inv,
+                                            __uint_as_float(r[4 * k + 3]) * inv);
+          }
         }
-      }
-      if (vq < si.n) p.part_lse[prow0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(b_epi);
-      if (warp_wait(b_epi, 0, abort_flag, p.err) && warp == 2 && lane == 0) {
-#pragma unroll
-        for (int c4 = 0; c4 < D / 32; ++c4)
-          tma_store_2d(&p.tm_po, sK + c4 * (BM * 128), c4 * 32, (int)prow0);
-        bulk_commit();
-        bulk_wait_read<0>();  // the staging buffer stays until the stores have read it
+        if (vq < si.n) p.part_lse[prow0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
+        // every writer fences its stores; the block's flag is released once
+        // all four softmax warps have (a bounded wait: an aborted warp never
+        // arrives, and then no flag is released)
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_epi);
+        if (warp == 2 && lane == 0 && mbar_wait(b_epi, 0, abort_flag, p.err))
+          st_release_gpu(p.flags + (prow0 >> 7), 1);
       }
     }
     tc_fence_before();

@@ -46,8 +46,8 @@ struct MergeParams {
   const float* part_o;
   const float* part_lse;
   __nv_bfloat16* out;
-  float* out_f32;  // fp32 copy of out (for the backward's D)
-  float* lse;      // may be null
+  __nv_bfloat16* out_res;  // bf16(O - out), may be null
+  float* lse;              // may be null
 };
 
 // DILATTN_MERGE_TPR threads per output row (default 4; 8 and 16 were measured
@@ -110,24 +110,56 @@ __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ Merg
     for (int e = 0; e < PER; ++e) acc[e] *= inv;
     L = m + logf(l);
   }
-  float4* dst32 = reinterpret_cast<float4*>(p.out_f32 + row * D + sub * PER);
+  uint32_t pk[PER / 2], rk[PER / 2];
 #pragma unroll
-  for (int e = 0; e < PER / 4; ++e)
-    dst32[e] = make_float4(acc[4 * e], acc[4 * e + 1], acc[4 * e + 2], acc[4 * e + 3]);
-  uint32_t pk[PER / 2];
-#pragma unroll
-  for (int e = 0; e < PER / 2; ++e) pk[e] = pack_bf16(acc[2 * e], acc[2 * e + 1]);
+  for (int e = 0; e < PER / 2; ++e) {
+    pk[e] = pack_bf16(acc[2 * e], acc[2 * e + 1]);
+    rk[e] = pack_bf16(acc[2 * e] - __uint_as_float(pk[e] << 16),
+                      acc[2 * e + 1] - __uint_as_float(pk[e] & 0xffff0000u));
+  }
   if (PER % 8 == 0) {
     uint4* dst = reinterpret_cast<uint4*>(p.out + row * D + sub * PER);
+    uint4* rdst = p.out_res != nullptr ? reinterpret_cast<uint4*>(p.out_res + row * D + sub * PER)
+                                       : nullptr;
 #pragma unroll
-    for (int e = 0; e < PER / 8; ++e)
+    for (int e = 0; e < PER / 8; ++e) {
       dst[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+      if (rdst != nullptr) rdst[e] = make_uint4(rk[4 * e], rk[4 * e + 1], rk[4 * e + 2], rk[4 * e + 3]);
+    }
   } else {
     uint2* dst = reinterpret_cast<uint2*>(p.out + row * D + sub * PER);
+    uint2* rdst = p.out_res != nullptr ? reinterpret_cast<uint2*>(p.out_res + row * D + sub * PER)
+                                       : nullptr;
 #pragma unroll
-    for (int e = 0; e < PER / 4; ++e) dst[e] = make_uint2(pk[2 * e], pk[2 * e + 1]);
+    for (int e = 0; e < PER / 4; ++e) {
+      dst[e] = make_uint2(pk[2 * e], pk[2 * e + 1]);
+      if (rdst != nullptr) rdst[e] = make_uint2(rk[2 * e], rk[2 * e + 1]);
+    }
   }
   if (p.lse != nullptr && sub == 0) p.lse[(long long)bh * p.N + n] = L;
+}
+
+// ---------------------------------------------------------------------------
+// Dilated rows of one rank's block for a sequence-parallel pattern:
+// buf[b][m][h] = x[b][(h mod r) + m r][h] for m < L / r (rows of 16-byte
+// pieces; pieces = d / 8 per row).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) pack_dilated_kernel(const uint4* __restrict__ x,
+                                                           uint4* __restrict__ buf, int B, int L,
+                                                           int H, int pieces, int r) {
+  const long long Lr = L / r;
+  const long long total = (long long)B * Lr * H * pieces;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(i % pieces);
+    long long t = i / pieces;
+    const int h = (int)(t % H);
+    t /= H;
+    const long long m = t % Lr;
+    const long long b = t / Lr;
+    const long long src_row = b * L + (h % r) + m * r;
+    buf[i] = x[(src_row * H + h) * pieces + c];
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -29,12 +29,13 @@ _ip = _c.POINTER(_c.c_int)
 SIGNATURES = {
     "dilattn_status_string": (_c.c_char_p, [_i]),
     "dilattn_last_error": (_c.c_char_p, []),
-    "dilattn_fwd_workspace_size": (_sz, [_i, _i, _i, _i, _ip, _ip, _i]),
-    "dilattn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp, _sz, _vp]),
+    "dilattn_fwd_scratch_size": (_sz, [_i, _i, _i, _i, _ip, _ip, _i]),
+    "dilattn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
+    "dilattn_fwd_train": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
     "dilattn_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
-    "dilattn_bwd_workspace_size": (_sz, [_i, _i, _i, _i, _ip, _ip, _i]),
-    "dilattn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i,
-                         _i, _vp, _sz, _vp, _sz, _vp]),
+    "dilattn_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
+    "dilattn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip,
+                         _i, _i, _vp, _sz, _vp]),
     "dilattn_fwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
     "dilattn_bwd_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip,
                              _i, _i, _vp]),
@@ -42,6 +43,9 @@ SIGNATURES = {
     "dilattn_set_trace_events": (_i, [_vp, _vp]),
     "dilattn_device_error": (_i, [_vp, _ip]),
     "dilattn_selftest_wait_timeout": (_i, [_c.c_ulonglong, _vp, _vp]),
+    "dilattn_fwd_seqpar": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _i, _i,
+                                _c.POINTER(_vp), _c.POINTER(_vp), _vp]),
+    "dilattn_pack_dilated": (_i, [_vp, _vp, _i, _i, _i, _i, _i, _vp]),
 }
 
 _lib = None
@@ -117,18 +121,16 @@ def _shape(q):
     return tuple(int(x) for x in q.shape)
 
 
-def fwd_workspace_size(B, N, H, d, patterns) -> int:
+def fwd_scratch_size(B, N, H, d, patterns) -> int:
     w, r, n = _patterns(patterns)
-    return int(load().dilattn_fwd_workspace_size(B, N, H, d, w, r, n))
+    return int(load().dilattn_fwd_scratch_size(B, N, H, d, w, r, n))
 
 
-def bwd_workspace_size(B, N, H, d, patterns) -> int:
-    w, r, n = _patterns(patterns)
-    return int(load().dilattn_bwd_workspace_size(B, N, H, d, w, r, n))
+def bwd_workspace_size(B, N, H, d) -> int:
+    return int(load().dilattn_bwd_workspace_size(B, N, H, d))
 
 
-def fwd(q, k, v, patterns, causal: bool = True, out=None, lse=None, workspace=None,
-        stream=None):
+def fwd(q, k, v, patterns, causal: bool = True, out=None, lse=None, stream=None):
     """Merged dilated attention. bf16 tensors go to dilattn_fwd, float32 to dilattn_fwd_f32.
 
     Returns (out [B, N, H, d] in q's dtype, lse [B, H, N] float32).
@@ -149,12 +151,8 @@ def fwd(q, k, v, patterns, causal: bool = True, out=None, lse=None, workspace=No
     s = _stream_handle(stream)
     lib = load()
     if q.dtype == torch.bfloat16:
-        need = int(lib.dilattn_fwd_workspace_size(B, N, H, d, w, r, n))
-        if workspace is None:
-            workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
         rc = lib.dilattn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                             lse.data_ptr(), B, N, H, d, w, r, n, int(causal),
-                             workspace.data_ptr(), workspace.numel() * workspace.element_size(), s)
+                             lse.data_ptr(), B, N, H, d, w, r, n, int(causal), s)
         _check(rc, "dilattn_fwd")
     elif q.dtype == torch.float32:
         rc = lib.dilattn_fwd_f32(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
@@ -165,33 +163,51 @@ def fwd(q, k, v, patterns, causal: bool = True, out=None, lse=None, workspace=No
     return out, lse
 
 
-def bwd(q, k, v, out, lse, dout, patterns, causal: bool = True, dq=None, dk=None, dv=None,
-        workspace=None, stream=None, fwd_workspace=None):
-    """Gradients (dq, dk, dv) of sum(out * dout) for the forward that produced out, lse.
+def fwd_train(q, k, v, patterns, causal: bool = True, out=None, lse=None, out_res=None,
+              stream=None):
+    """dilattn_fwd_train on bf16 tensors: (out, lse, out_res), out_res the bf16
+    rounding residual of out that the backward forms its row term from."""
+    torch = _torch()
+    B, N, H, d = _shape(q)
+    if q.dtype != torch.bfloat16:
+        raise ValueError("fwd_train takes bf16 tensors (the fp32 path needs no residual)")
+    out = torch.empty_like(q) if out is None else out
+    out_res = torch.empty_like(q) if out_res is None else out_res
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    w, r, n = _patterns(patterns)
+    rc = load().dilattn_fwd_train(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                  out_res.data_ptr(), lse.data_ptr(), B, N, H, d, w, r, n,
+                                  int(causal), _stream_handle(stream))
+    _check(rc, "dilattn_fwd_train")
+    return out, lse, out_res
 
-    ``fwd_workspace``: the workspace tensor of that forward call (bf16 only),
-    so the backward can take D = rowsum(dout * out) from the forward's fp32
-    copy of out; None uses the bf16 out."""
+
+def bwd(q, k, v, out, lse, dout, patterns, causal: bool = True, out_res=None, dq=None, dk=None,
+        dv=None, workspace=None, stream=None):
+    """Gradients (dq, dk, dv), float32, of sum(O * dout) for the forward that produced
+    out, lse (and, for bf16, out_res: use fwd_train)."""
     torch = _torch()
     B, N, H, d = _shape(q)
     for t in (k, v, out, dout):
         if tuple(t.shape) != (B, N, H, d) or t.dtype != q.dtype:
             raise ValueError("q, k, v, out, dout must share shape and dtype")
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(q) if dk is None else dk
-    dv = torch.empty_like(q) if dv is None else dv
+    gdt = torch.float32  # the bf16 path returns fp32 gradients, the fp32 path fp32 too
+    dq = torch.empty(q.shape, dtype=gdt, device=q.device) if dq is None else dq
+    dk = torch.empty(q.shape, dtype=gdt, device=q.device) if dk is None else dk
+    dv = torch.empty(q.shape, dtype=gdt, device=q.device) if dv is None else dv
     w, r, n = _patterns(patterns)
     s = _stream_handle(stream)
     lib = load()
     if q.dtype == torch.bfloat16:
-        need = int(lib.dilattn_bwd_workspace_size(B, N, H, d, w, r, n))
+        if out_res is None:
+            raise ValueError("the bf16 backward takes out_res from fwd_train")
+        need = int(lib.dilattn_bwd_workspace_size(B, N, H, d))
         if workspace is None:
             workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-        fptr = fwd_workspace.data_ptr() if fwd_workspace is not None else None
-        fbytes = fwd_workspace.numel() * fwd_workspace.element_size() if fwd_workspace is not None else 0
         rc = lib.dilattn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                             lse.data_ptr(), dout.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                             dv.data_ptr(), B, N, H, d, w, r, n, int(causal), fptr, fbytes,
+                             out_res.data_ptr(), lse.data_ptr(), dout.data_ptr(), dq.data_ptr(),
+                             dk.data_ptr(), dv.data_ptr(), B, N, H, d, w, r, n, int(causal),
                              workspace.data_ptr(), workspace.numel() * workspace.element_size(), s)
         _check(rc, "dilattn_bwd")
     elif q.dtype == torch.float32:
@@ -258,4 +274,37 @@ def fwd_noalloc(q, k, v, patterns, causal: bool = True, out=None, lse=None, stre
                                     lse.data_ptr(), B, N, H, d, w, r, n, int(causal),
                                     _stream_handle(stream))
     _check(rc, "dilattn_fwd_noalloc")
+    return out, lse
+
+
+def pack_dilated(x, r: int, out=None, stream=None):
+    """dilattn_pack_dilated: [B, L/r, H, d] with row m of head h = x[:, (h mod r) + m r, h]."""
+    torch = _torch()
+    B, L, H, d = _shape(x)
+    if out is None:
+        out = torch.empty((B, L // r, H, d), dtype=x.dtype, device=x.device)
+    rc = load().dilattn_pack_dilated(x.data_ptr(), out.data_ptr(), B, L, H, d, int(r),
+                                     _stream_handle(stream))
+    _check(rc, "dilattn_pack_dilated")
+    return out
+
+
+def fwd_seqpar(q, k, v, patterns, rank: int, world: int, kg=None, vg=None, causal: bool = True,
+               out=None, lse=None, stream=None):
+    """dilattn_fwd_seqpar on this rank's block; kg / vg: per pattern the gathered
+    [ranks, B, L/r, H, d] buffer or None."""
+    torch = _torch()
+    B, L, H, d = _shape(q)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    w, r, n = _patterns(patterns)
+    ptr = lambda t: t.data_ptr() if t is not None else None
+    kga = (_vp * max(n, 1))(*[ptr(t) for t in (kg or [None] * n)])
+    vga = (_vp * max(n, 1))(*[ptr(t) for t in (vg or [None] * n)])
+    rc = load().dilattn_fwd_seqpar(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   lse.data_ptr(), B, L, H, d, w, r, n, int(causal), int(rank),
+                                   int(world), kga, vga, _stream_handle(stream))
+    _check(rc, "dilattn_fwd_seqpar")
     return out, lse

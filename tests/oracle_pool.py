@@ -243,8 +243,9 @@ def bwd_rows(inputs: Dict[str, np.ndarray], qrows, krows, patterns, causal: bool
     shared = {n: _Shared(a) for n, a in inputs.items()}
     try:
         specs = {n: s.spec for n, s in shared.items()}
-        tasks = [(specs, "q", r, tuple(map(tuple, patterns)), causal) for r in qrows]
-        tasks += [(specs, "k", r, tuple(map(tuple, patterns)), causal) for r in krows]
+        pats = tuple(map(tuple, patterns))
+        tasks = [(specs, "q", r, pats, causal) for r in qrows]
+        tasks += [(specs, "k", r, pats, causal) for r in krows]
         nproc = max(1, min(len(tasks), usable_cpus()))
         ctx = mp.get_context("spawn")
         with _blas_threads(1):

@@ -50,10 +50,18 @@ def _pats(p):
 
 
 def _fwd(B=1, N=256, H=2, d=64, pats=((128, 1),), causal=1, q=FAKE, k=FAKE + 4096 * 1024,
-         v=FAKE + 8192 * 1024, out=FAKE + 16384 * 1024, lse=None, ws=None, wsb=0):
+         v=FAKE + 8192 * 1024, out=FAKE + 16384 * 1024, lse=None):
     w, r, n = _pats(pats)
     lib = dilattn.load()
-    return lib.dilattn_fwd(q, k, v, out, lse, B, N, H, d, w, r, n, causal, ws, wsb, None)
+    return lib.dilattn_fwd(q, k, v, out, lse, B, N, H, d, w, r, n, causal, None)
+
+
+def _bwd(ws=FAKE * 64, wsb=1 << 20, **kw):
+    B, N, H, d = kw.get("B", 1), 256, 2, 64
+    w, r, n = _pats(((128, 1),))
+    base = [FAKE + i * (4096 * 1024) for i in range(10)]  # 4 MiB apart: nothing overlaps
+    lib = dilattn.load()
+    return lib.dilattn_bwd(*base, B, N, H, d, w, r, n, 1, ws, wsb, None)
 
 
 @pytest.mark.parametrize("kw", [
@@ -70,28 +78,55 @@ def test_fwd_rejects_unsupported_head_dim():
     assert _fwd(d=96) == UNSUPPORTED
 
 
-def test_fwd_rejects_missing_or_small_workspace():
-    assert _fwd(ws=None) == WORKSPACE
-    assert _fwd(ws=FAKE * 64, wsb=16) == WORKSPACE
-    assert _fwd(ws=FAKE * 64 + 16, wsb=1 << 30) == WORKSPACE  # not 256-byte aligned
-
-
-def test_workspace_sizes():
+def test_fwd_train_needs_a_residual_buffer():
+    w, r, n = _pats(((128, 1),))
     lib = dilattn.load()
-    w, r, n = _pats(((128, 1), (256, 2), (512, 4)))
-    # partial rows: sum_i B*H*nseg_i*(128*ceil(ceil(min(w,N)/r)/128)) = 2*3*(4*128 + 2*128 + 1*128)
-    rows = 2 * 3 * (512 + 256 + 128)
+    args = (1, 256, 2, 64, w, r, n, 1, None)
+    assert lib.dilattn_fwd_train(FAKE, FAKE + (4 << 20), FAKE + (8 << 20), FAKE + (16 << 20), None,
+                                 None, *args) == INVALID
+    # out_res overlapping out
+    assert lib.dilattn_fwd_train(FAKE, FAKE + (4 << 20), FAKE + (8 << 20), FAKE + (16 << 20),
+                                 FAKE + (16 << 20) + 1024, None, *args) == INVALID
+
+
+def test_bwd_rejects_missing_or_small_workspace():
+    assert _bwd(ws=None) == WORKSPACE
+    assert _bwd(wsb=16) == WORKSPACE
+    assert _bwd(ws=FAKE * 64 + 16) == WORKSPACE  # not 256-byte aligned
+    assert _bwd(ws=FAKE) == INVALID               # overlaps the inputs
+    base = [FAKE + i * (4096 * 1024) for i in range(10)]
+    w, r, n = _pats(((128, 1),))
+    lib = dilattn.load()
+    # q k v out out_res lse dout, then dq dk dv: dk (fp32, 128 KiB) starting inside dq's
+    assert lib.dilattn_bwd(*base[:7], base[7], base[7] + 65536, base[9], 1, 256, 2, 64, w, r, n,
+                           1, FAKE * 64, 1 << 20, None) == INVALID
+    # out_res missing
+    assert lib.dilattn_bwd(*base[:4], None, *base[5:10], 1, 256, 2, 64, w, r, n, 1, FAKE * 64,
+                           1 << 20, None) == INVALID
+
+
+def test_scratch_and_workspace_sizes():
+    lib = dilattn.load()
     align = lambda x: (x + 255) // 256 * 256
-    assert lib.dilattn_fwd_workspace_size(1, 1000, 1, 64, *_pats(((1000, 3),))) == \
-        384 * 64 * 4 + align(384 * 4) + align(1000 * 64 * 4)  # 334 rows -> 384
-    # partial outputs, partial lse, then an fp32 copy of out
-    assert lib.dilattn_fwd_workspace_size(2, 512, 3, 64, w, r, n) == \
-        align(rows * 64 * 4) + align(rows * 4) + align(2 * 512 * 3 * 64 * 4)
-    t = 2 * 512 * 3 * 64 * 4
-    # dq, dk, dv accumulators, D, then 256 bytes for the key-tile kernel's unit counter
-    assert lib.dilattn_bwd_workspace_size(2, 512, 3, 64, w, r, n) == \
-        3 * align(t) + align(2 * 3 * 512 * 4) + 256
-    assert lib.dilattn_fwd_workspace_size(0, 512, 3, 64, w, r, n) == 0
+    w, r, n = _pats(((128, 1), (256, 2), (512, 4)))
+    # the r = 1 pattern merges and stores no partials; partial rows of the
+    # others: B*H*nseg_i*(128*ceil(ceil(min(w,N)/r)/128)) = 2*3*(2*128 + 1*128)
+    rows = 2 * 3 * (256 + 128)
+    flags = align((rows // 128 + 1) * 4 + 4)  # one flag per 128-row block, then the ticket counter
+    assert lib.dilattn_fwd_scratch_size(2, 512, 3, 64, w, r, n) == \
+        align(rows * 64 * 4) + align(rows * 4) + flags
+    # no r = 1 pattern: every pattern stores partials (334 rows -> 384)
+    assert lib.dilattn_fwd_scratch_size(1, 1000, 1, 64, *_pats(((1000, 3),))) == \
+        384 * 64 * 4 + align(384 * 4) + align((384 // 128 + 1) * 4 + 4)
+    # of two r = 1 patterns the shorter merges
+    w2, r2, n2 = _pats(((512, 1), (256, 1)))
+    assert lib.dilattn_fwd_scratch_size(1, 512, 1, 64, w2, r2, n2) == \
+        align(512 * 64 * 4) + align(512 * 4) + align((512 // 128 + 1) * 4 + 4)
+    # D, then 256 bytes for the key-tile kernel's unit counter (the fp32 gradients
+    # are the caller's outputs)
+    assert lib.dilattn_bwd_workspace_size(2, 512, 3, 64) == align(2 * 3 * 512 * 4) + 256
+    assert lib.dilattn_fwd_scratch_size(0, 512, 3, 64, w, r, n) == 0
+    assert lib.dilattn_bwd_workspace_size(0, 512, 3, 64) == 0
 
 
 def test_valid_call_without_gpu_reports_cuda_error():

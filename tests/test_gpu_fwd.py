@@ -38,6 +38,8 @@ def test_tiny_f32_workload():
     [(384, 1), (700, 3), (1000, 6), (1100, 12)],     # ragged: w and r do not divide N
     [(1100, 1)],                                      # one long segment, ragged tail tile
     [(64, 5), (96, 200), (1100, 7)],                  # r > w: empty segments; tiny tiles
+    [(256, 1), (1024, 1), (512, 2)],                  # two r = 1 patterns: the shorter merges
+    [(100, 1), (37, 3), (1100, 1)],                   # merging tiles cross many short segments
 ])
 def test_bf16_small(pats, causal):
     _run_full(2, 1100, 3, 64, pats, causal, "bf16", seed=1)

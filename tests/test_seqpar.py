@@ -1,0 +1,116 @@
+"""Host logic of the sequence-parallel forward, on the CPU.
+
+The plan decides which patterns stay inside a rank's block and how spanning
+patterns are gathered; two and four gloo ranks then run the exchange the GPU
+path runs (each rank sends the rows dilattn_pack_dilated extracts, the ranks
+all-gather in rank order, each keeps its segment's slice) and check the
+result against the oracle's kept rows: the gathered sequence of every head
+must be the segment's kept rows in order, and each rank's query rows must sit
+at the tile offset the kernel is given. The attention arithmetic of that path
+is checked on the GPU against the oracle (tests/test_gpu_seqpar.py)."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import oracle
+from sparse_long_sequence_dilated_b200 import seqpar
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CASES = {
+    2: (2048, [(256, 1), (512, 2), (2048, 4), (1024, 8)]),
+    4: (4096, [(512, 1), (1024, 2), (2048, 4), (4096, 8)]),
+}
+
+
+def test_plan_local_and_spanning_patterns():
+    pl = seqpar.plan(32768, 4, [(2048, 1), (4096, 2), (8192, 4), (16384, 8), (32768, 16)])
+    assert [p.spans for p in pl] == [False, False, False, True, True]
+    assert (pl[3].ranks, pl[3].rank_rows) == (2, 1024)
+    assert (pl[4].ranks, pl[4].rank_rows) == (4, 512)
+    assert pl[3].segment_ranks(3) == [2, 3] and pl[4].segment_ranks(1) == [0, 1, 2, 3]
+    assert pl[3].tile_offset(3) == 8 and pl[4].tile_offset(2) == 8 and pl[0].tile_offset(2) == 0
+    # w larger than N: one segment over every rank
+    pl = seqpar.plan(8192, 2, [(1 << 20, 2)])
+    assert pl[0].spans and pl[0].ranks == 2
+    # segments of 2 blocks of 3072 tile N = 4 blocks
+    assert seqpar.plan(12288, 4, [(6144, 1)])[0].ranks == 2
+
+
+@pytest.mark.parametrize("N,world,pats", [
+    (1000, 3, [(100, 1)]),            # N not a multiple of the ranks
+    (4096, 2, [(1000, 1)]),           # the block is not a multiple of w
+    (4096, 2, [(4096, 3)]),           # L not a multiple of r
+    (4096, 2, [(4096, 32)]),          # L / r not whole tiles
+    (12288, 4, [(9216, 1)]),          # a segment of 3 blocks does not tile 4 blocks
+])
+def test_plan_rejects_splits_the_kernels_do_not_take(N, world, pats):
+    with pytest.raises(ValueError):
+        seqpar.plan(N, world, pats)
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, out_dir: str):
+    import sys
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        N, pats = CASES[world]
+        H, d = 3, 4
+        L = N // world
+        # every rank draws the same full tensor and keeps its block; the value
+        # of a row encodes its position and head, so a misplaced row shows
+        k_full = (np.arange(N)[None, :, None, None] * 10 + np.arange(H)[None, None, :, None]
+                  + 0.25 * np.arange(d)[None, None, None, :]).astype(np.float64)
+        block = torch.from_numpy(k_full[:, rank * L:(rank + 1) * L].copy())
+        bad = []
+        for p in seqpar.plan(N, world, pats):
+            if not p.spans:
+                continue
+            send = torch.empty((1, L // p.r, H, d), dtype=torch.float64)
+            for h in range(H):
+                loc = [x - rank * L for x in seqpar.packed_positions(p, L, rank, h)]
+                send[0, :, h] = block[0, loc, h]
+            recv = [torch.empty_like(send) for _ in range(world)]
+            dist.all_gather(recv, send)
+            seg = p.segment_ranks(rank)
+            gathered = torch.cat([recv[g] for g in seg], dim=1)  # [1, ranks * L / r, H, d]
+            s_idx = (rank * L) // p.w if p.w < N else 0
+            for h in range(H):
+                want = oracle.kept_rows(N, p.w, p.r, h)[s_idx]
+                if not np.array_equal(gathered[0, :, h].numpy(), k_full[0, want, h]):
+                    bad.append(("gathered", p.index, h))
+                # this rank's kept rows sit at the tile offset the kernel gets
+                mine = [x for x in want if rank * L <= x < (rank + 1) * L]
+                first = int(np.searchsorted(want, mine[0]))
+                if first != p.tile_offset(rank) * seqpar.BM or len(mine) != p.rank_rows:
+                    bad.append(("offset", p.index, h))
+        with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
+            f.write(repr(bad))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 4])
+def test_gloo_ranks_gather_the_segments_kept_rows(tmp_path, world):
+    port = _free_port()
+    mp.start_processes(_rank_main, args=(world, port, str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    for r in range(world):
+        assert (tmp_path / f"r{r}.txt").read_text() == "[]"

@@ -5,10 +5,11 @@ its input and output pointers, a server that reserves all device memory at
 start-up and forbids cudaMalloc afterwards. For them the library keeps the
 forward's scratch (per-pattern partial results) in a fixed 64 MiB array of its
 own. These tests run that entry point through the C ABI and compare it with
-dilattn_fwd, which uses a caller workspace, on two calls in a row with
-different shapes, patterns and inputs, so scratch read from the wrong place
-or left over from the first call would show up in the second; and they check
-that a problem too large for the array is refused.
+dilattn_fwd, which takes its scratch from the library's memory pool, on
+calls in a row with different shapes, patterns and inputs (with and without
+an r = 1 pattern, so both ways of merging run on the shared array), so
+scratch read from the wrong place or left over from an earlier call would
+show up; and they check that a problem too large for the array is refused.
 
 This file is named to be collected last: a failure here stops a -x run only
 after every other test has run.
@@ -43,19 +44,20 @@ def _noalloc(q, k, v, out, lse, pats):
 CALLS = [
     (2, 2048, 8, PATS, 21),
     (1, 3000, 6, [(300, 1), (700, 3), (3000, 5)], 22),
+    (1, 1500, 4, [(500, 2), (1500, 3)], 23),  # no r = 1 pattern: separate merge pass
 ]
 
 
 @pytest.mark.parametrize("d", [64, 128])
-def test_noalloc_matches_workspace_forward_on_two_calls(d):
+def test_noalloc_matches_pooled_forward_on_consecutive_calls(d):
     calls = []
     for B, N, H, pats, seed in CALLS:
-        assert dilattn.fwd_workspace_size(B, N, H, d, pats) <= dilattn.NOALLOC_SCRATCH_BYTES
+        assert dilattn.fwd_scratch_size(B, N, H, d, pats) <= dilattn.NOALLOC_SCRATCH_BYTES
         q, k, v = to_device(make_inputs(B, N, H, d, seed, "bf16"))
         out = torch.empty_like(q)
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
         calls.append((q, k, v, out, lse, pats))
-    # two calls in a row on the shared scratch
+    # the calls in a row on the shared scratch
     for q, k, v, out, lse, pats in calls:
         _noalloc(q, k, v, out, lse, pats)
     torch.cuda.synchronize()
@@ -69,7 +71,7 @@ def test_noalloc_matches_workspace_forward_on_two_calls(d):
 
 def test_noalloc_refuses_problems_larger_than_its_scratch():
     wl = WORKLOADS["longnet_base_32k"]
-    need = dilattn.fwd_workspace_size(wl.B, wl.N, wl.H, wl.d, wl.patterns)
+    need = dilattn.fwd_scratch_size(wl.B, wl.N, wl.H, wl.d, wl.patterns)
     assert need > dilattn.NOALLOC_SCRATCH_BYTES
     w, r, n = dilattn._patterns(wl.patterns)
     base = 1 << 20  # aligned stand-in pointers: a refused call touches no memory

@@ -24,8 +24,9 @@ sampled through NVML every few milliseconds during the timed steps.
 
 The JSON detail adds the other workloads the metric is quoted on: the
 training step at B = 4, N = 32768 (forward + backward), the length sweep
-N = 8K .. 1M (forward + backward), the wide d = 128 forward, and the N = 8K
-step replayed back to back from a CUDA graph.
+N = 8K .. 1M (forward + backward), the wide d = 128 forward (bf16, and FP8
+with e4m3 q and k), and the N = 8K step replayed back to back from a CUDA
+graph.
 
 cpu_baseline: the float64 CPU oracle on the whole LongNet-base layer, one
 worker process per (batch, head) slice, one BLAS thread each, on the host's
@@ -491,6 +492,51 @@ def time_workload(dilattn, dev, name: str, flush_buf, peak: float, steps: int = 
     return ent
 
 
+def time_fp8(dilattn, dev, flush_buf, peak: float, name: str = WIDE, steps: int = 3,
+             warmup: int = 2):
+    """The FP8 forward (e4m3 q and k, bf16 v) of a d = 128 workload next to the bf16
+    forward of the same inputs. Peak: S runs at the FP8 rate (twice bf16, the
+    nominal ratio) and PV at the bf16 rate, half of the FLOPs each, so the
+    kernel's ceiling is 4/3 of the bf16 peak."""
+    import torch
+
+    wl = WORKLOADS[name]
+    B, N, H, d, pats = wl.B, wl.N, wl.H, wl.d, wl.patterns
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(0)
+    q, k, v = (torch.randn((B, N, H, d), generator=gen, device=dev, dtype=torch.float32)
+               .to(torch.bfloat16) for _ in range(3))
+    q8, k8 = [], []
+    scales = []
+    for x, dst in ((q, q8), (k, k8)):
+        sc = float(x.float().abs().max()) / 448.0
+        dst.append((x.float() / sc).to(torch.float8_e4m3fn))
+        scales.append(sc)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    t8, tb = [], []
+    for i in range(warmup + steps):
+        for fn, acc in ((lambda: dilattn.fwd_fp8(q8[0], k8[0], v, pats, scales[0], scales[1],
+                                                   wl.causal), t8),
+                        (lambda: dilattn.fwd(q, k, v, pats, wl.causal), tb)):
+            a, b = ev(), ev()
+            flush_buf.fill_(1)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= warmup:
+                acc.append(a.elapsed_time(b))
+    fw = flops.fwd_flops(B, N, H, d, pats, wl.causal)
+    m8, mb = statistics.median(t8), statistics.median(tb)
+    peak8 = peak * 4.0 / 3.0
+    del q, k, v, q8, k8
+    torch.cuda.empty_cache()
+    return {"workload": name, "fp8_fwd_ms": m8, "fp8_fwd_tflops": fw / m8 / 1e9,
+            "fp8_peak_tflops": peak8, "fp8_frac_of_peak": fw / m8 / 1e9 / peak8,
+            "peak_note": "S at the FP8 rate (2x bf16, nominal ratio), PV at bf16: 4/3 of bf16",
+            "bf16_fwd_ms": mb, "bf16_fwd_tflops": fw / mb / 1e9, "speedup": mb / m8}
+
+
 def graph_step(dilattn, dev, name: str = "sweep_8192", replays: int = 50):
     """The N = 8192 step captured once in a CUDA graph and replayed back to back,
     without L2 flushes: the launch-bound regime. The training step
@@ -771,6 +817,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         det["length_sweep"] = [time_workload(dilattn, dev, n, flush_buf, peak) for n in SWEEP]
         det["wide_d128"] = time_workload(dilattn, dev, WIDE, flush_buf, peak)
         det["graph_8k"] = graph_step(dilattn, dev)
+        det["fp8_wide_d128"] = time_fp8(dilattn, dev, flush_buf, peak)
         if dilattn.device_error() != 0:
             raise RuntimeError("a kernel reported a device-side error in the detail runs")
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -116,6 +116,21 @@ int dilattn_fwd_train(const void* q, const void* k, const void* v, void* out, vo
                       int causal, cudaStream_t stream);
 
 /*
+ * Forward with e4m3 q and k (FP8 variant; the gptget.net summary, "方法详解"
+ * bullet 8, names quantisation among the engineering measures). q8, k8:
+ * [B][N][H][d] e4m3 bytes holding q / q_scale and k / k_scale (per-tensor
+ * scales > 0); v bf16. S = Q K^T runs on the FP8 tensor cores (kind::f8f6f4,
+ * twice the bf16 rate) and is exact for the quantised inputs; P, V and the
+ * PV product stay bf16, because an e4m3 P (3 mantissa bits) would cost far
+ * more than the 2e-2 bound. d = 128 only: at d = 64 the forward is bound by
+ * the exponentials, not by S. Results as dilattn_fwd for the inputs
+ * q8 * q_scale, k8 * k_scale, v; scratch as in dilattn_fwd.
+ */
+int dilattn_fwd_fp8(const void* q8, const void* k8, const void* v, void* out, float* lse,
+                    int B, int N, int H, int d, const int* w, const int* r, int npat, int causal,
+                    float q_scale, float k_scale, cudaStream_t stream);
+
+/*
  * Forward for callers that cannot allocate device memory: same arguments and
  * results as dilattn_fwd. Some callers have no way to get scratch memory: a
  * plugin handed only its input and output pointers by a host framework, a

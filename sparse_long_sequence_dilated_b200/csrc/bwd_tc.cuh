@@ -28,13 +28,13 @@
 // SdP_1(i+1) run. An S / dP half is overwritten only by MMAs issued after
 // the MMAs that read its P / dS, and tcgen05 MMAs of one thread execute in
 // issue order.
-// P and dS enter the products as bf16. On the first query tile of a segment
-// (rows with few keys, where single probabilities approach 1) P enters dV and
-// dS enters dK as two bf16 halves, hi + lo, so those products are fp32-grade:
-// the gradients' own bf16 rounding (half an ulp is 0.0156 at |g| in [4, 8))
-// leaves little room for a 2^-9 rounding of a large P under a 2e-2 bound.
-// Elsewhere a row spreads its weight over at least 129 keys, and the
-// rounding of P and dS averages out far inside the bound.
+// P enters dV as bf16 and dS enters dK and dQ as fp16 (dS reaches tens, where
+// bf16's 8 significant bits cost up to 2e-2 in dq and dk; q and k are
+// converted exactly to fp16 for those products, and for S). On the first
+// query tile of a segment (rows with few keys, where single probabilities
+// approach 1) P enters dV and dS enters dK as two halves, hi + lo, so those
+// products are fp32-grade. Elsewhere a row spreads its weight over at least
+// 129 keys, and the rounding of P averages out far inside the bound.
 // dQ goes through a double-buffered TMEM accumulator; after each pair every
 // row warp stages its 32 x 32 block in a private shared-memory slab and adds
 // it to the fp32 accumulator with a TMA reduce-add. dK, dV are added the same
@@ -153,16 +153,15 @@ __device__ __forceinline__ void bwd_chunk(const uint32_t (&sv)[32], const uint32
       const uint64_t ds2 = f2_mul(
           p2, f2_sub(f2_pack(__uint_as_float(dv[e]), __uint_as_float(dv[e + 1])), dd2[h2]));
       const uint32_t hi = pack_bf16_rn(p0, p1);
-      const uint32_t dhi = pack_bf16_rn(f2_lo(ds2), f2_hi(ds2));
+      const uint32_t dhi = pack_f16_rn(f2_lo(ds2), f2_hi(ds2));
       pk[o] = hi;
       dk[o] = dhi;
       if (SPLIT) {
         const uint64_t lo2 =
             f2_sub(p2, f2_pack(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u)));
         plo[o] = pack_bf16_rn(f2_lo(lo2), f2_hi(lo2));
-        const uint64_t dlo2 =
-            f2_sub(ds2, f2_pack(__uint_as_float(dhi << 16), __uint_as_float(dhi & 0xffff0000u)));
-        dkl[o] = pack_bf16_rn(f2_lo(dlo2), f2_hi(dlo2));
+        const uint64_t dlo2 = f2_sub(ds2, f2_pack(f16_lo(dhi), f16_hi(dhi)));
+        dkl[o] = pack_f16_rn(f2_lo(dlo2), f2_hi(dlo2));
       }
     }
   }
@@ -389,9 +388,12 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
     // ------------------------------------------------------------ MMA issuer
     // The whole warp runs the loop; one elected lane issues each MMA group.
     {
-      constexpr uint32_t kIdSh = idesc_bf16(BM, 64, 0, 0);  // K x Q_h^T, V x dO_h^T
-      constexpr uint32_t kIdKV = idesc_bf16(BM, D, 0, 1);   // P^T / dS^T (TMEM) x dO / Q
-      constexpr uint32_t kIdQ = idesc_bf16(BM, D, 1, 1);    // dS (MN-major SMEM) x K
+      // Q, K (and dS) are fp16, V, dO (and P) bf16: every product has one type
+      constexpr uint32_t kIdS = idesc_f16(BM, 64, 0, 0);    // K x Q_h^T
+      constexpr uint32_t kIdDP = idesc_bf16(BM, 64, 0, 0);  // V x dO_h^T
+      constexpr uint32_t kIdV = idesc_bf16(BM, D, 0, 1);    // P^T (TMEM) x dO
+      constexpr uint32_t kIdK = idesc_f16(BM, D, 0, 1);     // dS^T (TMEM) x Q
+      constexpr uint32_t kIdQ = idesc_f16(BM, D, 1, 1);     // dS (MN-major SMEM) x K
       // Descriptors are built once; each MMA only adds a byte offset to the
       // low word, which keeps the issuing thread's work per MMA small (it
       // shares its scheduler with two row warps).
@@ -405,10 +407,10 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         const uint32_t ts = tmem + C::TM_S + h * 64, tp = tmem + C::TM_DP + h * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(ts, dKk.at(kk * 32), dQk.at(qo + kk * 32), kIdSh, kk > 0 ? 1u : 0u);
+          mma_ss(ts, dKk.at(kk * 32), dQk.at(qo + kk * 32), kIdS, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tp, dVk.at(kk * 32), dDOk.at(qo + kk * 32), kIdSh, kk > 0 ? 1u : 0u);
+          mma_ss(tp, dVk.at(kk * 32), dDOk.at(qo + kk * 32), kIdDP, kk > 0 ? 1u : 0u);
         mma_commit(b_sdp(h));
       };
       // dV += P^T_h dO_h, dK += dS^T_h Q_h (each hi + lo when `split`); `first`
@@ -420,16 +422,16 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           const int kk = 4 * h + kq;  // 16 queries
           const uint64_t bdo = dDOm.at(qo + kk * 2048);
           const uint32_t a = tmem + C::TM_S + (kk >> 1) * 32 + (kk & 1) * 8;
-          mma_ts(tmem + C::TM_DV, a, bdo, kIdKV, (first && kq == 0) ? 0u : 1u);
-          if (split) mma_ts(tmem + C::TM_DV, a + 16, bdo, kIdKV, 1u);
+          mma_ts(tmem + C::TM_DV, a, bdo, kIdV, (first && kq == 0) ? 0u : 1u);
+          if (split) mma_ts(tmem + C::TM_DV, a + 16, bdo, kIdV, 1u);
         }
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
           const int kk = 4 * h + kq;
           const uint64_t bq = dQm.at(qo + kk * 2048);
           const uint32_t a = tmem + C::TM_DP + (kk >> 1) * 32 + (kk & 1) * 8;
-          mma_ts(tmem + C::TM_DK, a, bq, kIdKV, (first && kq == 0) ? 0u : 1u);
-          if (split) mma_ts(tmem + C::TM_DK, a + 16, bq, kIdKV, 1u);
+          mma_ts(tmem + C::TM_DK, a, bq, kIdK, (first && kq == 0) ? 0u : 1u);
+          if (split) mma_ts(tmem + C::TM_DK, a + 16, bq, kIdK, 1u);
         }
       };
       // dQ = dS K into TMEM buffer g & 1 (dS from shared memory)
@@ -708,6 +710,11 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
 // significant bits), and zeroed fp32 gradients; one warp per row.
 struct PrepParams {
   int B, N, H;
+  const __nv_bfloat16* q;
+  const __nv_bfloat16* k;
+  __half* q16;  // fp16 copies of q and k for the products with dS
+  __half* k16;
+  ErrCtx err;   // a value outside the fp16 range records kErrF16Range
   const __nv_bfloat16* out;
   const __nv_bfloat16* out_res;  // bf16(O - out) from the training forward
   const __nv_bfloat16* dout;
@@ -730,6 +737,15 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(PrepParams p) {
   float acc = o0 * __low2float(d) + o1 * __high2float(d);
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  {
+    const __nv_bfloat162 a = reinterpret_cast<const __nv_bfloat162*>(p.q + row * 64)[lane];
+    const __nv_bfloat162 b = reinterpret_cast<const __nv_bfloat162*>(p.k + row * 64)[lane];
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    if (fmaxf(fmaxf(fabsf(fa.x), fabsf(fa.y)), fmaxf(fabsf(fb.x), fabsf(fb.y))) > 65504.f)
+      p.err.raise(kErrF16Range);
+    reinterpret_cast<__half2*>(p.q16 + row * 64)[lane] = __float22half2_rn(fa);
+    reinterpret_cast<__half2*>(p.k16 + row * 64)[lane] = __float22half2_rn(fb);
+  }
   const float2 z = make_float2(0.f, 0.f);
   reinterpret_cast<float2*>(p.dq + row * 64)[lane] = z;
   reinterpret_cast<float2*>(p.dk + row * 64)[lane] = z;

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace dil {
@@ -14,11 +15,13 @@ constexpr int BM = 128;   // query rows per tile (MMA M)
 constexpr int BN = 128;   // key rows per tile (MMA N of S = Q K^T)
 
 // Error codes a kernel may leave in the device error word.
-enum DevErr : int { kErrNone = 0, kErrWaitTimeout = 1, kErrBadTile = 2 };
+enum DevErr : int { kErrNone = 0, kErrWaitTimeout = 1, kErrBadTile = 2, kErrF16Range = 3 };
 
 // Geometry of one (w, r) pattern for a given N (host-computed, read on device).
 struct PatternGeom {
   int w, r;
+  uint32_t w_mul, r_mul;  // reciprocal multipliers of w and r (divisor_magic)
+  int w_sh, r_sh;
   int nseg;            // ceil(N / w): number of segments
   int nmax;            // ceil(min(w, N) / r): row capacity of one segment
   int ntiles;          // ceil(nmax / BM)
@@ -26,6 +29,22 @@ struct PatternGeom {
   int nmod;            // N mod r: phases below it have one row more in the strided view
   long long part_base; // first row of this pattern in the partial-result buffer
 };
+
+// Division of n < 2^31 by a divisor 1 <= d < 2^31 fixed for the launch, as a
+// multiply and a shift (the round-up method of Granlund and Montgomery,
+// "Division by invariant integers using multiplication", 1994): with
+// l = ceil(log2 d) and m = ceil(2^(31 + l) / d) < 2^32, floor(n / d) =
+// floor(n m / 2^(31 + l)), because n m / 2^(31 + l) exceeds n / d by less
+// than 2^-l <= 1 / d, too little to reach the next integer.
+inline void divisor_magic(uint32_t d, uint32_t& mul, int& sh) {
+  int l = 0;
+  while ((1ull << l) < d) ++l;
+  sh = 31 + l;
+  mul = (uint32_t)(((1ull << sh) + d - 1) / d);
+}
+__host__ __device__ __forceinline__ uint32_t udiv(uint32_t n, uint32_t mul, int sh) {
+  return (uint32_t)(((uint64_t)n * mul) >> sh);
+}
 
 // Segment s of pattern g for head h: first position, kept count, offset.
 // Segment s spans [s*w, min((s+1)*w, N)) and keeps s*w + (h mod r) + k*r.
@@ -150,6 +169,11 @@ __device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Bring the 128-byte line holding p into L2.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -187,6 +211,17 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc]^T, kind::f8f6f4 (8-bit in, fp32 accumulate).
+__device__ __forceinline__ void mma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16.
 __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                        uint32_t idesc, uint32_t accumulate) {
@@ -196,6 +231,15 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// Copy a 128-row x 32-byte shared-memory matrix (described like an MMA
+// operand) into TMEM: row i to lane i, its 32 bytes to 8 consecutive columns.
+// A tcgen05.mma that the same thread issues afterwards sees the copy (the two
+// execute in issue order).
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(s_desc)
+               : "memory");
 }
 
 // Arrive on an mbarrier once every tcgen05 operation this thread issued so far completes.
@@ -268,6 +312,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) |
          ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// The same for fp16 A and B (format code 0).
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N, int a_mn_major, int b_mn_major) {
+  return (1u << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -532,6 +582,15 @@ __device__ __forceinline__ uint32_t pack_bf16_rn(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
   return d;
 }
+// f16x2 of (lo, hi), round to nearest even, one instruction.
+__device__ __forceinline__ uint32_t pack_f16_rn(float lo, float hi) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+// The two halves of an f16x2 word as floats (exact).
+__device__ __forceinline__ float f16_lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu))); }
+__device__ __forceinline__ float f16_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
 // ex2_poly on a pair with packed arithmetic (same steps, same constants):
 // clamp at -125, j = rint(x) via x + 1.5 * 2^23, f = x - j, Horner for 2^f,
 // then j added to the exponent field. (t_bits << 23) equals j << 23 modulo

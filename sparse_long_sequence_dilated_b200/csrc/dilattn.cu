@@ -110,6 +110,10 @@ int device_state(DeviceState** out) {
       e = cudaFuncSetAttribute(fwd_tile_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                FwdCfg<128>::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+      e = cudaFuncSetAttribute(fwd_tile_kernel<128, true>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               FwdCfg<128, true>::SMEM_BYTES);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
       e = cudaFuncSetAttribute(bwd_tile_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                BwdCfg::SMEM_BYTES);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
@@ -196,7 +200,7 @@ int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CU
   }
   int rc = get_encoder();
   if (rc != DILATTN_OK) return rc;
-  const int esz = f32 ? 4 : 2;
+  const int esz = f32 == 1 ? 4 : f32 == 3 ? 1 : 2;  // f32: 0 bf16, 1 fp32, 2 fp16, 3 e4m3
   const long long rowb = (long long)H * d * esz;
   cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)(tail ? nmod : r),
                         (cuuint64_t)(tail ? nfloor + 1 : nfloor), (cuuint64_t)B};
@@ -205,8 +209,11 @@ int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CU
   cuuint32_t box[5] = {(cuuint32_t)(128 / esz), 1, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap m;
-  CUresult cr = g_encode(&m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                         5, const_cast<void*>(ptr), dims,
+  const CUtensorMapDataType dt = f32 == 1 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : f32 == 2 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                 : f32 == 3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                            : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  CUresult cr = g_encode(&m, dt, 5, const_cast<void*>(ptr), dims,
                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -327,6 +334,8 @@ long long make_geoms(int B, int N, int H, const int* w, const int* r, int npat,
     PatternGeom& g = geo[i];
     g.w = w[i];
     g.r = r[i];
+    divisor_magic((uint32_t)w[i], g.w_mul, g.w_sh);
+    divisor_magic((uint32_t)r[i], g.r_mul, g.r_sh);
     g.nseg = (int)(((long long)N + w[i] - 1) / w[i]);
     const long long span = std::min<long long>(w[i], N);
     g.nmax = (int)((span + r[i] - 1) / r[i]);
@@ -397,7 +406,7 @@ FwdScratch fwd_scratch_layout(long long rows, int d) {
   FwdScratch f;
   f.o_bytes = align256((size_t)rows * d * 4);
   f.lse_bytes = align256((size_t)rows * 4);
-  f.flag_bytes = align256((size_t)(rows / BM + 1) * 4 + 4);  // flags, then the counter
+  f.flag_bytes = align256((size_t)(rows / BM + 1) * 4 + 8);  // flags, the ticket and done counters
   return f;
 }
 
@@ -407,10 +416,11 @@ size_t fwd_scratch_bytes(int B, int N, int H, int d, const int* w, const int* r,
   return fwd_scratch_layout(rows, d).total();
 }
 
-template <int D>
+template <int D, bool QK8 = false>
 int launch_fwd(const void* q, const void* k, const void* v, void* out, void* out_res, float* lse,
                int B, int N, int H, const int* w, const int* r, int npat, int causal, void* ws,
-               DeviceState* st, cudaStream_t stream, const SeqParPlan* sp = nullptr) {
+               DeviceState* st, cudaStream_t stream, const SeqParPlan* sp = nullptr,
+               float qk_scale = 1.f) {
   static_assert(sizeof(FwdParams) < 32000, "kernel parameter block too large");
   FwdParams p;
   memset(&p, 0, sizeof(p));
@@ -419,7 +429,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, void* out
   p.N = N;
   p.H = H;
   p.causal = causal;
-  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D) * (double)qk_scale);
   p.merger = pick_merger(w, r, npat);
   const long long rows = make_geoms(B, N, H, w, r, npat, p.pat, p.merger);
   const FwdScratch lay = fwd_scratch_layout(rows, D);
@@ -428,17 +438,19 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, void* out
   p.part_lse = reinterpret_cast<float*>(wsb + lay.o_bytes);
   p.flags = reinterpret_cast<int*>(wsb + lay.o_bytes + lay.lse_bytes);
   p.counter = p.flags + rows / BM + 1;
+  p.done = p.counter + 1;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.out_res = reinterpret_cast<__nv_bfloat16*>(out_res);
   p.lse = lse;
   p.err = ErrCtx{st->err_word, next_tag()};
   for (int i = 0; i < npat; ++i) {
     const void* src[3] = {q, k, v};
+    const int dtype[3] = {QK8 ? 3 : 0, QK8 ? 3 : 0, 0};
     CUtensorMap* dst[3] = {&p.tmq[i], &p.tmk[i], &p.tmv[i]};
     CUtensorMap* dst_t[3] = {&p.tmq_t[i], &p.tmk_t[i], &p.tmv_t[i]};
     for (int j = 0; j < 3; ++j) {
-      int rc = strided_map(src[j], B, N, H, D, r[i], 0, dst[j]);
-      if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j]);
+      int rc = strided_map(src[j], B, N, H, D, r[i], 0, dst[j], dtype[j]);
+      if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j], dtype[j]);
       if (rc != DILATTN_OK) return rc;
     }
     if (sp != nullptr && sp->kv_rows[i] > 0) {
@@ -462,7 +474,8 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, void* out
   int rc = trace_mark(g_trace_begin, stream);
   if (rc != DILATTN_OK) return rc;
   if (units > 0)
-    fwd_tile_kernel<D><<<(unsigned)units, FwdCfg<D>::THREADS, FwdCfg<D>::SMEM_BYTES, stream>>>(p);
+    fwd_tile_kernel<D, QK8>
+        <<<(unsigned)units, FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::SMEM_BYTES, stream>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "fwd_tile_kernel launch");
   rc = trace_mark(g_trace_end, stream);
@@ -508,20 +521,25 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   p.tau = (float)(1.0 / std::sqrt((double)D));
   p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
   make_geoms(B, N, H, w, r, npat, p.pat);
-  // workspace: D [B][H][N] fp32, then 256 bytes for the key-tile kernel's unit counter
+  // workspace: D [B][H][N] fp32, 256 bytes for the key-tile kernel's unit
+  // counter, then fp16 copies of q and k
   char* wsb = reinterpret_cast<char*>(ws);
   float* drow = reinterpret_cast<float*>(wsb);
   p.drow = drow;
   p.lse = lse;
-  p.counter = reinterpret_cast<int*>(wsb + align256((size_t)B * H * N * 4));
+  const size_t dbytes = align256((size_t)B * H * N * 4);
+  p.counter = reinterpret_cast<int*>(wsb + dbytes);
+  __half* q16 = reinterpret_cast<__half*>(wsb + dbytes + 256);
+  __half* k16 = reinterpret_cast<__half*>(wsb + dbytes + 256 + align256((size_t)B * N * H * D * 2));
   p.err = ErrCtx{st->err_word, next_tag()};
   for (int i = 0; i < npat; ++i) {
-    const void* src[4] = {q, k, v, dout};
+    const void* src[4] = {q16, k16, v, dout};
+    const int dtype[4] = {2, 2, 0, 0};
     CUtensorMap* dst[4] = {&p.tmq[i], &p.tmk[i], &p.tmv[i], &p.tmdo[i]};
     CUtensorMap* dst_t[4] = {&p.tmq_t[i], &p.tmk_t[i], &p.tmv_t[i], &p.tmdo_t[i]};
     for (int j = 0; j < 4; ++j) {
-      int rc = strided_map(src[j], B, N, H, D, r[i], 0, dst[j]);
-      if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j]);
+      int rc = strided_map(src[j], B, N, H, D, r[i], 0, dst[j], dtype[j]);
+      if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j], dtype[j]);
       if (rc != DILATTN_OK) return rc;
     }
     // reduce-add targets: one row warp adds a 32-row x 32-column block
@@ -556,6 +574,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
   pp.B = B;
   pp.N = N;
   pp.H = H;
+  pp.q = reinterpret_cast<const __nv_bfloat16*>(q);
+  pp.k = reinterpret_cast<const __nv_bfloat16*>(k);
+  pp.q16 = q16;
+  pp.k16 = k16;
+  pp.err = p.err;
   pp.out = reinterpret_cast<const __nv_bfloat16*>(out);
   pp.out_res = reinterpret_cast<const __nv_bfloat16*>(out_res);
   pp.dout = reinterpret_cast<const __nv_bfloat16*>(dout);
@@ -666,6 +689,42 @@ int dilattn_fwd(const void* q, const void* k, const void* v, void* out, float* l
   return fwd_pooled(q, k, v, out, nullptr, lse, B, N, H, d, w, r, npat, causal, stream);
 }
 
+int dilattn_fwd_fp8(const void* q8, const void* k8, const void* v, void* out, float* lse, int B,
+                    int N, int H, int d, const int* w, const int* r, int npat, int causal,
+                    float q_scale, float k_scale, cudaStream_t stream) {
+  int rc = check_shape(B, N, H, d, w, r, npat, causal);
+  if (rc != DILATTN_OK) return rc;
+  if (d != 128) {
+    snprintf(g_last_error, sizeof(g_last_error), "the fp8 forward is built for d = 128");
+    return DILATTN_ERR_UNSUPPORTED;
+  }
+  if (!(q_scale > 0.f) || !(k_scale > 0.f) || !std::isfinite(q_scale) || !std::isfinite(k_scale))
+    return DILATTN_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(out) ||
+      (lse != nullptr && !aligned16(lse)))
+    return DILATTN_ERR_INVALID_ARG;
+  const size_t t8 = (size_t)B * N * H * d, tb = 2 * t8, lb = (size_t)B * H * N * 4;
+  if (overlaps(out, tb, q8, t8) || overlaps(out, tb, k8, t8) || overlaps(out, tb, v, tb) ||
+      (lse != nullptr && (overlaps(lse, lb, q8, t8) || overlaps(lse, lb, k8, t8) ||
+                          overlaps(lse, lb, v, tb) || overlaps(lse, lb, out, tb))))
+    return DILATTN_ERR_INVALID_ARG;
+  DeviceState* st = nullptr;
+  rc = device_state(&st);
+  if (rc != DILATTN_OK) return rc;
+  cudaMemPool_t pool = nullptr;
+  rc = scratch_pool(st, &pool);
+  if (rc != DILATTN_OK) return rc;
+  const size_t need = fwd_scratch_bytes(B, N, H, d, w, r, npat);
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocFromPoolAsync(&scratch, need, pool, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMallocFromPoolAsync (forward scratch)");
+  rc = launch_fwd<128, true>(q8, k8, v, out, nullptr, lse, B, N, H, w, r, npat, causal, scratch,
+                             st, stream, nullptr, q_scale * k_scale);
+  e = cudaFreeAsync(scratch, stream);
+  if (rc == DILATTN_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync (forward scratch)");
+  return rc;
+}
+
 int dilattn_fwd_train(const void* q, const void* k, const void* v, void* out, void* out_res,
                       float* lse, int B, int N, int H, int d, const int* w, const int* r, int npat,
                       int causal, cudaStream_t stream) {
@@ -675,7 +734,8 @@ int dilattn_fwd_train(const void* q, const void* k, const void* v, void* out, vo
 
 size_t dilattn_bwd_workspace_size(int B, int N, int H, int d) {
   if (B < 1 || N < 1 || H < 1 || d < 1 || (double)B * N * H * d >= 1099511627776.0) return 0;
-  return align256((size_t)B * H * N * 4) + 256;  // D, then the unit counter
+  // D, the unit counter, then fp16 copies of q and k
+  return align256((size_t)B * H * N * 4) + 256 + 2 * align256((size_t)B * N * H * d * 2);
 }
 
 int dilattn_bwd(const void* q, const void* k, const void* v, const void* out,

@@ -56,6 +56,7 @@ struct FwdParams {
   long long units_p; // units of `sched`
   int merger;        // index of the merging pattern, or -1 (a separate merge kernel combines)
   int* counter;      // ticket counter: the order in which CTAs take units (zero at launch)
+  int* done;         // partial-storing units finished (zero at launch)
   int* flags;        // one per 128-row block of partial rows: nonzero once the block is stored
   float* part_o;     // [rows][D] normalised per-pattern outputs
   float* part_lse;   // [rows] natural-log lse of each pattern's partial
@@ -106,31 +107,38 @@ __device__ __forceinline__ bool wait_flag(const int* f, volatile int* abort, con
 }
 
 // Partial row of position n in pattern g for head h of slice bh (= b * H + h),
-// if g keeps n: segment n / w, kept iff (n - start - h mod r) is a
-// non-negative multiple of r.
-__device__ __forceinline__ bool partial_row(const PatternGeom& g, int n, int h, int bh,
-                                            long long& pr) {
-  const uint32_t seg = (uint32_t)n / (uint32_t)g.w;
-  const int rel = n - (int)(seg * (uint32_t)g.w) - h % g.r;
-  if (rel < 0) return false;
-  const uint32_t v = (uint32_t)rel / (uint32_t)g.r;
-  if ((int)(v * (uint32_t)g.r) != rel) return false;
-  pr = g.part_base + ((long long)bh * g.nseg + seg) * g.pstride + v;
-  return true;
+// or -1 when g does not keep n: segment n / w, kept iff rel = n - start -
+// (h mod r) is a non-negative multiple of r, row rel / r of the segment's
+// block. off = h mod r. The quotients use the patterns' reciprocal
+// multipliers (udiv), so the lookup costs a few instructions per pattern.
+__device__ __forceinline__ int partial_row(const PatternGeom& g, int n, int off, int bh) {
+  const uint32_t seg = udiv((uint32_t)n, g.w_mul, g.w_sh);
+  const int rel = n - (int)(seg * (uint32_t)g.w) - off;
+  if (rel < 0) return -1;
+  const uint32_t v = udiv((uint32_t)rel, g.r_mul, g.r_sh);
+  if ((int)(v * (uint32_t)g.r) != rel) return -1;
+  return (int)(g.part_base + ((long long)bh * g.nseg + seg) * g.pstride + v);
 }
 
-template <int D>
+// QK8: q and k are e4m3 (one byte per element; the fp8 variant, d = 128):
+// their 128-row tiles are single 128-byte chunks and S = Q K^T runs as
+// kind::f8f6f4; V, P and O stay as in the bf16 kernel.
+template <int D, bool QK8 = false>
 struct FwdCfg {
-  static constexpr int KCH = D / 64;                 // 128-byte column chunks per row
+  static constexpr int KCH = D / 64;                 // 128-byte chunks of a bf16 row (V)
+  static constexpr int KCH_QK = QK8 ? D / 128 : D / 64;  // 128-byte chunks of a Q or K row
   static constexpr int KST = 3;                      // K ring depth (a stage frees after its S MMA)
   static constexpr int VST = 2;                      // V ring depth (a stage frees after its PV MMA)
-  static constexpr int CHUNK_BYTES = BM * 128;       // 128 rows x 64 bf16
-  static constexpr int Q_BYTES = KCH * CHUNK_BYTES;
-  static constexpr int KV_BYTES = KCH * CHUNK_BYTES;
+  static constexpr int CHUNK_BYTES = BM * 128;       // 128 rows x 128 bytes
+  static constexpr int Q_BYTES = KCH_QK * CHUNK_BYTES;
+  static constexpr int K_BYTES = KCH_QK * CHUNK_BYTES;
+  static constexpr int V_BYTES = KCH * CHUNK_BYTES;
+  static constexpr int QK_COLS = QK8 ? 128 : 64;     // elements of a 128-byte chunk of Q or K
+  static constexpr int S_KSTEPS = QK8 ? D / 32 : D / 16;  // MMA K steps of S (32 bytes each)
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + KST * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_V + VST * KV_BYTES;
+  static constexpr int OFF_V = OFF_K + KST * K_BYTES;
+  static constexpr int OFF_BAR = OFF_V + VST * V_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
   static constexpr int TM_S = 0, TM_P = 128, TM_O = 192;
   static constexpr int TMEM_COLS = (TM_O + D <= 256) ? 256 : 512;
@@ -147,41 +155,91 @@ struct FwdCfg {
 // One thread per row; out is written once, in bf16 (and, for training, the
 // bf16 rounding residual of out, so that the backward's D = dO . O keeps
 // fp32-grade accuracy).
+
+struct MergeWeights {
+  float M;                // the largest of the row's log2 denominators
+  float Z;                // sum of the weights, own included
+  float w_own;            // weight of the tile's own O accumulator (already / l)
+  float w[kMaxPat];       // weight of pattern i's partial, 0 if it does not keep the row
+  int pr[kMaxPat];        // pattern i's partial row of this row, -1 if none
+  bool ok;
+};
+
+// Part 1 runs once the tile's last P is stored, while its last PV product is
+// still in flight: which partial rows the row has (checking that they are
+// stored), their lse_i turned into weights, and an L2 prefetch of their O_i
+// rows so that part 2 finds them on chip.
+template <int D>
+__device__ __forceinline__ MergeWeights merge_weights(const FwdParams& p, const TileUnit& wu,
+                                                      const SegInfo& si, int vq, float m_run,
+                                                      float l_run, bool all_done,
+                                                      volatile int* abort_flag) {
+  constexpr float kLog2e = 1.4426950408889634f;
+  MergeWeights mw;
+  mw.ok = true;
+  const int n = (int)si.start + vq;  // r = 1, offset 0
+  const int bh = wu.b * p.H + wu.h;
+  const bool valid = vq < si.n;
+  const float own = m_run + __log2f(l_run);
+#pragma unroll
+  for (int i = 0; i < kMaxPat; ++i) {
+    mw.pr[i] = -1;
+    if (i >= p.npat || i == p.merger || !valid) continue;
+    const PatternGeom& gi = p.pat[i];
+    const int off = wu.h - (int)(udiv((uint32_t)wu.h, gi.r_mul, gi.r_sh) * (uint32_t)gi.r);
+    mw.pr[i] = partial_row(gi, n, off, bh);
+  }
+  // every row's flag first (skipped once every partial-storing unit is done),
+  // then the lse loads, independent of one another
+  if (!all_done) {
+#pragma unroll
+    for (int i = 0; i < kMaxPat; ++i)
+      if (mw.pr[i] >= 0 && !wait_flag(p.flags + (mw.pr[i] >> 7), abort_flag, p.err)) mw.ok = false;
+  }
+  float L[kMaxPat];
+  mw.M = own;
+#pragma unroll
+  for (int i = 0; i < kMaxPat; ++i) {
+    L[i] = -INFINITY;
+    if (mw.pr[i] < 0) continue;
+    L[i] = __ldcg(p.part_lse + mw.pr[i]) * kLog2e;
+    const char* row = reinterpret_cast<const char*>(p.part_o + (long long)mw.pr[i] * D);
+#pragma unroll
+    for (int c = 0; c < D * 4; c += 128) prefetch_l2(row + c);
+    mw.M = fmaxf(mw.M, L[i]);
+  }
+  mw.Z = ex2(own - mw.M);
+  mw.w_own = mw.Z / l_run;
+#pragma unroll
+  for (int i = 0; i < kMaxPat; ++i) {
+    mw.w[i] = L[i] == -INFINITY ? 0.f : ex2(L[i] - mw.M);
+    mw.Z += mw.w[i];
+  }
+  return mw;
+}
+
+// Part 2, once the last PV is complete: O from TMEM, the partials' rows, the
+// normalised result to out (and out_res), lse.
 template <int D>
 __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const TileUnit& wu,
                                                const SegInfo& si, int vq, uint32_t tl_o,
-                                               float m_run, float l_run,
-                                               volatile int* abort_flag) {
-  constexpr float kLog2e = 1.4426950408889634f;
+                                               const MergeWeights& mw) {
   float acc[D];
 #pragma unroll
   for (int c4 = 0; c4 < D / 32; ++c4) {
     uint32_t r[32];
     tmem_ld32_sync(tl_o + c4 * 32, r);  // warp-collective: every lane loads
 #pragma unroll
-    for (int c = 0; c < 32; ++c) acc[c4 * 32 + c] = __uint_as_float(r[c]);
+    for (int c = 0; c < 32; ++c) acc[c4 * 32 + c] = __uint_as_float(r[c]) * mw.w_own;
   }
-  if (vq >= si.n) return;
-  const int n = (int)si.start + vq;  // r = 1, offset 0
+  if (vq >= si.n || !mw.ok) return;
+  const int n = (int)si.start + vq;
   const int bh = wu.b * p.H + wu.h;
-  const float own = m_run + __log2f(l_run);
-  float M = own;
-  for (int i = 0; i < p.npat; ++i) {
-    long long pr;
-    if (i == p.merger || !partial_row(p.pat[i], n, wu.h, bh, pr)) continue;
-    if (!wait_flag(p.flags + (pr >> 7), abort_flag, p.err)) return;
-    M = fmaxf(M, __ldcg(p.part_lse + pr) * kLog2e);
-  }
-  float Z = ex2(own - M);
-  const float w_own = Z / l_run;
 #pragma unroll
-  for (int c = 0; c < D; ++c) acc[c] *= w_own;
-  for (int i = 0; i < p.npat; ++i) {
-    long long pr;
-    if (i == p.merger || !partial_row(p.pat[i], n, wu.h, bh, pr)) continue;
-    const float wi = ex2(__ldcg(p.part_lse + pr) * kLog2e - M);
-    Z += wi;
-    const float4* src = reinterpret_cast<const float4*>(p.part_o + pr * D);
+  for (int i = 0; i < kMaxPat; ++i) {
+    if (mw.pr[i] < 0 || mw.w[i] == 0.f) continue;
+    const float wi = mw.w[i];
+    const float4* src = reinterpret_cast<const float4*>(p.part_o + (long long)mw.pr[i] * D);
 #pragma unroll
     for (int e = 0; e < D / 4; ++e) {
       const float4 x = __ldcg(src + e);
@@ -191,7 +249,7 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const TileUni
       acc[4 * e + 3] = fmaf(wi, x.w, acc[4 * e + 3]);
     }
   }
-  const float inv = 1.f / Z;
+  const float inv = 1.f / mw.Z;
   const long long o0 = (((long long)wu.b * p.N + n) * p.H + wu.h) * D;
   uint4* dst = reinterpret_cast<uint4*>(p.out + o0);
   uint4* rdst = p.out_res != nullptr ? reinterpret_cast<uint4*>(p.out_res + o0) : nullptr;
@@ -207,13 +265,14 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const TileUni
     dst[e] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     if (rdst != nullptr) rdst[e] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
-  if (p.lse != nullptr) p.lse[(long long)bh * p.N + n] = (M + __log2f(Z)) * 0.69314718055994531f;
+  if (p.lse != nullptr)
+    p.lse[(long long)bh * p.N + n] = (mw.M + __log2f(mw.Z)) * 0.69314718055994531f;
 }
 
-template <int D>
-__global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
+template <int D, bool QK8 = false>
+__global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_BLOCKS)
     fwd_tile_kernel(const __grid_constant__ FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, QK8>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t base = (raw_s + 1023u) & ~1023u;
@@ -231,7 +290,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       : decode_unit(p.sched_m, p.pat, p.B, p.H, ticket - p.units_p);
   const PatternGeom g = p.pat[wu.pat];
   const SegInfo si = seg_info(g, p.N, wu.h, wu.seg);
-  if (wu.t * BM >= si.n) return;  // tile past the segment's kept rows (uniform exit)
+  if (wu.t * BM >= si.n) {  // tile past the segment's kept rows (uniform exit)
+    if (threadIdx.x == 0 && ticket < p.units_p) atomicAdd(p.done, 1);
+    return;
+  }
+  const bool merging = wu.pat == p.merger;
   const bool gathered = p.kv_rows[wu.pat] > 0;
   const int kv_n = gathered ? p.kv_rows[wu.pat] : si.n;  // key rows of the segment
   const int tq = wu.t + p.toff[wu.pat];                   // the query tile among the key tiles
@@ -315,17 +378,17 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       int ph, m;
       view_coords(g, si, wu.t * BM, ph, m);
       mbar_arrive_expect_tx(b_qfull, C::Q_BYTES);
-      for (int c = 0; c < C::KCH; ++c)
-        tma_load_5d(sQ + c * C::CHUNK_BYTES, mq, b_qfull, c * 64, wu.h, ph, m, wu.b);
+      for (int c = 0; c < C::KCH_QK; ++c)
+        tma_load_5d(sQ + c * C::CHUNK_BYTES, mq, b_qfull, c * C::QK_COLS, wu.h, ph, m, wu.b);
       int issued = 0;
       for (int it = 0; it < nkv; ++it) {
         const int s = it % C::KST;
         if (!mbar_wait(b_kempty(s), ((it / C::KST) & 1) ^ 1, abort_flag, p.err)) break;
         kv_coords(it, ph, m);
-        mbar_arrive_expect_tx(b_kfull(s), C::KV_BYTES);
-        for (int c = 0; c < C::KCH; ++c)
-          tma_load_5d(sK + s * C::KV_BYTES + c * C::CHUNK_BYTES, mk, b_kfull(s), c * 64, wu.h, ph,
-                      m, wu.b);
+        mbar_arrive_expect_tx(b_kfull(s), C::K_BYTES);
+        for (int c = 0; c < C::KCH_QK; ++c)
+          tma_load_5d(sK + s * C::K_BYTES + c * C::CHUNK_BYTES, mk, b_kfull(s), c * C::QK_COLS,
+                      wu.h, ph, m, wu.b);
         ++issued;
       }
       if (*abort_flag) {
@@ -342,9 +405,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         const int s = it % C::VST;
         if (!mbar_wait(b_vempty(s), ((it / C::VST) & 1) ^ 1, abort_flag, p.err)) break;
         kv_coords(it, ph, m);
-        mbar_arrive_expect_tx(b_vfull(s), C::KV_BYTES);
+        mbar_arrive_expect_tx(b_vfull(s), C::V_BYTES);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_5d(sV + s * C::KV_BYTES + c * C::CHUNK_BYTES, mv, b_vfull(s), c * 64, wu.h, ph,
+          tma_load_5d(sV + s * C::V_BYTES + c * C::CHUNK_BYTES, mv, b_vfull(s), c * 64, wu.h, ph,
                       m, wu.b);
         ++issued;
       }
@@ -363,7 +426,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
     // the other's operands. The whole warp runs the loop; one elected lane
     // issues each MMA group (descriptors are built once and advanced by adds).
     {
-      constexpr uint32_t kIdS = idesc_bf16(BM, BN, 0, 0);  // Q (K-major) x K (K-major)
+      // Q (K-major) x K (K-major): bf16, or e4m3 (format code 0 of kind::f8f6f4)
+      constexpr uint32_t kIdS = QK8 ? idesc_f16(BM, BN, 0, 0) : idesc_bf16(BM, BN, 0, 0);
       constexpr uint32_t kIdO = idesc_bf16(BM, D, 0, 1);   // P (TMEM) x V (MN-major)
       const SDesc dQ = sdesc_sw128(sQ, 16, 1024), dK = sdesc_sw128(sK, 16, 1024);
       const SDesc dV = sdesc_sw128(sV, C::CHUNK_BYTES, 1024);
@@ -378,12 +442,15 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         if (ns < nkv && test(b_kfull(ns % C::KST), (ns / C::KST) & 1) &&
             (ns == 0 || test(b_sfree, (ns - 1) & 1))) {
           tc_fence_after();
-          const uint32_t ko = (ns % C::KST) * C::KV_BYTES;
+          const uint32_t ko = (ns % C::KST) * C::K_BYTES;
           if (elect_one_sync()) {
 #pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
+            for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
               const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-              mma_ss(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
+              if (QK8)
+                mma_ss_f8(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
+              else
+                mma_ss(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
             }
             mma_commit(b_sfull);
             mma_commit(b_kempty(ns % C::KST));
@@ -395,7 +462,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         if (npv < ns && test(b_pfull, npv & 1) &&
             test(b_vfull(npv % C::VST), (npv / C::VST) & 1)) {
           tc_fence_after();
-          const uint32_t vo = (npv % C::VST) * C::KV_BYTES;
+          const uint32_t vo = (npv % C::VST) * C::V_BYTES;
           if (elect_one_sync()) {
 #pragma unroll
             for (int kk = 0; kk < BN / 16; ++kk)
@@ -446,16 +513,20 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
         for (int c = 0; c < BN; ++c)
           if (c >= lim) raw[c] = 0xff800000u;
       }
-      // row max: four independent chains of 3-input max
+      // row max: four independent chains of 3-input max over columns
+      // [4, BN - 4), then the last four columns
+      static_assert(BN % 8 == 0, "the row max takes columns in groups of 8");
       float a0 = __uint_as_float(raw[0]), a1 = __uint_as_float(raw[1]);
       float a2 = __uint_as_float(raw[2]), a3 = __uint_as_float(raw[3]);
 #pragma unroll
-      for (int c = 4; c < BN; c += 8) {
+      for (int c = 4; c + 8 <= BN; c += 8) {
         a0 = max3(a0, __uint_as_float(raw[c]), __uint_as_float(raw[c + 1]));
         a1 = max3(a1, __uint_as_float(raw[c + 2]), __uint_as_float(raw[c + 3]));
         a2 = max3(a2, __uint_as_float(raw[c + 4]), __uint_as_float(raw[c + 5]));
         a3 = max3(a3, __uint_as_float(raw[c + 6]), __uint_as_float(raw[c + 7]));
       }
+      a0 = max3(a0, __uint_as_float(raw[BN - 4]), __uint_as_float(raw[BN - 3]));
+      a1 = max3(a1, __uint_as_float(raw[BN - 2]), __uint_as_float(raw[BN - 1]));
       const float mx = max3(a0, a1, fmaxf(a2, a3));
       // The exponent reference m_run moves only when the tile's max exceeds it
       // by more than 8 (log2 units); otherwise P <= 2^8 and O is not rescaled.
@@ -514,10 +585,20 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
       __syncwarp();
       if (lane == 0) mbar_arrive(b_pfull);
     }
+    MergeWeights mw;
+    if (ok && merging) {
+      // while the last PV runs: the other patterns' lse values and the
+      // weights, after checking that the partials are stored (once every
+      // partial-storing unit is done, no per-block flag needs reading)
+      int all_done = 0;
+      if (lane == 0) all_done = ld_acquire_gpu(p.done) >= (int)p.units_p;
+      all_done = __shfl_sync(0xffffffffu, all_done, 0);
+      mw = merge_weights<D>(p, wu, si, vq, m_run, l_run, all_done != 0, abort_flag);
+    }
     if (ok && warp_wait(b_odone, (nkv - 1) & 1, abort_flag, p.err)) {
       tc_fence_after();
-      if (wu.pat == p.merger) {
-        merge_epilogue<D>(p, wu, si, vq, tl + C::TM_O, m_run, l_run, abort_flag);
+      if (merging) {
+        merge_epilogue<D>(p, wu, si, vq, tl + C::TM_O, mw);
       } else {
         // The tile's 128 partial rows are one contiguous block of the partial
         // buffer (segments own whole tiles there); each thread stores its row
@@ -541,14 +622,18 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, FwdCfg<D>::MIN_BLOCKS)
           }
         }
         if (vq < si.n) p.part_lse[prow0 + row] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
-        // every writer fences its stores; the block's flag is released once
-        // all four softmax warps have (a bounded wait: an aborted warp never
-        // arrives, and then no flag is released)
-        __threadfence();
+        // The block's flag is released once all four softmax warps have
+        // stored their rows (mbarrier, release/acquire within the CTA; a
+        // bounded wait: an aborted warp never arrives, and then no flag is
+        // released), by one thread whose gpu-scope fence and release store
+        // cover the stores the mbarrier ordered before it.
         __syncwarp();
         if (lane == 0) mbar_arrive(b_epi);
-        if (warp == 2 && lane == 0 && mbar_wait(b_epi, 0, abort_flag, p.err))
+        if (warp == 2 && lane == 0 && mbar_wait(b_epi, 0, abort_flag, p.err)) {
+          __threadfence();
           st_release_gpu(p.flags + (prow0 >> 7), 1);
+          atomicAdd(p.done, 1);
+        }
       }
     }
     tc_fence_before();

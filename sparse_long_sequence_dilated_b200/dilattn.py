@@ -32,6 +32,8 @@ SIGNATURES = {
     "dilattn_fwd_scratch_size": (_sz, [_i, _i, _i, _i, _ip, _ip, _i]),
     "dilattn_fwd": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
     "dilattn_fwd_train": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
+    "dilattn_fwd_fp8": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _c.c_float,
+                             _c.c_float, _vp]),
     "dilattn_fwd_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip, _i, _i, _vp]),
     "dilattn_bwd_workspace_size": (_sz, [_i, _i, _i, _i]),
     "dilattn_bwd": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _ip, _ip,
@@ -307,4 +309,21 @@ def fwd_seqpar(q, k, v, patterns, rank: int, world: int, kg=None, vg=None, causa
                                    lse.data_ptr(), B, L, H, d, w, r, n, int(causal), int(rank),
                                    int(world), kga, vga, _stream_handle(stream))
     _check(rc, "dilattn_fwd_seqpar")
+    return out, lse
+
+
+def fwd_fp8(q8, k8, v, patterns, q_scale: float, k_scale: float, causal: bool = True, out=None,
+            lse=None, stream=None):
+    """dilattn_fwd_fp8: q8, k8 e4m3 codes (uint8 or float8 tensors [B, N, H, 128]) with
+    per-tensor scales; v bf16. Returns (out bf16, lse)."""
+    torch = _torch()
+    B, N, H, d = _shape(v)
+    out = torch.empty_like(v) if out is None else out
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=v.device)
+    w, r, n = _patterns(patterns)
+    rc = load().dilattn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), B, N, H, d, w, r, n, int(causal), float(q_scale),
+                                float(k_scale), _stream_handle(stream))
+    _check(rc, "dilattn_fwd_fp8")
     return out, lse

@@ -133,3 +133,37 @@ def make_inputs(B: int, N: int, H: int, d: int, seed: int = 0, dtype: str = "bf1
 def workload_inputs(wl: Workload, with_dout: bool = False) -> Dict[str, np.ndarray]:
     names = ("q", "k", "v", "dout") if with_dout else ("q", "k", "v")
     return make_inputs(wl.B, wl.N, wl.H, wl.d, wl.seed, wl.dtype, names)
+
+
+def e4m3_values() -> np.ndarray:
+    """The value of every e4m3 code 0..255 (sign, 4 exponent bits with bias 7, 3
+    mantissa bits; exponent 0 is subnormal, m * 2^-9; code 0x7F / 0xFF is NaN)."""
+    vals = np.zeros(256, dtype=np.float64)
+    for c in range(256):
+        s, e, m = c >> 7, (c >> 3) & 15, c & 7
+        v = m * 2.0 ** -9 if e == 0 else (1 + m / 8.0) * 2.0 ** (e - 7)
+        vals[c] = -v if s else v
+    vals[0x7F] = vals[0xFF] = np.nan
+    return vals
+
+
+def quantize_e4m3(x: np.ndarray, amax: float = 448.0):
+    """Per-tensor e4m3 quantisation of an input: scale = max|x| / amax; each
+    x / scale rounded to the nearest e4m3 value (ties to even code).
+
+    Returns (codes uint8, scale float32, values float64 = decoded codes * scale,
+    exactly the numbers an e4m3 kernel computes on)."""
+    x = np.asarray(x, dtype=np.float64)
+    scale = np.float32(max(float(np.abs(x).max()), 1e-30) / amax)
+    y = x / np.float64(scale)
+    table = e4m3_values()
+    pos = table[:0x7F]                      # non-negative finite values, increasing
+    a = np.minimum(np.abs(y), pos[-1]).ravel()
+    hi = np.searchsorted(pos, a)            # first value >= a
+    hi = np.minimum(hi, len(pos) - 1)
+    lo = np.maximum(hi - 1, 0)
+    d_lo, d_hi = a - pos[lo], pos[hi] - a
+    pick_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    code = np.where(pick_hi, hi, lo).astype(np.uint8)
+    code = np.where(y.ravel() < 0, code | 0x80, code).astype(np.uint8).reshape(x.shape)
+    return code, scale, table[code] * np.float64(scale)

@@ -62,10 +62,14 @@ def as_f64(a: np.ndarray) -> np.ndarray:
 
 
 def _err(got: np.ndarray, want: np.ndarray):
+    """(max-abs, sum err^2, sum want^2, non-finite count, (row, col, got, want) at the max)."""
     fin = np.isfinite(got)
     e = np.abs(np.where(fin, got, 0.0) - want)
-    return (float(e.max()) if e.size else 0.0, float((e * e).sum()), float((want * want).sum()),
-            int((~fin).sum()))
+    if not e.size:
+        return 0.0, 0.0, float((want * want).sum()), int((~fin).sum()), None
+    i = int(np.argmax(e))
+    at = (i // e.shape[-1], i % e.shape[-1], float(got.ravel()[i]), float(want.ravel()[i]))
+    return float(e.max()), float((e * e).sum()), float((want * want).sum()), int((~fin).sum()), at
 
 
 def _lse_err(got: np.ndarray, want: np.ndarray):
@@ -100,7 +104,7 @@ def _task(args):
                 stats[name] = _lse_err(as_f64(arrs[name][b, h]), want_l)
             else:
                 stats[name] = _err(as_f64(arrs[name][b, :, h, :]), want[what])
-        return b, h, stats
+        return b, h, {k: (v + ((b, h),) if len(v) == 5 else v) for k, v in stats.items()}
     finally:
         for shm in held.values():
             shm.close()
@@ -194,15 +198,20 @@ def check(stats: Dict[str, list], dtype: str, lse_atol: float, what: str = ""):
             continue
         nonfinite = sum(r[3] for r in rows)
         assert nonfinite == 0, f"{label}: {nonfinite} non-finite values"
-        max_abs = max(r[0] for r in rows)
+        worst = max(rows, key=lambda r: r[0])
+        max_abs = worst[0]
         err2 = sum(r[1] for r in rows)
         want2 = sum(r[2] for r in rows)
         rel = math.sqrt(err2 / want2) if want2 > 0 else math.sqrt(err2)
+        where = ""
+        if len(worst) > 5 and worst[4] is not None:
+            (b, h), (n, c, g, w) = worst[5], worst[4]
+            where = f" at (b={b}, n={n}, h={h}, c={c}): got {g:.6f}, want {w:.6f}"
         if dtype == "bf16":
             assert max_abs <= BF16_ATOL and rel <= BF16_REL_L2, \
-                f"{label}: max_abs={max_abs:.3e} rel_l2={rel:.3e}"
+                f"{label}: max_abs={max_abs:.3e} rel_l2={rel:.3e}{where}"
         else:
-            assert max_abs <= F32_ATOL, f"{label}: max_abs={max_abs:.3e}"
+            assert max_abs <= F32_ATOL, f"{label}: max_abs={max_abs:.3e}{where}"
         summary[name] = (max_abs, rel)
     return summary
 

@@ -112,19 +112,20 @@ def test_scratch_and_workspace_sizes():
     # the r = 1 pattern merges and stores no partials; partial rows of the
     # others: B*H*nseg_i*(128*ceil(ceil(min(w,N)/r)/128)) = 2*3*(2*128 + 1*128)
     rows = 2 * 3 * (256 + 128)
-    flags = align((rows // 128 + 1) * 4 + 4)  # one flag per 128-row block, then the ticket counter
+    flags = align((rows // 128 + 1) * 4 + 8)  # one flag per 128-row block, then two counters
     assert lib.dilattn_fwd_scratch_size(2, 512, 3, 64, w, r, n) == \
         align(rows * 64 * 4) + align(rows * 4) + flags
     # no r = 1 pattern: every pattern stores partials (334 rows -> 384)
     assert lib.dilattn_fwd_scratch_size(1, 1000, 1, 64, *_pats(((1000, 3),))) == \
-        384 * 64 * 4 + align(384 * 4) + align((384 // 128 + 1) * 4 + 4)
+        384 * 64 * 4 + align(384 * 4) + align((384 // 128 + 1) * 4 + 8)
     # of two r = 1 patterns the shorter merges
     w2, r2, n2 = _pats(((512, 1), (256, 1)))
     assert lib.dilattn_fwd_scratch_size(1, 512, 1, 64, w2, r2, n2) == \
-        align(512 * 64 * 4) + align(512 * 4) + align((512 // 128 + 1) * 4 + 4)
-    # D, then 256 bytes for the key-tile kernel's unit counter (the fp32 gradients
-    # are the caller's outputs)
-    assert lib.dilattn_bwd_workspace_size(2, 512, 3, 64) == align(2 * 3 * 512 * 4) + 256
+        align(512 * 64 * 4) + align(512 * 4) + align((512 // 128 + 1) * 4 + 8)
+    # D, 256 bytes for the key-tile kernel's unit counter, fp16 copies of q and k
+    # (the fp32 gradients are the caller's outputs)
+    assert lib.dilattn_bwd_workspace_size(2, 512, 3, 64) == \
+        align(2 * 3 * 512 * 4) + 256 + 2 * align(2 * 512 * 3 * 64 * 2)
     assert lib.dilattn_fwd_scratch_size(0, 512, 3, 64, w, r, n) == 0
     assert lib.dilattn_bwd_workspace_size(0, 512, 3, 64) == 0
 

@@ -94,3 +94,37 @@ def test_selection_bit_exact(N, H, pats):
     sig = dilattn.selection(N, H, pats).cpu().numpy().view(np.uint32)
     want = oracle.selection_signature(N, H, pats)
     assert np.array_equal(sig, want)
+
+
+def _one_key_rows(N, H, pats, causal=True):
+    """(n, h) of every row whose attended set is one key (itself) in exactly one
+    pattern, from the oracle's kept-row sets: the result there must be that
+    key's v, bit for bit (P = 1, l = 1, merge weight 1)."""
+    count = np.zeros((H, N), dtype=np.int64)
+    for w, r in pats:
+        for h in range(H):
+            for seg in oracle.kept_rows(N, w, r, h):
+                count[h, seg] += np.arange(1, len(seg) + 1) if causal else len(seg)
+    h_idx, n_idx = np.nonzero(count == 1)
+    return n_idx, h_idx
+
+
+@pytest.mark.parametrize("N,H,d,pats", [
+    (16384, 8, 64, [(2048, 1), (4096, 2), (8192, 4), (16384, 8)]),
+    (8192, 4, 128, [(512, 1), (2048, 2), (8192, 4)]),
+    (4096, 3, 64, [(1024, 1)]),
+])
+def test_one_key_rows_return_v_exactly(N, H, d, pats):
+    inp = make_inputs(1, N, H, d, 11, "bf16")
+    q, k, v = to_device(inp)
+    out, lse, res = dilattn.fwd_train(q, k, v, pats, True)
+    torch.cuda.synchronize()
+    assert dilattn.device_error() == 0
+    n, h = _one_key_rows(N, H, pats)
+    assert len(n) >= H
+    got = out[0].float().cpu().numpy()[n, h]
+    assert np.array_equal(got, inp["v"][0][n, h]), "a one-key row's out differs from its v"
+    assert np.all(res[0].float().cpu().numpy()[n, h] == 0)
+    s = np.einsum("id,id->i", inp["q"][0][n, h].astype(np.float64),
+                  inp["k"][0][n, h].astype(np.float64)) / np.sqrt(d)
+    np.testing.assert_allclose(lse.cpu().numpy()[0][h, n], s, rtol=0, atol=1e-5)

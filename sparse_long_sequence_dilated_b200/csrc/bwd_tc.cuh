@@ -18,7 +18,7 @@
 // the same time on different SMs and share its Q, dO tiles and dq rows in L2.
 // Each query tile is handled as two halves h of 64
 // queries so that the tensor pipe and the row threads overlap:
-//   S^T_h  = K Q_h^T,  dP^T_h = V dO_h^T                   (SMEM x SMEM -> TMEM)
+//   S^T_h  = K Q_h^T,  dP^T_h = V dO_h^T                   (TMEM x SMEM -> TMEM)
 //   P^T_h  = exp2(S^T_h tau log2e - L log2e), dS^T_h = P^T_h (dP^T_h - D)  (threads)
 //   dV += P^T_h dO_h,  dK += dS^T_h Q_h                    (TMEM x SMEM -> TMEM)
 //   dQ  = dS K  (both halves; dS from SMEM)                (SMEM x SMEM -> TMEM)
@@ -48,9 +48,15 @@
 // (key rows) and column group cg = (w - 2) / 4, i.e. 32-column chunk 2h + cg
 // of half h.
 // TMEM columns: S^T [0,128) (half h at 64h), dP^T [128,256), dV [256,320),
-// dK [320,384), dQ two buffers [384,448), [448,512). P^T and dS^T (hi, lo)
-// overwrite S^T and dP^T in place: chunk q = [32q, 32q + 32) keeps hi at
-// +[0,16) and lo at +[16,32).
+// dK [320,384), dQ [384,448), the unit's K [448,480) and V [480,512) (fp16 and
+// bf16 pairs). P^T and dS^T (hi, lo) overwrite S^T and dP^T in place: chunk
+// q = [32q, 32q + 32) keeps hi at +[0,16) and lo at +[16,32).
+// K and V are the A operands of every S^T and dP^T product of their unit, so
+// at the start of a unit the MMA thread copies them from shared memory into
+// TMEM (tcgen05.cp) and those products read only Q and dO from shared memory:
+// half the operand bytes of a shared x shared product. One dQ accumulator
+// suffices: the row warps read pair g's dQ out while they work on half 0 of
+// pair g + 1, before dQ of pair g + 1 is issued.
 #pragma once
 
 #include "common.cuh"
@@ -102,6 +108,7 @@ struct BwdCfg {
   static constexpr int OFF_BAR = OFF_D + QST * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;
   static constexpr int TM_S = 0, TM_DP = 128, TM_DV = 256, TM_DK = 320, TM_DQ = 384;
+  static constexpr int TM_K = 448, TM_V = 480;
   static constexpr int TMEM_COLS = 512;
 };
 static_assert(BwdCfg::SMEM_BYTES <= 232448, "backward tile kernel exceeds shared memory");
@@ -233,8 +240,8 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   auto b_qempty = [&](int s) { return bars + 168u + 8u * s; };
   auto b_sdp = [&](int h) { return bars + 48u + 8u * h; };      // S^T_h, dP^T_h in TMEM
   auto b_rows = [&](int h) { return bars + 64u + 8u * h; };     // P^T_h, dS^T_h written
-  auto b_dq = [&](int j) { return bars + 80u + 8u * j; };       // dQ buffer j complete
-  auto b_dqfree = [&](int j) { return bars + 96u + 8u * j; };   // dQ buffer j read out
+  auto b_dq = [&](int j) { return bars + 80u + 8u * j; };       // dQ of pairs g = j mod 2 complete
+  auto b_dqfree = [&](int j) { return bars + 96u + 8u * j; };   // dQ of pairs g = j mod 2 read out
   const uint32_t b_accfree = bars + 112u;  // dV, dK of the unit read out
   const uint32_t b_fin = bars + 120u;      // MMA pipe drained at exit
   auto b_unit = [&](int j) { return bars + 128u + 8u * j; };    // unit index published in slot j
@@ -389,8 +396,8 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
     // The whole warp runs the loop; one elected lane issues each MMA group.
     {
       // Q, K (and dS) are fp16, V, dO (and P) bf16: every product has one type
-      constexpr uint32_t kIdS = idesc_f16(BM, 64, 0, 0);    // K x Q_h^T
-      constexpr uint32_t kIdDP = idesc_bf16(BM, 64, 0, 0);  // V x dO_h^T
+      constexpr uint32_t kIdS = idesc_f16(BM, 64, 0, 0);    // K (TMEM) x Q_h^T
+      constexpr uint32_t kIdDP = idesc_bf16(BM, 64, 0, 0);  // V (TMEM) x dO_h^T
       constexpr uint32_t kIdV = idesc_bf16(BM, D, 0, 1);    // P^T (TMEM) x dO
       constexpr uint32_t kIdK = idesc_f16(BM, D, 0, 1);     // dS^T (TMEM) x Q
       constexpr uint32_t kIdQ = idesc_f16(BM, D, 1, 1);     // dS (MN-major SMEM) x K
@@ -401,16 +408,24 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       const SDesc dQk = sdesc_sw128(sQ, 16, 1024), dDOk = sdesc_sw128(sDO, 16, 1024);
       const SDesc dQm = sdesc_sw128(sQ, C::TILE, 1024), dDOm = sdesc_sw128(sDO, C::TILE, 1024);
       const SDesc dDSm = sdesc_sw128(sDS, C::TILE, 1024), dKm = sdesc_sw128(sK, C::TILE, 1024);
+      // the unit's K and V into TMEM, 16 columns of a row per copy
+      auto copy_kv = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          tmem_cp_128x256b(tmem + C::TM_K + kk * 8, dKk.at(kk * 32));
+          tmem_cp_128x256b(tmem + C::TM_V + kk * 8, dVk.at(kk * 32));
+        }
+      };
       // S^T_h = K Q_h^T and dP^T_h = V dO_h^T for the 64 queries of half h
       auto issue_sdp = [&](uint32_t g, int h) {
         const uint32_t qo = (g % C::QST) * C::TILE + h * C::HALF;
         const uint32_t ts = tmem + C::TM_S + h * 64, tp = tmem + C::TM_DP + h * 64;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(ts, dKk.at(kk * 32), dQk.at(qo + kk * 32), kIdS, kk > 0 ? 1u : 0u);
+          mma_ts(ts, tmem + C::TM_K + kk * 8, dQk.at(qo + kk * 32), kIdS, kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tp, dVk.at(kk * 32), dDOk.at(qo + kk * 32), kIdDP, kk > 0 ? 1u : 0u);
+          mma_ts(tp, tmem + C::TM_V + kk * 8, dDOk.at(qo + kk * 32), kIdDP, kk > 0 ? 1u : 0u);
         mma_commit(b_sdp(h));
       };
       // dV += P^T_h dO_h, dK += dS^T_h Q_h (each hi + lo when `split`); `first`
@@ -434,14 +449,12 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           if (split) mma_ts(tmem + C::TM_DK, a + 16, bq, kIdK, 1u);
         }
       };
-      // dQ = dS K into TMEM buffer g & 1 (dS from shared memory)
+      // dQ = dS K into the TMEM accumulator (dS from shared memory)
       auto issue_dq = [&](uint32_t g) {
-        const int j = g & 1;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)
-          mma_ss(tmem + C::TM_DQ + j * 64, dDSm.at(kk * 2048), dKm.at(kk * 2048), kIdQ,
-                 kk > 0 ? 1u : 0u);
-        mma_commit(b_dq(j));
+          mma_ss(tmem + C::TM_DQ, dDSm.at(kk * 2048), dKm.at(kk * 2048), kIdQ, kk > 0 ? 1u : 0u);
+        mma_commit(b_dq(g & 1));
       };
       // warp-uniform non-blocking test of a barrier phase
       auto test = [&](uint32_t bar, uint32_t par) -> bool {
@@ -461,7 +474,10 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           break;
         }
         tc_fence_after();
+        // The previous unit's S^T / dP^T products, the only readers of the
+        // TMEM copies of K and V, are complete: the row warps have read them.
         if (elect_one_sync()) {
+          copy_kv();
           issue_sdp(gp, 0);
           issue_sdp(gp, 1);
         }
@@ -493,7 +509,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
               prog = true;
             }
             if (need_1 && test(b_rows(1), gp & 1) &&
-                (gp < 2 || test(b_dqfree(gp & 1), ((gp >> 1) & 1) ^ 1))) {
+                (gp < 1 || test(b_dqfree((gp - 1) & 1), ((gp - 1) >> 1) & 1))) {
               tc_fence_after();
               if (elect_one_sync()) {
                 issue_dq(gp);  // first: the row warps wait for it before their next dS store
@@ -545,7 +561,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       if (!warp_wait(b_dq(j), (g >> 1) & 1, abort_flag, p.err)) return false;
       tc_fence_after();
       uint32_t r[32];
-      tmem_ld32_sync(tl + C::TM_DQ + j * 64 + cg * 32, r);
+      tmem_ld32_sync(tl + C::TM_DQ + cg * 32, r);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

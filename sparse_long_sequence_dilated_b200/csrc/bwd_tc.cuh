@@ -47,6 +47,14 @@
 // issuer, warps 2..9 the row work: warp w serves TMEM lanes 32 (w % 4) .. + 31
 // (key rows) and column group cg = (w - 2) / 4, i.e. 32-column chunk 2h + cg
 // of half h.
+// Key tiles rotate through three shared-memory slots: unit k's K sits in slot
+// k % 3 (the B operand of its dQ products) and its V in slot (k + 1) % 3 (read
+// only by the copy into TMEM). Both of unit k + 1's slots are free once unit
+// k's copy into TMEM has completed (that commit also covers every earlier MMA,
+// unit k - 1's last dQ included), so the producer loads the next key tile
+// while the current unit runs and the MMA thread moves from one unit to the
+// next without waiting for a load. The row warps read dV and dK after the
+// commit that follows the unit's last dV / dK products.
 // TMEM columns: S^T [0,128) (half h at 64h), dP^T [128,256), dV [256,320),
 // dK [320,384), dQ [384,448), the unit's K [448,480) and V [480,512) (fp16 and
 // bf16 pairs). P^T and dS^T (hi, lo) overwrite S^T and dP^T in place: chunk
@@ -96,10 +104,12 @@ struct BwdCfg {
   static constexpr int TILE = BM * 128;   // 128 rows x 64 bf16
   static constexpr int HALF = TILE / 2;   // 64 rows
   static constexpr int SLAB = 32 * 128;   // one row warp's 32 x 32 fp32 staging block
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + TILE;
+  // K / V slots: unit k keeps K in slot k % 3 and V in slot (k + 1) % 3, so
+  // the next unit's key tile loads while this unit runs
+  static constexpr int KVS = 3;
+  static constexpr int OFF_KV = 0;
   static constexpr int QST = 3;                               // Q / dO / L / D stages
-  static constexpr int OFF_Q = OFF_V + TILE;
+  static constexpr int OFF_Q = OFF_KV + KVS * TILE;
   static constexpr int OFF_DO = OFF_Q + QST * TILE;
   static constexpr int OFF_DS = OFF_DO + QST * TILE;          // 2 halves x [128 keys][64 q]
   static constexpr int OFF_STG = OFF_DS + 2 * TILE;           // ROW_WARPS slabs
@@ -229,13 +239,16 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t sK = base + C::OFF_K, sV = base + C::OFF_V;
+  const uint32_t sKV = base + C::OFF_KV;
   const uint32_t sQ = base + C::OFF_Q, sDO = base + C::OFF_DO, sDS = base + C::OFF_DS;
   float* sL = reinterpret_cast<float*>(base_g + C::OFF_L);
   float* sD = reinterpret_cast<float*>(base_g + C::OFF_D);
   const uint32_t bars = base + C::OFF_BAR;
   const uint32_t b_kvfull = bars;         // K, V of the unit landed
-  const uint32_t b_kvempty = bars + 8u;   // every MMA of the unit is complete
+  // K, V of the unit copied into TMEM, and every MMA issued before that
+  // complete: the previous unit's V slot and the unit before's K slot are free
+  const uint32_t b_cpdone = bars + 8u;
+  const uint32_t b_accdone = bars + 16u;  // every MMA of the unit is complete (dV, dK final)
   auto b_qfull = [&](int s) { return bars + 144u + 8u * s; };   // Q, dO, L, D of stage s
   auto b_qempty = [&](int s) { return bars + 168u + 8u * s; };
   auto b_sdp = [&](int h) { return bars + 48u + 8u * h; };      // S^T_h, dP^T_h in TMEM
@@ -244,14 +257,15 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   auto b_dqfree = [&](int j) { return bars + 96u + 8u * j; };   // dQ of pairs g = j mod 2 read out
   const uint32_t b_accfree = bars + 112u;  // dV, dK of the unit read out
   const uint32_t b_fin = bars + 120u;      // MMA pipe drained at exit
-  auto b_unit = [&](int j) { return bars + 128u + 8u * j; };    // unit index published in slot j
-  volatile int* uslot = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 232);
+  auto b_unit = [&](int j) { return bars + 192u + 8u * j; };    // unit index published in slot j
+  volatile int* uslot = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 232);  // 4 slots
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
 
   if (threadIdx.x == 0) {
     mbar_init(b_kvfull, 1);
-    mbar_init(b_kvempty, 1);
+    mbar_init(b_cpdone, 1);
+    mbar_init(b_accdone, 1);
     for (int s = 0; s < C::QST; ++s) {
       mbar_init(b_qfull(s), 1);
       mbar_init(b_qempty(s), 1);
@@ -264,8 +278,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
     }
     mbar_init(b_accfree, C::ROW_WARPS);
     mbar_init(b_fin, 1);
-    mbar_init(b_unit(0), 1);
-    mbar_init(b_unit(1), 1);
+    for (int j = 0; j < 4; ++j) mbar_init(b_unit(j), 1);
     *abort_flag = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -280,9 +293,10 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   const float log2e = 1.4426950408889634f;
   // The producer takes units from the global counter one ahead of use and
-  // publishes each in slot k & 1 (phase k >> 1); p.units marks the end.
-  // Slot k & 1 is rewritten only after the MMAs of unit k - 1 completed, by
-  // which time every role has read it.
+  // publishes each in slot k & 3 (phase k >> 2); p.units marks the end. It
+  // publishes unit k + 2 only after unit k's K and V were copied into TMEM,
+  // when the row warps are at unit k - 1 or later; they read slot k & 3 at
+  // the start of unit k, before it is rewritten with unit k + 4.
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -307,20 +321,21 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
     while (cur < p.units) {
       BwdUnit U;
       bwd_unit(p, cur, U);
-      if (k > 0 && !warp_wait(b_kvempty, (k - 1) & 1, abort_flag, p.err)) {
+      // unit k's slots held V of unit k - 1 and K of unit k - 2
+      if (k > 0 && !warp_wait(b_cpdone, (k - 1) & 1, abort_flag, p.err)) {
         ok = false;
         break;
       }
       long long nxt = 0;
       if (lane == 0) {
         nxt = fetch();
-        uslot[(k + 1) & 1] = (int)nxt;
-        mbar_arrive(b_unit((k + 1) & 1));
+        uslot[(k + 1) & 3] = (int)nxt;
+        mbar_arrive(b_unit((k + 1) & 3));
         int ph, m;
         view_coords(U.g, U.si, U.u * BN, ph, m);
         mbar_arrive_expect_tx(b_kvfull, 2 * C::TILE);
-        tma_load_5d(sK, U.mk, b_kvfull, 0, U.wu.h, ph, m, U.wu.b);
-        tma_load_5d(sV, U.mv, b_kvfull, 0, U.wu.h, ph, m, U.wu.b);
+        tma_load_5d(sKV + (k % C::KVS) * C::TILE, U.mk, b_kvfull, 0, U.wu.h, ph, m, U.wu.b);
+        tma_load_5d(sKV + ((k + 1) % C::KVS) * C::TILE, U.mv, b_kvfull, 0, U.wu.h, ph, m, U.wu.b);
         BwdUnit nx;
         if (nxt < p.units && bwd_unit(p, nxt, nx)) {  // warm the L2 for the next unit
           view_coords(nx.g, nx.si, nx.u * BN, ph, m);
@@ -401,15 +416,18 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       constexpr uint32_t kIdV = idesc_bf16(BM, D, 0, 1);    // P^T (TMEM) x dO
       constexpr uint32_t kIdK = idesc_f16(BM, D, 0, 1);     // dS^T (TMEM) x Q
       constexpr uint32_t kIdQ = idesc_f16(BM, D, 1, 1);     // dS (MN-major SMEM) x K
-      // Descriptors are built once; each MMA only adds a byte offset to the
-      // low word, which keeps the issuing thread's work per MMA small (it
-      // shares its scheduler with two row warps).
-      const SDesc dKk = sdesc_sw128(sK, 16, 1024), dVk = sdesc_sw128(sV, 16, 1024);
+      // Descriptors are built once (the K / V slot ones once per unit); each
+      // MMA only adds a byte offset to the low word, which keeps the issuing
+      // thread's work per MMA small (it shares its scheduler with two row warps).
       const SDesc dQk = sdesc_sw128(sQ, 16, 1024), dDOk = sdesc_sw128(sDO, 16, 1024);
       const SDesc dQm = sdesc_sw128(sQ, C::TILE, 1024), dDOm = sdesc_sw128(sDO, C::TILE, 1024);
-      const SDesc dDSm = sdesc_sw128(sDS, C::TILE, 1024), dKm = sdesc_sw128(sK, C::TILE, 1024);
-      // the unit's K and V into TMEM, 16 columns of a row per copy
-      auto copy_kv = [&]() {
+      const SDesc dDSm = sdesc_sw128(sDS, C::TILE, 1024);
+      SDesc dKm = sdesc_sw128(sKV, C::TILE, 1024);
+      // unit k's K and V (slots k % 3, (k + 1) % 3) into TMEM, 16 columns of
+      // a row per copy; K stays in its slot as the B operand of dQ
+      auto copy_kv = [&](uint32_t k) {
+        const uint32_t sK = sKV + (k % C::KVS) * C::TILE, sV = sKV + ((k + 1) % C::KVS) * C::TILE;
+        const SDesc dKk = sdesc_sw128(sK, 16, 1024), dVk = sdesc_sw128(sV, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           tmem_cp_128x256b(tmem + C::TM_K + kk * 8, dKk.at(kk * 32));
@@ -463,11 +481,12 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       uint32_t gp = 0, k = 0;
       bool ok = true;
       for (;; ++k) {
-        if (!warp_wait(b_unit(k & 1), (k >> 1) & 1, abort_flag, p.err)) break;
-        const long long uu = uslot[k & 1];
+        if (!warp_wait(b_unit(k & 3), (k >> 2) & 1, abort_flag, p.err)) break;
+        const long long uu = uslot[k & 3];
         if (uu >= p.units) break;
         BwdUnit U;
         bwd_unit(p, uu, U);
+        dKm = sdesc_sw128(sKV + (k % C::KVS) * C::TILE, C::TILE, 1024);
         if (!warp_wait(b_kvfull, k & 1, abort_flag, p.err) ||
             !warp_wait(b_qfull(gp % C::QST), (gp / C::QST) & 1, abort_flag, p.err)) {
           ok = false;
@@ -477,7 +496,8 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         // The previous unit's S^T / dP^T products, the only readers of the
         // TMEM copies of K and V, are complete: the row warps have read them.
         if (elect_one_sync()) {
-          copy_kv();
+          copy_kv(k);
+          mma_commit(b_cpdone);
           issue_sdp(gp, 0);
           issue_sdp(gp, 1);
         }
@@ -528,7 +548,7 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           if (!ok) break;
           if (elect_one_sync()) {
             if (more) issue_sdp(gp + 1, 1);
-            else mma_commit(b_kvempty);
+            else mma_commit(b_accdone);
           }
           __syncwarp();
         }
@@ -581,8 +601,8 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
       return true;
     };
     for (uint32_t k = 0; ok; ++k) {
-      if (!warp_wait(b_unit(k & 1), (k >> 1) & 1, abort_flag, p.err)) break;
-      const long long uu = uslot[k & 1];
+      if (!warp_wait(b_unit(k & 3), (k >> 2) & 1, abort_flag, p.err)) break;
+      const long long uu = uslot[k & 3];
       if (uu >= p.units) break;
       BwdUnit U;
       bwd_unit(p, uu, U);
@@ -676,9 +696,15 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
         ok = false;
         break;
       }
-      // dV, dK of the key tile: every MMA of the unit is complete (the last dQ
-      // commit tracks them all). Rows past the segment are exact zeros (their
-      // P was forced to 0).
+      // dV, dK of the key tile, once the unit's last dV / dK products are
+      // complete (they are issued after the last dQ, so its commit does not
+      // cover them). Rows past the segment are exact zeros (their P was forced
+      // to 0).
+      if (!warp_wait(b_accdone, k & 1, abort_flag, p.err)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
       {
         uint32_t rv[32], rk[32];
         tmem_ld32_sync(tl + C::TM_DV + cg * 32, rv);

@@ -90,15 +90,10 @@ struct BwdParams {
   ErrCtx err;  // device error word and this launch's tag
 };
 
-// hi + lo products: 0 never, 1 on the first query tile of a segment, 2 always
-#ifndef DILATTN_BWD_SPLIT
-#define DILATTN_BWD_SPLIT 1
-#endif
-
 struct BwdCfg {
   static constexpr int D = 64;
-  static constexpr int SPLIT = DILATTN_BWD_SPLIT;
-  __host__ __device__ static constexpr bool split(int t) { return SPLIT == 2 || (SPLIT == 1 && t == 0); }
+  // P and dS enter dV and dK as hi + lo on the first query tile of a segment
+  __host__ __device__ static constexpr bool split(int t) { return t == 0; }
   static constexpr int ROW_WARPS = 8;
   static constexpr int THREADS = 64 + 32 * ROW_WARPS;
   static constexpr int TILE = BM * 128;   // 128 rows x 64 bf16

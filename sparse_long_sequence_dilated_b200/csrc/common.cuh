@@ -479,21 +479,6 @@ __device__ __forceinline__ void tmem_ld128_sync(uint32_t taddr, uint32_t (&v)[12
       : "memory");
 }
 
-// 2^x on the FMA and integer pipes (no MUFU), for x <= 126: x = j + f with
-// j = rint(x) taken from the low mantissa bits of x + 1.5 * 2^23, 2^f by the
-// degree-3 minimax polynomial on [-1/2, 1/2] that csrc/fit_exp2_poly.py
-// computes with the Remez exchange algorithm (max relative error 7.5e-5 in
-// float32), and 2^j added to the exponent field. x is clamped at -125, so
-// -inf gives 2^-125 (about 2.4e-38) instead of 0.
-__device__ __forceinline__ float ex2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;
-  const float f = x - (t - 12582912.f);
-  const float p = fmaf(fmaf(fmaf(5.517166853e-02f, f, 2.426111251e-01f), f, 6.932609677e-01f), f,
-                       9.999280572e-01f);
-  const unsigned j = (unsigned)(__float_as_int(t) - 0x4B400000);
-  return __uint_as_float(__float_as_uint(p) + (j << 23));
-}
 }  // namespace dil
 
 namespace dil {
@@ -591,24 +576,6 @@ __device__ __forceinline__ uint32_t pack_f16_rn(float lo, float hi) {
 // The two halves of an f16x2 word as floats (exact).
 __device__ __forceinline__ float f16_lo(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v & 0xffffu))); }
 __device__ __forceinline__ float f16_hi(uint32_t v) { return __half2float(__ushort_as_half((unsigned short)(v >> 16))); }
-// ex2_poly on a pair with packed arithmetic (same steps, same constants):
-// clamp at -125, j = rint(x) via x + 1.5 * 2^23, f = x - j, Horner for 2^f,
-// then j added to the exponent field. (t_bits << 23) equals j << 23 modulo
-// 2^32 because the rounding constant's own bits shift out.
-__device__ __forceinline__ uint64_t ex2_poly2(uint64_t x2) {
-  const float xl = fmaxf(f2_lo(x2), -125.f), xh = fmaxf(f2_hi(x2), -125.f);
-  const uint64_t xc = f2_pack(xl, xh);
-  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
-  const uint64_t t = f2_add(xc, magic);
-  const uint64_t f = f2_sub(xc, f2_sub(t, magic));
-  uint64_t p = f2_fma(f2_pack(5.517166853e-02f, 5.517166853e-02f), f,
-                      f2_pack(2.426111251e-01f, 2.426111251e-01f));
-  p = f2_fma(p, f, f2_pack(6.932609677e-01f, 6.932609677e-01f));
-  p = f2_fma(p, f, f2_pack(9.999280572e-01f, 9.999280572e-01f));
-  const uint32_t lo = (uint32_t)p + ((uint32_t)t << 23);
-  const uint32_t hi = (uint32_t)(p >> 32) + ((uint32_t)(t >> 32) << 23);
-  return ((uint64_t)hi << 32) | lo;
-}
 }  // namespace dil
 
 namespace dil {

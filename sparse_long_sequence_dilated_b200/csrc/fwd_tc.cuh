@@ -22,8 +22,7 @@
 //               S = Q K^T (SMEM x SMEM -> TMEM), O += P V (TMEM x SMEM -> TMEM).
 //   warps 2..5  softmax: warp w takes TMEM lanes 32 (w % 4) .. + 31, one query
 //               row per thread: fp32 row max (3-input max), P = exp2(S*scale - m)
-//               with packed fp32x2 arithmetic and the exp2 on the MUFU unit
-//               (DILATTN_FWD_POLY moves a share to an FMA-pipe polynomial), P
+//               with packed fp32x2 arithmetic and the exp2 on the MUFU unit, P
 //               stored to TMEM as bf16, O rescaled in TMEM when the reference
 //               max moves, epilogue.
 // Rows are one per thread: at d = 64 the softmax, not the MMA, bounds a tile,
@@ -32,12 +31,6 @@
 #pragma once
 
 #include "common.cuh"
-
-// Column pairs, of every 8, whose exp2 runs as a polynomial on the FMA pipe
-// instead of the MUFU unit.
-#ifndef DILATTN_FWD_POLY
-#define DILATTN_FWD_POLY 0
-#endif
 
 namespace dil {
 
@@ -543,12 +536,7 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
       for (int c = 0; c < BN / 2; ++c) {
         const uint64_t x2 = f2_fma(f2_pack(__uint_as_float(raw[2 * c]),
                                            __uint_as_float(raw[2 * c + 1])), sc2, negm2);
-        uint64_t p2;
-        if ((c & 7) >= 8 - DILATTN_FWD_POLY) {
-          p2 = ex2_poly2(x2);  // DILATTN_FWD_POLY pairs in 8 on the FMA pipe
-        } else {
-          p2 = f2_pack(ex2(f2_lo(x2)), ex2(f2_hi(x2)));
-        }
+        const uint64_t p2 = f2_pack(ex2(f2_lo(x2)), ex2(f2_hi(x2)));
         if (c & 1)
           sum2a = f2_add(sum2a, p2);
         else

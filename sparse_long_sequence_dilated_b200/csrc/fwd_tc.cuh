@@ -271,28 +271,6 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
   const uint32_t base = (raw_s + 1023u) & ~1023u;
   uint8_t* base_g = smem_raw + (base - raw_s);
 
-  // Units are taken in ticket order, not blockIdx order: every tile that
-  // stores partials has a smaller ticket than every merging tile, so a merging
-  // tile only ever waits for tiles that running CTAs already hold.
-  __shared__ int s_ticket;
-  if (threadIdx.x == 0) s_ticket = atomicAdd(p.counter, 1);
-  __syncthreads();
-  const long long ticket = s_ticket;
-  const TileUnit wu = ticket < p.units_p
-      ? decode_unit(p.sched, p.pat, p.B, p.H, ticket)
-      : decode_unit(p.sched_m, p.pat, p.B, p.H, ticket - p.units_p);
-  const PatternGeom g = p.pat[wu.pat];
-  const SegInfo si = seg_info(g, p.N, wu.h, wu.seg);
-  if (wu.t * BM >= si.n) {  // tile past the segment's kept rows (uniform exit)
-    if (threadIdx.x == 0 && ticket < p.units_p) atomicAdd(p.done, 1);
-    return;
-  }
-  const bool merging = wu.pat == p.merger;
-  const bool gathered = p.kv_rows[wu.pat] > 0;
-  const int kv_n = gathered ? p.kv_rows[wu.pat] : si.n;  // key rows of the segment
-  const int tq = wu.t + p.toff[wu.pat];                   // the query tile among the key tiles
-  const int nkv = p.causal ? (tq + 1) : (kv_n + BN - 1) / BN;
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -313,7 +291,14 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_g + C::OFF_BAR + 224);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_g + C::OFF_BAR + 228);
 
-  if (threadIdx.x == 0) {
+  // Units are taken in ticket order, not blockIdx order: every tile that
+  // stores partials has a smaller ticket than every merging tile, so a merging
+  // tile only ever waits for tiles that running CTAs already hold. The
+  // barriers and the TMEM allocation do not depend on the unit, so they are
+  // set up while the ticket's atomic is in flight.
+  __shared__ int s_ticket;
+  if (threadIdx.x == 0) s_ticket = atomicAdd(p.counter, 1);
+  if (threadIdx.x == 64) {
     mbar_init(b_qfull, 1);
     for (int s = 0; s < C::KST; ++s) {
       mbar_init(b_kfull(s), 1);
@@ -332,6 +317,31 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  const long long ticket = s_ticket;
+  const TileUnit wu = ticket < p.units_p
+      ? decode_unit(p.sched, p.pat, p.B, p.H, ticket)
+      : decode_unit(p.sched_m, p.pat, p.B, p.H, ticket - p.units_p);
+  const PatternGeom g = p.pat[wu.pat];
+  const SegInfo si = seg_info(g, p.N, wu.h, wu.seg);
+  if (wu.t * BM >= si.n) {  // tile past the segment's kept rows (uniform exit)
+    if (threadIdx.x == 0 && ticket < p.units_p) atomicAdd(p.done, 1);
+    if (warp == 1) tmem_dealloc(tmem, C::TMEM_COLS);
+    return;
+  }
+  const bool merging = wu.pat == p.merger;
+  const bool gathered = p.kv_rows[wu.pat] > 0;
+  const int kv_n = gathered ? p.kv_rows[wu.pat] : si.n;  // key rows of the segment
+  const int tq = wu.t + p.toff[wu.pat];                   // the query tile among the key tiles
+  const int nkv = p.causal ? (tq + 1) : (kv_n + BN - 1) / BN;
+
   // All tiles of a (pattern, segment, head) share one phase, hence one view.
   int phase0, m0;
   view_coords(g, si, 0, phase0, m0);
@@ -355,14 +365,6 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
     prefetch_tmap(mk);
     prefetch_tmap(mv);
   }
-  if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer

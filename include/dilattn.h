@@ -156,6 +156,9 @@ int dilattn_fwd_fp8(const void* q8, const void* k8, const void* v, void* out, fl
  *     overlap on the GPU -- on different streams, or from different host
  *     threads -- race on the array; the caller must order them, e.g. on one
  *     stream.
+ *   - It returns out and lse like dilattn_fwd, not the out_res residual that
+ *     dilattn_bwd takes: it serves inference; training uses
+ *     dilattn_fwd_train.
  */
 #define DILATTN_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, float* lse,

@@ -469,10 +469,6 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           mma_ss(tmem + C::TM_DQ, dDSm.at(kk * 2048), dKm.at(kk * 2048), kIdQ, kk > 0 ? 1u : 0u);
         mma_commit(b_dq(g & 1));
       };
-      // warp-uniform non-blocking test of a barrier phase
-      auto test = [&](uint32_t bar, uint32_t par) -> bool {
-        return __shfl_sync(0xffffffffu, mbar_test(bar, par) ? 1 : 0, 0) != 0;
-      };
       uint32_t gp = 0, k = 0;
       bool ok = true;
       for (;; ++k) {
@@ -508,38 +504,34 @@ __global__ void __launch_bounds__(BwdCfg::THREADS, 1) bwd_tile_kernel(const __gr
           const bool split = C::split(U.t0 + it);
           if (elect_one_sync()) issue_dvdk(gp, 0, it == 0, split);
           __syncwarp();
-          // Then, in whichever order their inputs arrive: S / dP half 0 of the
-          // next pair (Q, dO landed) and dV / dK half 1 plus dQ of this pair
-          // (half 1 written, dQ buffer read out). S / dP half 1 of the next
-          // pair goes last: it overwrites what dV / dK half 1 reads.
-          bool need_s0 = more, need_1 = true;
-          PollGuard pg;
-          while (need_s0 || need_1) {
-            bool prog = false;
-            if (need_s0 && test(b_qfull((gp + 1) % C::QST), ((gp + 1) / C::QST) & 1)) {
-              tc_fence_after();
-              if (elect_one_sync()) issue_sdp(gp + 1, 0);
-              __syncwarp();
-              need_s0 = false;
-              prog = true;
-            }
-            if (need_1 && test(b_rows(1), gp & 1) &&
-                (gp < 1 || test(b_dqfree((gp - 1) & 1), ((gp - 1) >> 1) & 1))) {
-              tc_fence_after();
-              if (elect_one_sync()) {
-                issue_dq(gp);  // first: the row warps wait for it before their next dS store
-                issue_dvdk(gp, 1, false, split);
-                mma_commit(b_qempty(gp % C::QST));
-              }
-              __syncwarp();
-              need_1 = false;
-              prog = true;
-            }
-            if (!__all_sync(0xffffffffu, pg.step(prog, abort_flag, p.err))) {
+          // Then S / dP half 0 of the next pair (its Q, dO have landed: the
+          // producer runs up to three pairs ahead), and dV / dK half 1 plus dQ
+          // of this pair once half 1 is written and the dQ accumulator read
+          // out. Both waits suspend the warp in hardware, leaving its
+          // scheduler's issue slots to the row warps that share it. S / dP
+          // half 1 of the next pair goes last: it overwrites what dV / dK
+          // half 1 reads.
+          if (more) {
+            if (!warp_wait(b_qfull((gp + 1) % C::QST), ((gp + 1) / C::QST) & 1, abort_flag, p.err)) {
               ok = false;
               break;
             }
+            tc_fence_after();
+            if (elect_one_sync()) issue_sdp(gp + 1, 0);
+            __syncwarp();
           }
+          if (!warp_wait(b_rows(1), gp & 1, abort_flag, p.err) ||
+              (gp >= 1 && !warp_wait(b_dqfree((gp - 1) & 1), ((gp - 1) >> 1) & 1, abort_flag, p.err))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one_sync()) {
+            issue_dq(gp);  // first: the row warps wait for it before their next dS store
+            issue_dvdk(gp, 1, false, split);
+            mma_commit(b_qempty(gp % C::QST));
+          }
+          __syncwarp();
           if (!ok) break;
           if (elect_one_sync()) {
             if (more) issue_sdp(gp + 1, 1);

@@ -514,21 +514,6 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16
 }  // namespace dil
 
 namespace dil {
-// Non-blocking test of an mbarrier phase.
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-}  // namespace dil
-
-namespace dil {
 // Packed fp32 pairs (sm_100): one instruction operates on two floats held in
 // a 64-bit register pair.
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
@@ -617,36 +602,6 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
 }
-}  // namespace dil
-
-namespace dil {
-// Bookkeeping of a polling loop with the same bounds as mbar_wait: step()
-// returns false once the loop has gone 4 s without progress, another warp of
-// the CTA raised *abort, or any CTA of the launch recorded a failure.
-struct PollGuard {
-  uint32_t spins = 0;
-  unsigned long long t0 = 0;
-  __device__ __forceinline__ bool step(bool progressed, volatile int* abort, const ErrCtx& err) {
-    if (progressed) {
-      spins = 0;
-      t0 = 0;
-      return true;
-    }
-    if ((++spins & 1023u) != 0) return true;
-    if (*abort || err.raised()) {
-      *abort = 1;
-      return false;
-    }
-    if (t0 == 0) {
-      t0 = globaltimer_ns();
-    } else if (globaltimer_ns() - t0 > 4000000000ull) {
-      err.raise(kErrWaitTimeout);
-      *abort = 1;
-      return false;
-    }
-    return true;
-  }
-};
 }  // namespace dil
 
 namespace dil {

@@ -10,14 +10,16 @@
 // has two views with the tensor's own base address: phases [0, r) over
 // floor(N/r) rows, and phases [0, N mod r) over floor(N/r) + 1 rows; a tile
 // at phase ph uses the second when ph < N mod r, so the view's bounds are
-// exactly the rows below N and rows past N read as zeros. The CTA writes
-// the pattern's normalised output O_i and its log-sum-exp for those rows to
-// an fp32 partial buffer; the merge kernel combines patterns.
+// exactly the rows below N and rows past N read as zeros. A CTA of the
+// merging pattern (r = 1: it keeps every row) combines every pattern's result
+// for its rows and writes out; the other patterns' CTAs write their
+// normalised output O_i and log-sum-exp to an fp32 partial buffer for it
+// (families with no r = 1 pattern combine them in a separate merge kernel).
 //
 // Warp roles (192 threads, two CTAs per SM at d = 64):
 //   warp 0      TMA producer: lane 0 loads the Q tile once, then the K ring;
 //               lane 1 the V ring.
-//   warp 1      TMEM allocator and MMA issuer (the whole warp runs the event
+//   warp 1      TMEM allocator and MMA issuer (the whole warp runs the
 //               loop, one elected lane issues each group):
 //               S = Q K^T (SMEM x SMEM -> TMEM), O += P V (TMEM x SMEM -> TMEM).
 //   warps 2..5  softmax: warp w takes TMEM lanes 32 (w % 4) .. + 31, one query
@@ -416,61 +418,63 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Event loop: S(j) = Q K_j^T as soon as K_j is resident and the softmax has
-    // read S(j-1); PV(j) as soon as P(j) and V_j are ready. Neither waits for
-    // the other's operands. The whole warp runs the loop; one elected lane
-    // issues each MMA group (descriptors are built once and advanced by adds).
+    // S(j) = Q K_j^T once K_j is resident and the softmax has read S(j-1);
+    // PV(j) once P(j) and V_j are ready. The whole warp runs the loop; one
+    // elected lane issues each MMA group (descriptors are built once and
+    // advanced by adds).
     {
       // Q (K-major) x K (K-major): bf16, or e4m3 (format code 0 of kind::f8f6f4)
       constexpr uint32_t kIdS = QK8 ? idesc_f16(BM, BN, 0, 0) : idesc_bf16(BM, BN, 0, 0);
       constexpr uint32_t kIdO = idesc_bf16(BM, D, 0, 1);   // P (TMEM) x V (MN-major)
       const SDesc dQ = sdesc_sw128(sQ, 16, 1024), dK = sdesc_sw128(sK, 16, 1024);
       const SDesc dV = sdesc_sw128(sV, C::CHUNK_BYTES, 1024);
-      auto test = [&](uint32_t bar, uint32_t par) -> bool {
-        return __shfl_sync(0xffffffffu, mbar_test(bar, par) ? 1 : 0, 0) != 0;
+      // S(j + 1) needs only that the softmax has read S(j), which it does
+      // before it stores P(j), so the products go S(0), S(1), PV(0), S(2),
+      // PV(1), ...; each wait suspends the warp in hardware.
+      auto issue_s = [&](int j) {
+        const uint32_t ko = (j % C::KST) * C::K_BYTES;
+        if (elect_one_sync()) {
+#pragma unroll
+          for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
+            const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+            if (QK8)
+              mma_ss_f8(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
+            else
+              mma_ss(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(b_sfull);
+          mma_commit(b_kempty(j % C::KST));
+        }
+        __syncwarp();
+      };
+      auto issue_pv = [&](int j) {
+        const uint32_t vo = (j % C::VST) * C::V_BYTES;
+        if (elect_one_sync()) {
+#pragma unroll
+          for (int kk = 0; kk < BN / 16; ++kk)
+            mma_ts(tmem + C::TM_O, tmem + C::TM_P + kk * 8, dV.at(vo + kk * 2048), kIdO,
+                   (j > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(b_vempty(j % C::VST));
+          mma_commit(b_odone);
+        }
+        __syncwarp();
       };
       bool ok = warp_wait(b_qfull, 0, abort_flag, p.err);
-      int ns = 0, npv = 0;
-      PollGuard pg;
-      while (ok && npv < nkv) {
-        bool progressed = false;
-        if (ns < nkv && test(b_kfull(ns % C::KST), (ns / C::KST) & 1) &&
-            (ns == 0 || test(b_sfree, (ns - 1) & 1))) {
+      for (int j = 0; ok && j <= nkv; ++j) {
+        if (j < nkv) {
+          ok = warp_wait(b_kfull(j % C::KST), (j / C::KST) & 1, abort_flag, p.err) &&
+               (j == 0 || warp_wait(b_sfree, (j - 1) & 1, abort_flag, p.err));
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t ko = (ns % C::KST) * C::K_BYTES;
-          if (elect_one_sync()) {
-#pragma unroll
-            for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
-              const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
-              if (QK8)
-                mma_ss_f8(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
-              else
-                mma_ss(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(b_sfull);
-            mma_commit(b_kempty(ns % C::KST));
-          }
-          __syncwarp();
-          ++ns;
-          progressed = true;
+          issue_s(j);
         }
-        if (npv < ns && test(b_pfull, npv & 1) &&
-            test(b_vfull(npv % C::VST), (npv / C::VST) & 1)) {
+        if (j > 0) {
+          ok = warp_wait(b_pfull, (j - 1) & 1, abort_flag, p.err) &&
+               warp_wait(b_vfull((j - 1) % C::VST), ((j - 1) / C::VST) & 1, abort_flag, p.err);
+          if (!ok) break;
           tc_fence_after();
-          const uint32_t vo = (npv % C::VST) * C::V_BYTES;
-          if (elect_one_sync()) {
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk)
-              mma_ts(tmem + C::TM_O, tmem + C::TM_P + kk * 8, dV.at(vo + kk * 2048), kIdO,
-                     (npv > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(b_vempty(npv % C::VST));
-            mma_commit(b_odone);
-          }
-          __syncwarp();
-          ++npv;
-          progressed = true;
+          issue_pv(j - 1);
         }
-        if (!__all_sync(0xffffffffu, pg.step(progressed, abort_flag, p.err))) ok = false;
       }
     }
     __syncwarp();

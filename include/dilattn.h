@@ -208,8 +208,9 @@ int dilattn_pack_dilated(const void* x, void* buf, int B, int L, int H, int d, i
  * [B][N][H][d] FLOAT32, the precision they are accumulated in (a caller
  * that keeps bf16 gradients rounds them). The probabilities are recomputed
  * from the saved lse; the row term D = rowsum(dout * O) is formed from
- * out + out_res. Workspace: D and the key-tile kernel's work counter,
- * at least dilattn_bwd_workspace_size(B, N, H, d) bytes, 256-byte aligned;
+ * out + out_res. Workspace: D, the key-tile kernel's work counter and fp16
+ * copies of q and k (the products with dS run in fp16), at least
+ * dilattn_bwd_workspace_size(B, N, H, d) bytes, 256-byte aligned;
  * the workspace and dq, dk, dv must not overlap any input or each other.
  * Calls that share a workspace or gradient buffers must not overlap on the
  * GPU. d = 64 only (DILATTN_ERR_UNSUPPORTED otherwise; the fp32 entry point

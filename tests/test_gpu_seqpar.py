@@ -20,7 +20,7 @@ from tests.gpu_util import check_close, check_lse, to_device, to_f64
 pytestmark = pytest.mark.gpu
 
 
-def _emulate(q, k, v, pats, world):
+def _emulate(q, k, v, pats, world, causal=True):
     B, N, H, d = q.shape
     L = N // world
     plans = seqpar.plan(N, world, pats)
@@ -40,7 +40,7 @@ def _emulate(q, k, v, pats, world):
                 first = p.segment_ranks(g)[0]
                 kg[p.index] = packs[p.index][0][first:first + p.ranks]
                 vg[p.index] = packs[p.index][1][first:first + p.ranks]
-        o, l = dilattn.fwd_seqpar(*blocks[g], pats, g, world, kg, vg, True)
+        o, l = dilattn.fwd_seqpar(*blocks[g], pats, g, world, kg, vg, causal)
         out[:, g * L:(g + 1) * L] = o
         lse[:, :, g * L:(g + 1) * L] = l
     return out, lse
@@ -54,17 +54,18 @@ def test_pack_dilated_rows():
         np.testing.assert_array_equal(got[:, :, h], inp["k"][:, (h % 4)::4, h])
 
 
+@pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("world", [2, 4])
-def test_small_against_oracle(world):
+def test_small_against_oracle(world, causal):
     N, H, d = 4096, 4, 64
     pats = [(512, 1), (1024, 2), (2048, 4), (4096, 8)]
     inp = make_inputs(1, N, H, d, 9, "bf16")
     q, k, v = to_device(inp)
-    out, lse = _emulate(q, k, v, pats, world)
+    out, lse = _emulate(q, k, v, pats, world, causal)
     torch.cuda.synchronize()
     assert dilattn.device_error() == 0
-    want_o, want_l = oracle.fwd(inp["q"], inp["k"], inp["v"], pats, True)
-    check_close(to_f64(out), want_o, "bf16", f"out, {world} ranks")
+    want_o, want_l = oracle.fwd(inp["q"], inp["k"], inp["v"], pats, causal)
+    check_close(to_f64(out), want_o, "bf16", f"out, {world} ranks, causal={causal}")
     check_lse(to_f64(lse), want_l, 2e-2)
 
 

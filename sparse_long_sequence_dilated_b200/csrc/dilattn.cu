@@ -232,10 +232,11 @@ int strided_map(const void* ptr, int B, int N, int H, int d, int r, int tail, CU
 
 // View of a gathered dilated buffer [ranks][B][rank_rows][H][d] bf16 whose
 // row j of head h is dilated row j of that head's segment: dims
-// {d, H, rank_rows, ranks, B}; a 128-row box never crosses a rank's block
-// (rank_rows is a multiple of 128).
-int gathered_map(const void* ptr, int B, int H, int d, int rank_rows, int ranks, CUtensorMap* out) {
-  MapKey key{ptr, B, rank_rows, H, d, -ranks, 2, 0, BM};
+// {d, H, rank_rows, ranks, B}; a box of box_rows (64 or 128) rows never
+// crosses a rank's block (rank_rows is a multiple of 128).
+int gathered_map(const void* ptr, int B, int H, int d, int rank_rows, int ranks, CUtensorMap* out,
+                 int box_rows = BM) {
+  MapKey key{ptr, B, rank_rows, H, d, -ranks, 2, 0, box_rows};
   {
     std::lock_guard<std::mutex> lk(g_map_mu);
     auto it = g_maps.find(key);
@@ -250,7 +251,7 @@ int gathered_map(const void* ptr, int B, int H, int d, int rank_rows, int ranks,
   cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rank_rows, (cuuint64_t)ranks,
                         (cuuint64_t)B};
   cuuint64_t strides[4] = {(cuuint64_t)d * 2, rowb, rowb * rank_rows * B, rowb * rank_rows};
-  cuuint32_t box[5] = {64, 1, (cuuint32_t)BM, 1, 1};
+  cuuint32_t box[5] = {64, 1, (cuuint32_t)box_rows, 1, 1};
   cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUtensorMap m;
   CUresult cr = g_encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims,
@@ -448,18 +449,21 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, void* out
     const int dtype[3] = {QK8 ? 3 : 0, QK8 ? 3 : 0, 0};
     CUtensorMap* dst[3] = {&p.tmq[i], &p.tmk[i], &p.tmv[i]};
     CUtensorMap* dst_t[3] = {&p.tmq_t[i], &p.tmk_t[i], &p.tmv_t[i]};
+    // Q tiles are BM rows; K and V tiles the kernel's key-tile rows
+    constexpr int kbn = FwdCfg<D, QK8>::BN;
     for (int j = 0; j < 3; ++j) {
-      int rc = strided_map(src[j], B, N, H, D, r[i], 0, dst[j], dtype[j]);
-      if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j], dtype[j]);
+      const int rows = j == 0 ? BM : kbn;
+      int rc = strided_map(src[j], B, N, H, D, r[i], 0, dst[j], dtype[j], rows);
+      if (rc == DILATTN_OK) rc = strided_map(src[j], B, N, H, D, r[i], 1, dst_t[j], dtype[j], rows);
       if (rc != DILATTN_OK) return rc;
     }
     if (sp != nullptr && sp->kv_rows[i] > 0) {
       p.kv_rows[i] = sp->kv_rows[i];
       p.kv_rank_rows[i] = sp->kv_rank_rows[i];
       p.toff[i] = sp->toff[i];
-      int rc = gathered_map(sp->kg[i], B, H, D, sp->kv_rank_rows[i], sp->ranks[i], &p.tmk[i]);
+      int rc = gathered_map(sp->kg[i], B, H, D, sp->kv_rank_rows[i], sp->ranks[i], &p.tmk[i], kbn);
       if (rc == DILATTN_OK)
-        rc = gathered_map(sp->vg[i], B, H, D, sp->kv_rank_rows[i], sp->ranks[i], &p.tmv[i]);
+        rc = gathered_map(sp->vg[i], B, H, D, sp->kv_rank_rows[i], sp->ranks[i], &p.tmv[i], kbn);
       if (rc != DILATTN_OK) return rc;
     }
   }

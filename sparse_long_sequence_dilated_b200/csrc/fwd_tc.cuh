@@ -29,7 +29,10 @@
 //               max moves, epilogue.
 // Rows are one per thread: at d = 64 the softmax, not the MMA, bounds a tile,
 // so its issue slots are the budget every choice above is made against.
-// TMEM columns: S [0,128), P [128,192) (bf16 pairs), O [192, 192+D).
+// Key tiles are 128 rows at d = 64 and 64 rows at d = 128, so that at both
+// sizes two CTAs share an SM (99.6 KB of shared memory and 256 TMEM columns
+// each). TMEM columns: S [0, BN), P [BN, 3 BN / 2) (bf16 pairs), O
+// [3 BN / 2, 3 BN / 2 + D).
 #pragma once
 
 #include "common.cuh"
@@ -120,14 +123,16 @@ __device__ __forceinline__ int partial_row(const PatternGeom& g, int n, int off,
 // kind::f8f6f4; V, P and O stay as in the bf16 kernel.
 template <int D, bool QK8 = false>
 struct FwdCfg {
+  static constexpr int BN = (D == 128) ? 64 : 128;  // key rows per tile (MMA N of S = Q K^T)
   static constexpr int KCH = D / 64;                 // 128-byte chunks of a bf16 row (V)
   static constexpr int KCH_QK = QK8 ? D / 128 : D / 64;  // 128-byte chunks of a Q or K row
-  static constexpr int KST = 3;                      // K ring depth (a stage frees after its S MMA)
+  static constexpr int KST = (D == 128) ? 2 : 3;     // K ring depth (a stage frees after its S MMA)
   static constexpr int VST = 2;                      // V ring depth (a stage frees after its PV MMA)
-  static constexpr int CHUNK_BYTES = BM * 128;       // 128 rows x 128 bytes
-  static constexpr int Q_BYTES = KCH_QK * CHUNK_BYTES;
-  static constexpr int K_BYTES = KCH_QK * CHUNK_BYTES;
-  static constexpr int V_BYTES = KCH * CHUNK_BYTES;
+  static constexpr int Q_CHUNK = BM * 128;           // one 128-byte column chunk of the Q tile
+  static constexpr int KV_CHUNK = BN * 128;          // ... of a K or V tile
+  static constexpr int Q_BYTES = KCH_QK * Q_CHUNK;
+  static constexpr int K_BYTES = KCH_QK * KV_CHUNK;
+  static constexpr int V_BYTES = KCH * KV_CHUNK;
   static constexpr int QK_COLS = QK8 ? 128 : 64;     // elements of a 128-byte chunk of Q or K
   static constexpr int S_KSTEPS = QK8 ? D / 32 : D / 16;  // MMA K steps of S (32 bytes each)
   static constexpr int OFF_Q = 0;
@@ -135,9 +140,9 @@ struct FwdCfg {
   static constexpr int OFF_V = OFF_K + KST * K_BYTES;
   static constexpr int OFF_BAR = OFF_V + VST * V_BYTES;
   static constexpr int SMEM_BYTES = OFF_BAR + 256 + 1024;  // + alignment slack
-  static constexpr int TM_S = 0, TM_P = 128, TM_O = 192;
+  static constexpr int TM_S = 0, TM_P = BN, TM_O = BN + BN / 2;
   static constexpr int TMEM_COLS = (TM_O + D <= 256) ? 256 : 512;
-  static constexpr int MIN_BLOCKS = (D == 64) ? 2 : 1;
+  static constexpr int MIN_BLOCKS = (TMEM_COLS == 256) ? 2 : 1;
   static constexpr int SM_WARPS = 4;             // softmax warps: one query row per thread
   static constexpr int THREADS = 64 + 32 * SM_WARPS;
 };
@@ -215,8 +220,9 @@ __device__ __forceinline__ MergeWeights merge_weights(const FwdParams& p, const 
 
 // Part 2, once the last PV is complete: O from TMEM, the partials' rows, the
 // normalised result to out (and out_res), lse.
+// All D columns at once (d = 64).
 template <int D>
-__device__ __forceinline__ void merge_epilogue(const FwdParams& p, const TileUnit& wu,
+__device__ __forceinline__ void merge_epilogue_whole(const FwdParams& p, const TileUnit& wu,
                                                const SegInfo& si, int vq, uint32_t tl_o,
                                                const MergeWeights& mw) {
   float acc[D];
@@ -264,10 +270,78 @@ __device__ __forceinline__ void merge_epilogue(const FwdParams& p, const TileUni
     p.lse[(long long)bh * p.N + n] = (mw.M + __log2f(mw.Z)) * 0.69314718055994531f;
 }
 
+// In column halves of 64, which bounds the registers the accumulator takes
+// (d = 128).
+template <int D>
+__device__ __forceinline__ void merge_epilogue_halves(const FwdParams& p, const TileUnit& wu,
+                                               const SegInfo& si, int vq, uint32_t tl_o,
+                                               const MergeWeights& mw) {
+  constexpr int CW = 64;
+#pragma unroll
+  for (int h = 0; h < D / CW; ++h) {
+    float acc[CW];
+#pragma unroll
+    for (int c4 = 0; c4 < CW / 32; ++c4) {
+      uint32_t r[32];
+      tmem_ld32_sync(tl_o + h * CW + c4 * 32, r);  // warp-collective: every lane loads
+#pragma unroll
+      for (int c = 0; c < 32; ++c) acc[c4 * 32 + c] = __uint_as_float(r[c]) * mw.w_own;
+    }
+    // rows with no result skip the rest, but still take part in the next
+    // half's (warp-collective) TMEM load
+    if (vq >= si.n || !mw.ok) continue;
+    const int n = (int)si.start + vq;
+#pragma unroll
+    for (int i = 0; i < kMaxPat; ++i) {
+      if (mw.pr[i] < 0 || mw.w[i] == 0.f) continue;
+      const float wi = mw.w[i];
+      const float4* src =
+          reinterpret_cast<const float4*>(p.part_o + (long long)mw.pr[i] * D + h * CW);
+#pragma unroll
+      for (int e = 0; e < CW / 4; ++e) {
+        const float4 x = __ldcg(src + e);
+        acc[4 * e] = fmaf(wi, x.x, acc[4 * e]);
+        acc[4 * e + 1] = fmaf(wi, x.y, acc[4 * e + 1]);
+        acc[4 * e + 2] = fmaf(wi, x.z, acc[4 * e + 2]);
+        acc[4 * e + 3] = fmaf(wi, x.w, acc[4 * e + 3]);
+      }
+    }
+    const float inv = 1.f / mw.Z;
+    const long long o0 = (((long long)wu.b * p.N + n) * p.H + wu.h) * D + h * CW;
+    uint4* dst = reinterpret_cast<uint4*>(p.out + o0);
+    uint4* rdst = p.out_res != nullptr ? reinterpret_cast<uint4*>(p.out_res + o0) : nullptr;
+#pragma unroll
+    for (int e = 0; e < CW / 8; ++e) {
+      uint32_t hi[4], lo[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float a = acc[8 * e + 2 * j] * inv, b = acc[8 * e + 2 * j + 1] * inv;
+        hi[j] = pack_bf16_rn(a, b);
+        lo[j] = pack_bf16_rn(a - __uint_as_float(hi[j] << 16), b - __uint_as_float(hi[j] & 0xffff0000u));
+      }
+      dst[e] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+      if (rdst != nullptr) rdst[e] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    if (h == D / CW - 1 && p.lse != nullptr)
+      p.lse[(long long)(wu.b * p.H + wu.h) * p.N + n] = (mw.M + __log2f(mw.Z)) * 0.69314718055994531f;
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void merge_epilogue(const FwdParams& p, const TileUnit& wu,
+                                               const SegInfo& si, int vq, uint32_t tl_o,
+                                               const MergeWeights& mw) {
+  if constexpr (D <= 64)
+    merge_epilogue_whole<D>(p, wu, si, vq, tl_o, mw);
+  else
+    merge_epilogue_halves<D>(p, wu, si, vq, tl_o, mw);
+}
+
 template <int D, bool QK8 = false>
 __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_BLOCKS)
     fwd_tile_kernel(const __grid_constant__ FwdParams p) {
   using C = FwdCfg<D, QK8>;
+  constexpr int BN = C::BN;  // this kernel's key-tile rows (the library-wide BN is 128)
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_s = smem_u32(smem_raw);
   const uint32_t base = (raw_s + 1023u) & ~1023u;
@@ -342,7 +416,12 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
   const bool gathered = p.kv_rows[wu.pat] > 0;
   const int kv_n = gathered ? p.kv_rows[wu.pat] : si.n;  // key rows of the segment
   const int tq = wu.t + p.toff[wu.pat];                   // the query tile among the key tiles
-  const int nkv = p.causal ? (tq + 1) : (kv_n + BN - 1) / BN;
+  const int qbase = tq * BM;  // key index of the tile's first query row
+  // causal: key tiles up to the one holding the tile's last query row (with
+  // BN = BM, the query tile's own)
+  const int nkv = !p.causal ? (kv_n + BN - 1) / BN
+                 : BN == BM ? tq + 1
+                            : (qbase + min(BM, si.n - wu.t * BM) - 1) / BN + 1;
 
   // All tiles of a (pattern, segment, head) share one phase, hence one view.
   int phase0, m0;
@@ -376,7 +455,7 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
       view_coords(g, si, wu.t * BM, ph, m);
       mbar_arrive_expect_tx(b_qfull, C::Q_BYTES);
       for (int c = 0; c < C::KCH_QK; ++c)
-        tma_load_5d(sQ + c * C::CHUNK_BYTES, mq, b_qfull, c * C::QK_COLS, wu.h, ph, m, wu.b);
+        tma_load_5d(sQ + c * C::Q_CHUNK, mq, b_qfull, c * C::QK_COLS, wu.h, ph, m, wu.b);
       int issued = 0;
       for (int it = 0; it < nkv; ++it) {
         const int s = it % C::KST;
@@ -384,7 +463,7 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
         kv_coords(it, ph, m);
         mbar_arrive_expect_tx(b_kfull(s), C::K_BYTES);
         for (int c = 0; c < C::KCH_QK; ++c)
-          tma_load_5d(sK + s * C::K_BYTES + c * C::CHUNK_BYTES, mk, b_kfull(s), c * C::QK_COLS,
+          tma_load_5d(sK + s * C::K_BYTES + c * C::KV_CHUNK, mk, b_kfull(s), c * C::QK_COLS,
                       wu.h, ph, m, wu.b);
         ++issued;
       }
@@ -404,7 +483,7 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
         kv_coords(it, ph, m);
         mbar_arrive_expect_tx(b_vfull(s), C::V_BYTES);
         for (int c = 0; c < C::KCH; ++c)
-          tma_load_5d(sV + s * C::V_BYTES + c * C::CHUNK_BYTES, mv, b_vfull(s), c * 64, wu.h, ph,
+          tma_load_5d(sV + s * C::V_BYTES + c * C::KV_CHUNK, mv, b_vfull(s), c * 64, wu.h, ph,
                       m, wu.b);
         ++issued;
       }
@@ -427,7 +506,7 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
       constexpr uint32_t kIdS = QK8 ? idesc_f16(BM, BN, 0, 0) : idesc_bf16(BM, BN, 0, 0);
       constexpr uint32_t kIdO = idesc_bf16(BM, D, 0, 1);   // P (TMEM) x V (MN-major)
       const SDesc dQ = sdesc_sw128(sQ, 16, 1024), dK = sdesc_sw128(sK, 16, 1024);
-      const SDesc dV = sdesc_sw128(sV, C::CHUNK_BYTES, 1024);
+      const SDesc dV = sdesc_sw128(sV, C::KV_CHUNK, 1024);
       // S(j + 1) needs only that the softmax has read S(j), which it does
       // before it stores P(j), so the products go S(0), S(1), PV(0), S(2),
       // PV(1), ...; each wait suspends the warp in hardware.
@@ -436,11 +515,12 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
         if (elect_one_sync()) {
 #pragma unroll
           for (int kk = 0; kk < C::S_KSTEPS; ++kk) {
-            const uint32_t off = (kk >> 2) * C::CHUNK_BYTES + (kk & 3) * 32;
+            const uint32_t oq = (kk >> 2) * C::Q_CHUNK + (kk & 3) * 32;
+            const uint32_t okk = C::Q_CHUNK == C::KV_CHUNK ? oq : (kk >> 2) * C::KV_CHUNK + (kk & 3) * 32;
             if (QK8)
-              mma_ss_f8(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
+              mma_ss_f8(tmem + C::TM_S, dQ.at(oq), dK.at(ko + okk), kIdS, kk > 0 ? 1u : 0u);
             else
-              mma_ss(tmem + C::TM_S, dQ.at(off), dK.at(ko + off), kIdS, kk > 0 ? 1u : 0u);
+              mma_ss(tmem + C::TM_S, dQ.at(oq), dK.at(ko + okk), kIdS, kk > 0 ? 1u : 0u);
           }
           mma_commit(b_sfull);
           mma_commit(b_kempty(j % C::KST));
@@ -495,16 +575,31 @@ __global__ void __launch_bounds__(FwdCfg<D, QK8>::THREADS, FwdCfg<D, QK8>::MIN_B
       }
       tc_fence_after();
       uint32_t raw[BN];
-      tmem_ld128_sync(tl + C::TM_S, raw);
+      if constexpr (BN == 128)
+        tmem_ld128_sync(tl + C::TM_S, raw);
+      else
+        tmem_ld32x2_sync(tl + C::TM_S, tl + C::TM_S + 32, *reinterpret_cast<uint32_t(*)[32]>(&raw[0]),
+                         *reinterpret_cast<uint32_t(*)[32]>(&raw[32]));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(b_sfree);
 
       if (p.causal) {
-        if (it == tq) {
+        // key it * BN + c against query qbase + row; only tiles that reach
+        // the diagonal hold masked columns (with BN = BM, the last one)
+        if constexpr (BN == BM) {
+          if (it == tq) {
 #pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c > row) raw[c] = 0xff800000u;  // -inf
+            for (int c = 0; c < BN; ++c)
+              if (c > row) raw[c] = 0xff800000u;  // -inf
+          }
+        } else {
+          const int off = it * BN - qbase;
+          if (off > -BN) {
+#pragma unroll
+            for (int c = 0; c < BN; ++c)
+              if (c + off > row) raw[c] = 0xff800000u;
+          }
         }
       } else if (it == nkv - 1) {
         const int lim = kv_n - it * BN;

@@ -43,6 +43,19 @@ def test_small_full(pats, causal):
     check_lse(to_f64(lse), want_l, 2e-2)
 
 
+@pytest.mark.parametrize("causal", [True, False])
+def test_ragged_full(causal):
+    # N and the segments not multiples of the 64-row key tiles or 128-row query tiles
+    pats = [(384, 1), (700, 3), (1000, 6), (1100, 12)]
+    (q8, k8, v, qs, ks), (qv, kv, vv, _) = _case(2, 1100, 3, 43)
+    out, lse = dilattn.fwd_fp8(q8, k8, v, pats, qs, ks, causal)
+    torch.cuda.synchronize()
+    assert dilattn.device_error() == 0
+    want_o, want_l = oracle.fwd(qv, kv, vv, pats, causal)
+    check_close(to_f64(out), want_o, "bf16", "fp8 out, ragged")
+    check_lse(to_f64(lse), want_l, 2e-2)
+
+
 def test_16k_every_element():
     N, H = 16384, 8
     pats = geometric_patterns(N)

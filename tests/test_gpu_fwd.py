@@ -65,6 +65,20 @@ def test_bf16_d128_small():
     _run_full(1, 1536, 4, 128, [(256, 1), (512, 2), (1536, 4)], True, "bf16", seed=2)
 
 
+# d = 128 runs 64-row key tiles against 128-row query tiles: ragged ends,
+# segments shorter than a key tile, tail views, and partial query tiles whose
+# causal extent ends inside a query tile
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("N,pats", [
+    (1100, [(384, 1), (700, 3), (1000, 6), (1100, 12)]),
+    (1100, [(100, 1), (37, 3), (1100, 1)]),
+    (1000, [(64, 5), (96, 200), (1000, 7)]),
+    (129, [(128, 1), (129, 3)]),
+])
+def test_bf16_d128_ragged(N, pats, causal):
+    _run_full(2, N, 3, 128, pats, causal, "bf16", seed=6)
+
+
 def test_f32_ragged():
     _run_full(1, 700, 3, 64, [(256, 1), (300, 3), (700, 5)], False, "f32", seed=3)
 

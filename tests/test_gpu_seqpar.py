@@ -54,10 +54,11 @@ def test_pack_dilated_rows():
         np.testing.assert_array_equal(got[:, :, h], inp["k"][:, (h % 4)::4, h])
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("world", [2, 4])
-def test_small_against_oracle(world, causal):
-    N, H, d = 4096, 4, 64
+def test_small_against_oracle(world, causal, d):
+    N, H = 4096, 4
     pats = [(512, 1), (1024, 2), (2048, 4), (4096, 8)]
     inp = make_inputs(1, N, H, d, 9, "bf16")
     q, k, v = to_device(inp)
@@ -65,7 +66,7 @@ def test_small_against_oracle(world, causal):
     torch.cuda.synchronize()
     assert dilattn.device_error() == 0
     want_o, want_l = oracle.fwd(inp["q"], inp["k"], inp["v"], pats, causal)
-    check_close(to_f64(out), want_o, "bf16", f"out, {world} ranks, causal={causal}")
+    check_close(to_f64(out), want_o, "bf16", f"out, {world} ranks, causal={causal}, d={d}")
     check_lse(to_f64(lse), want_l, 2e-2)
 
 

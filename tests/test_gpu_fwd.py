@@ -142,3 +142,33 @@ def test_one_key_rows_return_v_exactly(N, H, d, pats):
     s = np.einsum("id,id->i", inp["q"][0][n, h].astype(np.float64),
                   inp["k"][0][n, h].astype(np.float64)) / np.sqrt(d)
     np.testing.assert_allclose(lse.cpu().numpy()[0][h, n], s, rtol=0, atol=1e-5)
+
+
+@pytest.mark.parametrize("d,pats", [
+    (64, [(256, 1), (512, 2), (1024, 4)]),
+    (128, [(256, 1), (512, 2), (1024, 4)]),
+    (128, [(500, 2), (1100, 3)]),          # no r = 1 pattern: the merge pass writes it
+])
+def test_train_residual(d, pats):
+    """dilattn_fwd_train returns the same out as dilattn_fwd; out_res is the
+    rounding residual of out (at most half a bf16 unit in the last place of
+    out), and out + out_res is closer to the float64 oracle than out alone
+    (the residual removes the output rounding; what remains is the kernel's
+    own error, P entering PV as bf16)."""
+    inp = make_inputs(2, 1100, 3, d, 8, "bf16")
+    q, k, v = to_device(inp)
+    out, lse, res = dilattn.fwd_train(q, k, v, pats, True)
+    out_inf, _ = dilattn.fwd(q, k, v, pats, True)
+    torch.cuda.synchronize()
+    assert dilattn.device_error() == 0
+    assert torch.equal(out, out_inf)
+    want_o, _ = oracle.fwd(inp["q"], inp["k"], inp["v"], pats, True)
+    o1 = to_f64(out)
+    r = to_f64(res)
+    o2 = o1 + r
+    nz = o1 != 0
+    ulp = np.exp2(np.floor(np.log2(np.abs(o1[nz]))) - 7)
+    assert np.all(np.abs(r[nz]) <= ulp / 2)
+    assert np.any(r != 0)
+    rel = lambda x: np.linalg.norm(x - want_o) / np.linalg.norm(want_o)
+    assert rel(o2) < rel(o1), (rel(o2), rel(o1))

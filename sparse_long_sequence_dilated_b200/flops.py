@@ -30,11 +30,6 @@ def effective_pairs(B: int, N: int, H: int, patterns: Sequence[Tuple[int, int]],
     return B * total
 
 
-def kept_rows_total(B: int, N: int, H: int, patterns) -> int:
-    """Sum over patterns of the kept rows (the (row, pattern) count)."""
-    return B * sum(sum(segment_counts(N, w, r, h)) for (w, r) in patterns for h in range(H))
-
-
 def fwd_flops(B, N, H, d, patterns, causal=True) -> int:
     return 4 * d * effective_pairs(B, N, H, patterns, causal)
 

@@ -130,11 +130,6 @@ def make_inputs(B: int, N: int, H: int, d: int, seed: int = 0, dtype: str = "bf1
     return out
 
 
-def workload_inputs(wl: Workload, with_dout: bool = False) -> Dict[str, np.ndarray]:
-    names = ("q", "k", "v", "dout") if with_dout else ("q", "k", "v")
-    return make_inputs(wl.B, wl.N, wl.H, wl.d, wl.seed, wl.dtype, names)
-
-
 def e4m3_values() -> np.ndarray:
     """The value of every e4m3 code 0..255 (sign, 4 exponent bits with bias 7, 3
     mantissa bits; exponent 0 is subnormal, m * 2^-9; code 0x7F / 0xFF is NaN)."""

@@ -1,6 +1,6 @@
-// Backward kernels: preprocess (D = rowsum(dO * O) from the bf16 O the forward
-// returned; zero the fp32 accumulators),
-// the tcgen05 key-tile kernel, and the fp32 -> bf16 convert.
+// Backward kernels: the preprocess (D = rowsum(dO * O) from out + out_res, fp16
+// copies of q and k, the caller's fp32 gradients zeroed) and the tcgen05
+// key-tile kernel, which adds into those gradients.
 //
 // The merged forward is one softmax over the multiset union of the keys the
 // patterns give a row (LongNet pages: segments, dilation and per-head

@@ -16,7 +16,7 @@
 // normalised output O_i and log-sum-exp to an fp32 partial buffer for it
 // (families with no r = 1 pattern combine them in a separate merge kernel).
 //
-// Warp roles (192 threads, two CTAs per SM at d = 64):
+// Warp roles (192 threads, two CTAs per SM at d = 64 and at d = 128):
 //   warp 0      TMA producer: lane 0 loads the Q tile once, then the K ring;
 //               lane 1 the V ring.
 //   warp 1      TMEM allocator and MMA issuer (the whole warp runs the
@@ -119,7 +119,7 @@ __device__ __forceinline__ int partial_row(const PatternGeom& g, int n, int off,
 }
 
 // QK8: q and k are e4m3 (one byte per element; the fp8 variant, d = 128):
-// their 128-row tiles are single 128-byte chunks and S = Q K^T runs as
+// each of their rows is a single 128-byte chunk and S = Q K^T runs as
 // kind::f8f6f4; V, P and O stay as in the bf16 kernel.
 template <int D, bool QK8 = false>
 struct FwdCfg {

@@ -105,6 +105,52 @@ def test_bwd_rejects_missing_or_small_workspace():
                            1 << 20, None) == INVALID
 
 
+def test_fwd_fp8_rejects_invalid():
+    w, r, n = _pats(((128, 1),))
+    lib = dilattn.load()
+    base = (FAKE, FAKE + (4 << 20), FAKE + (8 << 20), FAKE + (16 << 20), None)
+
+    def call(d=128, qs=1.0, ks=1.0, q=FAKE):
+        return lib.dilattn_fwd_fp8(q, *base[1:], 1, 256, 2, d, w, r, n, 1, qs, ks, None)
+
+    assert call(d=64) == UNSUPPORTED                 # built for d = 128 only
+    assert call(qs=0.0) == INVALID                    # scales must be positive and finite
+    assert call(ks=-1.0) == INVALID
+    assert call(qs=float("nan")) == INVALID
+    assert call(ks=float("inf")) == INVALID
+    assert call(q=FAKE + 8) == INVALID                # misaligned
+    assert call(q=FAKE + (16 << 20)) == INVALID       # out aliases q8
+
+
+def test_seqpar_rejects_splits_it_cannot_run():
+    lib = dilattn.load()
+    L = 1024
+    q, k, v, out = (FAKE + i * (4 << 20) for i in range(4))
+
+    def call(pats, rank=0, world=2, kg=None, vg=None):
+        w, r, n = _pats(pats)
+        return lib.dilattn_fwd_seqpar(q, k, v, out, None, 1, L, 2, 64, w, r, n, 1, rank, world,
+                                      kg, vg, None)
+
+    assert call(((512, 1),), rank=2) == INVALID       # rank outside the group
+    assert call(((512, 1),), world=0) == INVALID
+    assert call(((384, 1),)) == INVALID               # a local pattern whose w does not tile L
+    assert call(((2048, 2),)) == INVALID              # spanning pattern without gathered K, V
+    arr = (ctypes.c_void_p * 1)(FAKE + (32 << 20))
+    assert call(((2048, 3),), kg=arr, vg=arr) == INVALID   # L not a multiple of r
+    assert call(((2048, 16),), kg=arr, vg=arr) == INVALID  # L / r not whole 128-row tiles
+    assert call(((3072, 2),), world=4, kg=arr, vg=arr) == INVALID  # N not a multiple of w
+
+
+def test_pack_dilated_rejects_invalid():
+    lib = dilattn.load()
+    x, buf = FAKE, FAKE + (8 << 20)
+    assert lib.dilattn_pack_dilated(x, buf, 1, 1000, 2, 64, 3, None) == INVALID  # L % r != 0
+    assert lib.dilattn_pack_dilated(x, buf, 1, 1024, 2, 96, 4, None) == INVALID  # d
+    assert lib.dilattn_pack_dilated(x + 8, buf, 1, 1024, 2, 64, 4, None) == INVALID
+    assert lib.dilattn_pack_dilated(x, x + 4096, 1, 1024, 2, 64, 4, None) == INVALID  # overlap
+
+
 def test_scratch_and_workspace_sizes():
     lib = dilattn.load()
     align = lambda x: (x + 255) // 256 * 256

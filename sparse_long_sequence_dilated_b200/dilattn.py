@@ -1,9 +1,11 @@
 """Thin ctypes binding of libdilattn (include/dilattn.h).
 
 The ``dilattn_*`` functions mirror the C entry points one to one (integer
-device pointers and sizes). ``fwd`` / ``bwd`` / ``selection`` add only
-argument marshalling for torch tensors: shape checks, output and workspace
-allocation with torch, and the current CUDA stream. Every step of the
+device pointers and sizes). The torch-facing functions (``fwd``,
+``fwd_train``, ``bwd``, ``fwd_fp8``, ``fwd_noalloc``, ``fwd_seqpar``,
+``pack_dilated``, ``selection``) add only argument marshalling for torch
+tensors: shape checks, output and workspace allocation with torch, and the
+current CUDA stream. Every step of the
 computation runs in the library's CUDA kernels; there is no other code path,
 and a missing or unloadable library raises.
 """

@@ -2,6 +2,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -417,12 +418,23 @@ size_t fwd_scratch_bytes(int B, int N, int H, int d, const int* w, const int* r,
   return fwd_scratch_layout(rows, d).total();
 }
 
+// A named host-side range for profilers (NVTX; a no-op unless a tool is
+// attached), around each launch sequence.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 template <int D, bool QK8 = false>
 int launch_fwd(const void* q, const void* k, const void* v, void* out, void* out_res, float* lse,
                int B, int N, int H, const int* w, const int* r, int npat, int causal, void* ws,
                DeviceState* st, cudaStream_t stream, const SeqParPlan* sp = nullptr,
                float qk_scale = 1.f) {
   static_assert(sizeof(FwdParams) < 32000, "kernel parameter block too large");
+  NvtxRange range(QK8 ? "dilattn forward (e4m3 q, k)" : sp != nullptr ? "dilattn forward (sequence-parallel rank)"
+                                                                        : "dilattn forward");
   FwdParams p;
   memset(&p, 0, sizeof(p));
   p.npat = npat;
@@ -513,6 +525,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* out, con
                int H,
                const int* w, const int* r, int npat, int causal, void* ws,
                DeviceState* st, cudaStream_t stream) {
+  NvtxRange range("dilattn backward");
   constexpr int D = 64;
   static_assert(sizeof(BwdParams) < 32000, "kernel parameter block too large");
   BwdParams p;

@@ -6,8 +6,13 @@ path runs (each rank sends the rows dilattn_pack_dilated extracts, the ranks
 all-gather in rank order, each keeps its segment's slice) and check the
 result against the oracle's kept rows: the gathered sequence of every head
 must be the segment's kept rows in order, and each rank's query rows must sit
-at the tile offset the kernel is given. The attention arithmetic of that path
-is checked on the GPU against the oracle (tests/test_gpu_seqpar.py)."""
+at the tile offset the kernel is given. A second set of gloo ranks carries
+the decomposition through in float64: each rank attends its block's local
+patterns, attends its kept query rows of every spanning pattern to the
+gathered rows (causal from the tile offset the plan gives), merges through
+the log-sum-exp of the denominators, and must reproduce the oracle's merged
+rows of its block. The kernels of that path are checked on the GPU against
+the oracle (tests/test_gpu_seqpar.py)."""
 import os
 import socket
 
@@ -15,6 +20,8 @@ import numpy as np
 import pytest
 import torch
 import torch.multiprocessing as mp
+
+import math
 
 import oracle
 from sparse_long_sequence_dilated_b200 import seqpar
@@ -114,3 +121,107 @@ def test_gloo_ranks_gather_the_segments_kept_rows(tmp_path, world):
                        start_method="spawn")
     for r in range(world):
         assert (tmp_path / f"r{r}.txt").read_text() == "[]"
+
+
+# (N, world, patterns): local and spanning patterns, one with w > N
+MATH_CASES = [
+    (2048, 2, [(256, 1), (512, 2), (2048, 4), (1024, 8)]),
+    (4096, 4, [(512, 1), (1024, 2), (2048, 4), (4096, 8)]),
+    (2048, 2, [(512, 1), (4096, 8)]),
+]
+
+
+def _attend(Q, K, V, tau, causal, q0):
+    """Softmax attention of rows Q, which sit at positions q0, q0 + 1, ... of
+    the key sequence K (causal: a row sees keys up to its own position)."""
+    S = tau * (Q @ K.T)
+    if causal:
+        pos = q0 + np.arange(Q.shape[0])[:, None]
+        S = np.where(np.arange(K.shape[0])[None, :] <= pos, S, -np.inf)
+    m = S.max(axis=1)
+    E = np.exp(S - m[:, None])
+    Z = E.sum(axis=1)
+    return (E @ V) / Z[:, None], m + np.log(Z)
+
+
+def _rank_math(rank: int, world: int, port: int, out_dir: str, case: int, causal: bool):
+    import sys
+    if ROOT not in sys.path:
+        sys.path.insert(0, ROOT)
+    import datetime
+
+    import torch.distributed as dist
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        N, _, pats = MATH_CASES[case]
+        H, d = 3, 8
+        L = N // world
+        tau = 1.0 / math.sqrt(d)
+        rng = np.random.default_rng(23)
+        q_full, k_full, v_full = (rng.standard_normal((1, N, H, d)) for _ in range(3))
+        blk = slice(rank * L, (rank + 1) * L)
+        qb, kb, vb = (x[0, blk] for x in (q_full, k_full, v_full))   # [L, H, d]
+        plans = seqpar.plan(N, world, pats)
+        outs, lses = [], []
+        local = [p for p in plans if not p.spans]
+        if local:
+            O_i, lse_i = oracle.fwd_per_pattern(qb[None], kb[None], vb[None],
+                                                [(p.w, p.r) for p in local], causal)
+            outs += [O_i[j, 0] for j in range(len(local))]
+            lses += [lse_i[j, 0] for j in range(len(local))]
+        for p in plans:
+            if not p.spans:
+                continue
+            send = torch.empty((2, L // p.r, H, d), dtype=torch.float64)
+            rows = {}
+            for h in range(H):
+                rows[h] = [x - rank * L for x in seqpar.packed_positions(p, L, rank, h)]
+                send[0, :, h] = torch.from_numpy(kb[rows[h], h])
+                send[1, :, h] = torch.from_numpy(vb[rows[h], h])
+            recv = [torch.empty_like(send) for _ in range(world)]
+            dist.all_gather(recv, send)
+            gathered = torch.cat([recv[g] for g in p.segment_ranks(rank)], dim=1).numpy()
+            O = np.zeros((L, H, d))
+            lse = np.full((H, L), -np.inf)
+            for h in range(H):
+                O[rows[h], h], lse[h, rows[h]] = _attend(
+                    qb[rows[h], h], gathered[0, :, h], gathered[1, :, h], tau, causal,
+                    p.tile_offset(rank) * seqpar.BM)
+            outs.append(O)
+            lses.append(lse)
+        # merge through the denominators, row by row of this block
+        lse_all = np.stack(lses)                        # [P, H, L]
+        mx = lse_all.max(axis=0)
+        sel = np.isfinite(mx)
+        mx0 = np.where(sel, mx, 0.0)
+        wts = np.exp(lse_all - mx0[None])               # exp(-inf) = 0 for rows not kept
+        tot = np.where(sel, wts.sum(axis=0), 1.0)
+        L_m = np.where(sel, mx0 + np.log(tot), -np.inf)
+        out = sum(np.transpose(wts[i] / tot, (1, 0))[:, :, None] * outs[i]
+                  for i in range(len(outs)))
+        want_o, want_l = oracle.fwd(q_full, k_full, v_full, pats, causal)
+        err_o = float(np.abs(out - want_o[0, blk]).max())
+        same_inf = bool(np.array_equal(np.isinf(L_m), np.isinf(want_l[0, :, blk])))
+        fin = np.isfinite(L_m)
+        err_l = float(np.abs(L_m[fin] - want_l[0, :, blk][fin]).max()) if fin.any() else 0.0
+        with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
+            f.write(repr((err_o, err_l, same_inf, int(sel.sum()))))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("case", range(len(MATH_CASES)))
+def test_gloo_ranks_reproduce_the_merged_rows(tmp_path, case, causal):
+    world = MATH_CASES[case][1]
+    port = _free_port()
+    mp.start_processes(_rank_math, args=(world, port, str(tmp_path), case, causal),
+                       nprocs=world, join=True, start_method="spawn")
+    for r in range(world):
+        err_o, err_l, same_inf, kept = eval((tmp_path / f"r{r}.txt").read_text())
+        assert same_inf and kept > 0
+        assert err_o < 1e-12 and err_l < 1e-12, (r, err_o, err_l)

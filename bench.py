@@ -362,12 +362,12 @@ def run_reference(args, rank: int, world: int):
     nproc = max(1, min(wl.B * wl.H, usable_cpus()))
     pool = OraclePool(nproc)
     try:
-        # size each step so that warm-up + timed steps take about three minutes
-        budget_s = 180.0 / max(1, args.steps + args.warmup)
+        # size each step so that warm-up + timed steps take about --reference-seconds
+        budget_s = args.reference_seconds / max(1, args.steps + args.warmup)
         cal_n = min(wl.N, 4096)
         wall, _, _ = pool.run(wl, cal_n, wl.backward, wl.seed)
         n_prefix = int(min(wl.N, max(2048, cal_n * budget_s / max(wall, 1e-3))))
-        n_prefix = max(2048, (n_prefix // 2048) * 2048)
+        n_prefix = min(wl.N, max(2048, (n_prefix // 2048) * 2048))
         for _ in range(args.warmup):
             pool.run(wl, n_prefix, wl.backward, wl.seed)
         tot_t, tot_w = 0.0, 0
@@ -837,6 +837,8 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--reference-seconds", type=float, default=180.0,
+                    help="--impl reference: host time the warm-up and timed steps aim for")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the detail runs (B = 4 step, length sweep, wide d = 128, graph)")
     args = ap.parse_args()

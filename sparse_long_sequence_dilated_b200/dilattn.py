@@ -4,8 +4,9 @@ The ``dilattn_*`` functions mirror the C entry points one to one (integer
 device pointers and sizes). The torch-facing functions (``fwd``,
 ``fwd_train``, ``bwd``, ``fwd_fp8``, ``fwd_noalloc``, ``fwd_seqpar``,
 ``pack_dilated``, ``selection``) add only argument marshalling for torch
-tensors: shape checks, output and workspace allocation with torch, and the
-current CUDA stream. Every step of the
+tensors: checks of every tensor's shape, dtype, layout and device (the C
+entry points take bare pointers and cannot see a buffer's size), output and
+workspace allocation with torch, and the current CUDA stream. Every step of the
 computation runs in the library's CUDA kernels; there is no other code path,
 and a missing or unloadable library raises.
 """
@@ -125,6 +126,19 @@ def _shape(q):
     return tuple(int(x) for x in q.shape)
 
 
+def _need(t, name, shape, dtypes, device=None):
+    """Raise ValueError unless t is a contiguous CUDA tensor of this shape, one of
+    these dtypes and (if given) on this device."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(map(str, dtypes))}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not t.is_cuda or (device is not None and t.device != device):
+        raise ValueError(f"{name} must be on {device if device is not None else 'a CUDA device'}")
+
+
 def fwd_scratch_size(B, N, H, d, patterns) -> int:
     w, r, n = _patterns(patterns)
     return int(load().dilattn_fwd_scratch_size(B, N, H, d, w, r, n))
@@ -141,16 +155,15 @@ def fwd(q, k, v, patterns, causal: bool = True, out=None, lse=None, stream=None)
     """
     torch = _torch()
     B, N, H, d = _shape(q)
-    for t in (k, v):
-        if tuple(t.shape) != (B, N, H, d) or t.dtype != q.dtype:
-            raise ValueError("q, k, v must share shape and dtype")
-    for t in (q, k, v):
-        if not t.is_cuda or not t.is_contiguous():
-            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    _need(q, "q", (B, N, H, d), (torch.bfloat16, torch.float32))
+    for name, t in (("k", k), ("v", v)):
+        _need(t, name, (B, N, H, d), (q.dtype,), q.device)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _need(out, "out", (B, N, H, d), (q.dtype,), q.device)
+    _need(lse, "lse", (B, H, N), (torch.float32,), q.device)
     w, r, n = _patterns(patterns)
     s = _stream_handle(stream)
     lib = load()
@@ -175,10 +188,16 @@ def fwd_train(q, k, v, patterns, causal: bool = True, out=None, lse=None, out_re
     B, N, H, d = _shape(q)
     if q.dtype != torch.bfloat16:
         raise ValueError("fwd_train takes bf16 tensors (the fp32 path needs no residual)")
+    _need(q, "q", (B, N, H, d), (torch.bfloat16,))
+    for name, t in (("k", k), ("v", v)):
+        _need(t, name, (B, N, H, d), (torch.bfloat16,), q.device)
     out = torch.empty_like(q) if out is None else out
     out_res = torch.empty_like(q) if out_res is None else out_res
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    for name, t in (("out", out), ("out_res", out_res)):
+        _need(t, name, (B, N, H, d), (torch.bfloat16,), q.device)
+    _need(lse, "lse", (B, H, N), (torch.float32,), q.device)
     w, r, n = _patterns(patterns)
     rc = load().dilattn_fwd_train(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                   out_res.data_ptr(), lse.data_ptr(), B, N, H, d, w, r, n,
@@ -193,19 +212,26 @@ def bwd(q, k, v, out, lse, dout, patterns, causal: bool = True, out_res=None, dq
     out, lse (and, for bf16, out_res: use fwd_train)."""
     torch = _torch()
     B, N, H, d = _shape(q)
-    for t in (k, v, out, dout):
-        if tuple(t.shape) != (B, N, H, d) or t.dtype != q.dtype:
-            raise ValueError("q, k, v, out, dout must share shape and dtype")
+    _need(q, "q", (B, N, H, d), (torch.bfloat16, torch.float32))
+    for name, t in (("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _need(t, name, (B, N, H, d), (q.dtype,), q.device)
+    _need(lse, "lse", (B, H, N), (torch.float32,), q.device)
     gdt = torch.float32  # the bf16 path returns fp32 gradients, the fp32 path fp32 too
     dq = torch.empty(q.shape, dtype=gdt, device=q.device) if dq is None else dq
     dk = torch.empty(q.shape, dtype=gdt, device=q.device) if dk is None else dk
     dv = torch.empty(q.shape, dtype=gdt, device=q.device) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _need(t, name, (B, N, H, d), (gdt,), q.device)
     w, r, n = _patterns(patterns)
-    s = _stream_handle(stream)
-    lib = load()
     if q.dtype == torch.bfloat16:
         if out_res is None:
             raise ValueError("the bf16 backward takes out_res from fwd_train")
+        _need(out_res, "out_res", (B, N, H, d), (torch.bfloat16,), q.device)
+        if workspace is not None:
+            _need(workspace, "workspace", (workspace.numel(),), (torch.uint8,), q.device)
+    s = _stream_handle(stream)
+    lib = load()
+    if q.dtype == torch.bfloat16:
         need = int(lib.dilattn_bwd_workspace_size(B, N, H, d))
         if workspace is None:
             workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
@@ -269,10 +295,15 @@ def fwd_noalloc(q, k, v, patterns, causal: bool = True, out=None, lse=None, stre
     given; pass them in to allocate nothing.)"""
     torch = _torch()
     B, N, H, d = _shape(q)
+    _need(q, "q", (B, N, H, d), (torch.bfloat16,))
+    for name, t in (("k", k), ("v", v)):
+        _need(t, name, (B, N, H, d), (torch.bfloat16,), q.device)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _need(out, "out", (B, N, H, d), (torch.bfloat16,), q.device)
+    _need(lse, "lse", (B, H, N), (torch.float32,), q.device)
     w, r, n = _patterns(patterns)
     rc = load().dilattn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                     lse.data_ptr(), B, N, H, d, w, r, n, int(causal),
@@ -285,8 +316,12 @@ def pack_dilated(x, r: int, out=None, stream=None):
     """dilattn_pack_dilated: [B, L/r, H, d] with row m of head h = x[:, (h mod r) + m r, h]."""
     torch = _torch()
     B, L, H, d = _shape(x)
+    if r < 1 or L % r != 0:
+        raise ValueError(f"the block length {L} must be a multiple of r = {r}")
+    _need(x, "x", (B, L, H, d), (torch.bfloat16,))
     if out is None:
         out = torch.empty((B, L // r, H, d), dtype=x.dtype, device=x.device)
+    _need(out, "out", (B, L // r, H, d), (torch.bfloat16,), x.device)
     rc = load().dilattn_pack_dilated(x.data_ptr(), out.data_ptr(), B, L, H, d, int(r),
                                      _stream_handle(stream))
     _check(rc, "dilattn_pack_dilated")
@@ -297,12 +332,29 @@ def fwd_seqpar(q, k, v, patterns, rank: int, world: int, kg=None, vg=None, causa
                out=None, lse=None, stream=None):
     """dilattn_fwd_seqpar on this rank's block; kg / vg: per pattern the gathered
     [ranks, B, L/r, H, d] buffer or None."""
+    from . import seqpar
+
     torch = _torch()
     B, L, H, d = _shape(q)
+    _need(q, "q", (B, L, H, d), (torch.bfloat16,))
+    for name, t in (("k", k), ("v", v)):
+        _need(t, name, (B, L, H, d), (torch.bfloat16,), q.device)
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, L), dtype=torch.float32, device=q.device)
+    _need(out, "out", (B, L, H, d), (torch.bfloat16,), q.device)
+    _need(lse, "lse", (B, H, L), (torch.float32,), q.device)
+    # the gathered rows of every pattern whose segments span ranks
+    for p in seqpar.plan(L * world, world, patterns):
+        for name, bufs in (("kg", kg), ("vg", vg)):
+            t = bufs[p.index] if bufs is not None and p.index < len(bufs) else None
+            if p.spans:
+                if t is None:
+                    raise ValueError(f"{name}[{p.index}]: pattern {p.index} spans ranks and "
+                                     "needs its gathered rows")
+                _need(t, f"{name}[{p.index}]", (p.ranks, B, p.rank_rows, H, d),
+                      (torch.bfloat16,), q.device)
     w, r, n = _patterns(patterns)
     ptr = lambda t: t.data_ptr() if t is not None else None
     kga = (_vp * max(n, 1))(*[ptr(t) for t in (kg or [None] * n)])
@@ -320,9 +372,15 @@ def fwd_fp8(q8, k8, v, patterns, q_scale: float, k_scale: float, causal: bool = 
     per-tensor scales; v bf16. Returns (out bf16, lse)."""
     torch = _torch()
     B, N, H, d = _shape(v)
+    _need(v, "v", (B, N, H, d), (torch.bfloat16,))
+    codes = (torch.uint8, torch.float8_e4m3fn)
+    _need(q8, "q8", (B, N, H, d), codes, v.device)
+    _need(k8, "k8", (B, N, H, d), codes, v.device)
     out = torch.empty_like(v) if out is None else out
     if lse is None:
         lse = torch.empty((B, H, N), dtype=torch.float32, device=v.device)
+    _need(out, "out", (B, N, H, d), (torch.bfloat16,), v.device)
+    _need(lse, "lse", (B, H, N), (torch.float32,), v.device)
     w, r, n = _patterns(patterns)
     rc = load().dilattn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), v.data_ptr(), out.data_ptr(),
                                 lse.data_ptr(), B, N, H, d, w, r, n, int(causal), float(q_scale),

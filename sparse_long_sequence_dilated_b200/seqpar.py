@@ -99,8 +99,12 @@ def forward(q, k, v, patterns, causal: bool = True, group=None, out=None, lse=No
         bufs = []
         for x in (k, v):
             send = dilattn.pack_dilated(x, p.r, stream=stream)
-            recv = torch.empty((world,) + tuple(send.shape), dtype=send.dtype, device=send.device)
+            # the ranks' packs concatenated along the batch dimension (the form
+            # every backend takes), the same memory as [world, B, L/r, H, d]
+            recv = torch.empty((world * send.shape[0],) + tuple(send.shape[1:]),
+                               dtype=send.dtype, device=send.device)
             dist.all_gather_into_tensor(recv, send, group=group)
+            recv = recv.view((world,) + tuple(send.shape))
             first = p.segment_ranks(rank)[0]
             bufs.append(recv[first:first + p.ranks])  # contiguous: [ranks, B, L/r, H, d]
         kg[p.index], vg[p.index] = bufs

@@ -11,8 +11,10 @@ the decomposition through in float64: each rank attends its block's local
 patterns, attends its kept query rows of every spanning pattern to the
 gathered rows (causal from the tile offset the plan gives), merges through
 the log-sum-exp of the denominators, and must reproduce the oracle's merged
-rows of its block. The kernels of that path are checked on the GPU against
-the oracle (tests/test_gpu_seqpar.py)."""
+rows of its block. A third set runs seqpar.forward itself (its packing calls,
+its all-gather and its slicing of the gathered buffers) with the two library
+calls replaced by host stand-ins, batch 2, against the oracle. The kernels of
+that path are checked on the GPU against the oracle (tests/test_gpu_seqpar.py)."""
 import os
 import socket
 
@@ -144,7 +146,54 @@ def _attend(Q, K, V, tau, causal, q0):
     return (E @ V) / Z[:, None], m + np.log(Z)
 
 
-def _rank_math(rank: int, world: int, port: int, out_dir: str, case: int, causal: bool):
+def _block_rows(qb, kb, vb, pats, plans, rank, gathered, causal):
+    """This rank's merged rows in float64: qb, kb, vb [L, H, d] its block;
+    gathered[i] = (K, V), each [rows, H, d], the kept rows of this rank's
+    segment of spanning pattern i in sequence order. Returns out [L, H, d] and
+    lse [H, L]."""
+    L, H, d = qb.shape
+    tau = 1.0 / math.sqrt(d)
+    outs, lses = [], []
+    local = [p for p in plans if not p.spans]
+    if local:
+        O_i, lse_i = oracle.fwd_per_pattern(qb[None], kb[None], vb[None],
+                                            [(p.w, p.r) for p in local], causal)
+        outs += [O_i[j, 0] for j in range(len(local))]
+        lses += [lse_i[j, 0] for j in range(len(local))]
+    for p in plans:
+        if not p.spans:
+            continue
+        K, V = gathered[p.index]
+        O = np.zeros((L, H, d))
+        lse = np.full((H, L), -np.inf)
+        for h in range(H):
+            rows = [x - rank * L for x in seqpar.packed_positions(p, L, rank, h)]
+            O[rows, h], lse[h, rows] = _attend(qb[rows, h], K[:, h], V[:, h], tau, causal,
+                                               p.tile_offset(rank) * seqpar.BM)
+        outs.append(O)
+        lses.append(lse)
+    # merge through the denominators, row by row of this block
+    lse_all = np.stack(lses)                        # [P, H, L]
+    mx = lse_all.max(axis=0)
+    sel = np.isfinite(mx)
+    mx0 = np.where(sel, mx, 0.0)
+    wts = np.exp(lse_all - mx0[None])               # exp(-inf) = 0 for rows not kept
+    tot = np.where(sel, wts.sum(axis=0), 1.0)
+    lse_m = np.where(sel, mx0 + np.log(tot), -np.inf)
+    out = sum(np.transpose(wts[i] / tot, (1, 0))[:, :, None] * outs[i] for i in range(len(outs)))
+    return out, lse_m
+
+
+def _errors(out, lse, want_o, want_l):
+    """(max |out error|, max |lse error| over finite rows, same -inf rows, kept rows)."""
+    err_o = float(np.abs(out - want_o).max())
+    same_inf = bool(np.array_equal(np.isinf(lse), np.isinf(want_l)))
+    fin = np.isfinite(lse)
+    err_l = float(np.abs(lse[fin] - want_l[fin]).max()) if fin.any() else 0.0
+    return err_o, err_l, same_inf, int(fin.sum())
+
+
+def _init_gloo(rank, world, port):
     import sys
     if ROOT not in sys.path:
         sys.path.insert(0, ROOT)
@@ -156,60 +205,41 @@ def _rank_math(rank: int, world: int, port: int, out_dir: str, case: int, causal
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=datetime.timedelta(seconds=60))
+    return dist
+
+
+def _full_inputs(N, H, d):
+    rng = np.random.default_rng(23)
+    return [rng.standard_normal((1, N, H, d)) for _ in range(3)]
+
+
+def _rank_math(rank: int, world: int, port: int, out_dir: str, case: int, causal: bool):
+    dist = _init_gloo(rank, world, port)
     try:
         N, _, pats = MATH_CASES[case]
         H, d = 3, 8
         L = N // world
-        tau = 1.0 / math.sqrt(d)
-        rng = np.random.default_rng(23)
-        q_full, k_full, v_full = (rng.standard_normal((1, N, H, d)) for _ in range(3))
+        q_full, k_full, v_full = _full_inputs(N, H, d)
         blk = slice(rank * L, (rank + 1) * L)
         qb, kb, vb = (x[0, blk] for x in (q_full, k_full, v_full))   # [L, H, d]
         plans = seqpar.plan(N, world, pats)
-        outs, lses = [], []
-        local = [p for p in plans if not p.spans]
-        if local:
-            O_i, lse_i = oracle.fwd_per_pattern(qb[None], kb[None], vb[None],
-                                                [(p.w, p.r) for p in local], causal)
-            outs += [O_i[j, 0] for j in range(len(local))]
-            lses += [lse_i[j, 0] for j in range(len(local))]
+        gathered = {}
         for p in plans:
             if not p.spans:
                 continue
             send = torch.empty((2, L // p.r, H, d), dtype=torch.float64)
-            rows = {}
             for h in range(H):
-                rows[h] = [x - rank * L for x in seqpar.packed_positions(p, L, rank, h)]
-                send[0, :, h] = torch.from_numpy(kb[rows[h], h])
-                send[1, :, h] = torch.from_numpy(vb[rows[h], h])
+                rows = [x - rank * L for x in seqpar.packed_positions(p, L, rank, h)]
+                send[0, :, h] = torch.from_numpy(kb[rows, h])
+                send[1, :, h] = torch.from_numpy(vb[rows, h])
             recv = [torch.empty_like(send) for _ in range(world)]
             dist.all_gather(recv, send)
-            gathered = torch.cat([recv[g] for g in p.segment_ranks(rank)], dim=1).numpy()
-            O = np.zeros((L, H, d))
-            lse = np.full((H, L), -np.inf)
-            for h in range(H):
-                O[rows[h], h], lse[h, rows[h]] = _attend(
-                    qb[rows[h], h], gathered[0, :, h], gathered[1, :, h], tau, causal,
-                    p.tile_offset(rank) * seqpar.BM)
-            outs.append(O)
-            lses.append(lse)
-        # merge through the denominators, row by row of this block
-        lse_all = np.stack(lses)                        # [P, H, L]
-        mx = lse_all.max(axis=0)
-        sel = np.isfinite(mx)
-        mx0 = np.where(sel, mx, 0.0)
-        wts = np.exp(lse_all - mx0[None])               # exp(-inf) = 0 for rows not kept
-        tot = np.where(sel, wts.sum(axis=0), 1.0)
-        L_m = np.where(sel, mx0 + np.log(tot), -np.inf)
-        out = sum(np.transpose(wts[i] / tot, (1, 0))[:, :, None] * outs[i]
-                  for i in range(len(outs)))
+            g = torch.cat([recv[r_] for r_ in p.segment_ranks(rank)], dim=1).numpy()
+            gathered[p.index] = (g[0], g[1])
+        out, lse = _block_rows(qb, kb, vb, pats, plans, rank, gathered, causal)
         want_o, want_l = oracle.fwd(q_full, k_full, v_full, pats, causal)
-        err_o = float(np.abs(out - want_o[0, blk]).max())
-        same_inf = bool(np.array_equal(np.isinf(L_m), np.isinf(want_l[0, :, blk])))
-        fin = np.isfinite(L_m)
-        err_l = float(np.abs(L_m[fin] - want_l[0, :, blk][fin]).max()) if fin.any() else 0.0
         with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
-            f.write(repr((err_o, err_l, same_inf, int(sel.sum()))))
+            f.write(repr(_errors(out, lse, want_o[0, blk], want_l[0, :, blk])))
     finally:
         dist.destroy_process_group()
 
@@ -225,3 +255,75 @@ def test_gloo_ranks_reproduce_the_merged_rows(tmp_path, case, causal):
         err_o, err_l, same_inf, kept = eval((tmp_path / f"r{r}.txt").read_text())
         assert same_inf and kept > 0
         assert err_o < 1e-12 and err_l < 1e-12, (r, err_o, err_l)
+
+
+def _rank_forward(rank: int, world: int, port: int, out_dir: str, case: int, causal: bool):
+    """seqpar.forward as a user calls it, on gloo ranks: its packing calls, its
+    all-gather and its slicing of the gathered buffers run as written; the two
+    library calls are replaced by host stand-ins (the packing rule, and the
+    float64 decomposition on the buffers forward hands over)."""
+    dist = _init_gloo(rank, world, port)
+    try:
+        from sparse_long_sequence_dilated_b200 import dilattn
+
+        N, _, pats = MATH_CASES[case]
+        B, H, d = 2, 3, 8
+        L = N // world
+        rng = np.random.default_rng(29)
+        q_full, k_full, v_full = (rng.standard_normal((B, N, H, d)) for _ in range(3))
+        blk = slice(rank * L, (rank + 1) * L)
+        plans = seqpar.plan(N, world, pats)
+        seen = []
+
+        def pack_dilated(x, r, out=None, stream=None):
+            Bx, Lx, Hx, dx = x.shape
+            buf = torch.empty((Bx, Lx // r, Hx, dx), dtype=x.dtype)
+            for h in range(Hx):
+                buf[:, :, h] = x[:, (h % r)::r, h]
+            return buf
+
+        def fwd_seqpar(q, k, v, patterns, rank_, world_, kg, vg, causal_, out, lse, stream):
+            seen.append((rank_, world_, causal_, [g is None for g in kg], [g is None for g in vg]))
+            out = torch.empty_like(q)
+            lse = torch.empty((q.shape[0], q.shape[2], q.shape[1]), dtype=torch.float64)
+            for b in range(q.shape[0]):
+                gathered = {}
+                for p in plans:
+                    if p.spans:
+                        assert tuple(kg[p.index].shape) == (p.ranks, q.shape[0], p.rank_rows, H, d)
+                        gathered[p.index] = tuple(
+                            t[:, b].reshape(p.ranks * p.rank_rows, H, d).numpy() for t in
+                            (kg[p.index], vg[p.index]))
+                o_b, l_b = _block_rows(q[b].numpy(), k[b].numpy(), v[b].numpy(), patterns, plans,
+                                       rank_, gathered, causal_)
+                out[b], lse[b] = torch.from_numpy(o_b), torch.from_numpy(l_b)
+            return out, lse
+
+        dilattn.pack_dilated = pack_dilated
+        dilattn.fwd_seqpar = fwd_seqpar
+        blocks = [torch.from_numpy(np.ascontiguousarray(x[:, blk])) for x in (q_full, k_full, v_full)]
+        out, lse = seqpar.forward(*blocks, pats, causal)
+        want_o, want_l = oracle.fwd(q_full, k_full, v_full, pats, causal)
+        errs = [_errors(out[b].numpy(), lse[b].numpy(), want_o[b, blk], want_l[b, :, blk])
+                for b in range(B)]
+        spans = [not p.spans for p in plans]
+        ok_calls = seen == [(rank, world, causal, spans, spans)]
+        with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
+            f.write(repr((errs, ok_calls)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("case", range(len(MATH_CASES)))
+def test_seqpar_forward_on_gloo_ranks(tmp_path, case, causal):
+    world = MATH_CASES[case][1]
+    port = _free_port()
+    mp.start_processes(_rank_forward, args=(world, port, str(tmp_path), case, causal),
+                       nprocs=world, join=True, start_method="spawn")
+    for r in range(world):
+        errs, ok_calls = eval((tmp_path / f"r{r}.txt").read_text())
+        assert ok_calls, r
+        for err_o, err_l, same_inf, kept in errs:
+            assert same_inf and kept > 0
+            assert err_o < 1e-12 and err_l < 1e-12, (r, err_o, err_l)

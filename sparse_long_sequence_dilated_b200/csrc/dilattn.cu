@@ -804,6 +804,12 @@ int dilattn_fwd_f32(const float* q, const float* k, const float* v, float* out, 
   const size_t tb = (size_t)B * N * H * d * 4;
   if (overlaps(out, tb, q, tb) || overlaps(out, tb, k, tb) || overlaps(out, tb, v, tb))
     return DILATTN_ERR_INVALID_ARG;
+  if (lse != nullptr) {
+    const size_t lb = (size_t)B * H * N * 4;
+    if (overlaps(lse, lb, q, tb) || overlaps(lse, lb, k, tb) || overlaps(lse, lb, v, tb) ||
+        overlaps(lse, lb, out, tb))
+      return DILATTN_ERR_INVALID_ARG;
+  }
   if (d != 64 && d != 128) return DILATTN_ERR_UNSUPPORTED;
   DeviceState* st = nullptr;
   rc = device_state(&st);

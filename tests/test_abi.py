@@ -74,6 +74,20 @@ def test_fwd_rejects_invalid(kw):
     assert _fwd(**kw) == INVALID
 
 
+def test_fwd_rejects_lse_overlapping_a_tensor():
+    # bf16 tensors of 64 KiB at 4 MiB spacing; lse (2 KiB) starting inside k or out
+    assert _fwd(lse=FAKE + 4096 * 1024 + 1024) == INVALID
+    assert _fwd(lse=FAKE + 16384 * 1024 + 65536 - 16) == INVALID
+    w, r, n = _pats(((128, 1),))
+    lib = dilattn.load()
+    t = [FAKE + i * (4096 * 1024) for i in range(5)]
+    args = (1, 256, 2, 64, w, r, n, 1, None)
+    # the fp32 forward: out over q, lse over out, lse over v
+    assert lib.dilattn_fwd_f32(t[0], t[1], t[2], t[0] + 4096, t[4], *args) == INVALID
+    assert lib.dilattn_fwd_f32(t[0], t[1], t[2], t[3], t[3] + 65536, *args) == INVALID
+    assert lib.dilattn_fwd_f32(t[0], t[1], t[2], t[3], t[2] + 16, *args) == INVALID
+
+
 def test_fwd_rejects_unsupported_head_dim():
     assert _fwd(d=96) == UNSUPPORTED
 

@@ -184,6 +184,11 @@ int dilattn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, 
  * [ranks][B][L/r][H][d] buffers of this rank's segment. Only those dilated
  * rows cross between ranks, never a full block. kg, vg may be NULL when no
  * pattern spans ranks. Scratch as in dilattn_fwd.
+ *
+ * Errors: DILATTN_ERR_INVALID_ARG for the argument errors of dilattn_fwd, a
+ * rank outside [0, world), a split the rules above do not allow, a missing
+ * or misaligned gathered buffer, or out / lse overlapping a gathered buffer
+ * (the kernel reads those while it writes out and lse).
  */
 int dilattn_fwd_seqpar(const void* q, const void* k, const void* v, void* out, float* lse,
                        int B, int L, int H, int d, const int* w, const int* r, int npat,

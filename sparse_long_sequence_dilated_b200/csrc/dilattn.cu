@@ -936,6 +936,12 @@ int dilattn_fwd_seqpar(const void* q, const void* k, const void* v, void* out, f
     sp.toff[i] = (rank % sp.ranks[i]) * (sp.kv_rank_rows[i] / BM);
     sp.kg[i] = kg[i];
     sp.vg[i] = vg[i];
+    // the gathered rows are read while out and lse are written
+    const size_t gb = (size_t)sp.kv_rows[i] * B * H * d * 2;
+    const size_t tb = (size_t)B * L * H * d * 2, lb = (size_t)B * H * L * 4;
+    if (overlaps(out, tb, kg[i], gb) || overlaps(out, tb, vg[i], gb) ||
+        (lse != nullptr && (overlaps(lse, lb, kg[i], gb) || overlaps(lse, lb, vg[i], gb))))
+      return DILATTN_ERR_INVALID_ARG;
   }
   DeviceState* st = nullptr;
   rc = device_state(&st);

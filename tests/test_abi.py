@@ -154,6 +154,15 @@ def test_seqpar_rejects_splits_it_cannot_run():
     assert call(((2048, 3),), kg=arr, vg=arr) == INVALID   # L not a multiple of r
     assert call(((2048, 16),), kg=arr, vg=arr) == INVALID  # L / r not whole 128-row tiles
     assert call(((3072, 2),), world=4, kg=arr, vg=arr) == INVALID  # N not a multiple of w
+    # out (256 KiB at FAKE + 12 MiB) over the gathered rows (2 ranks x 512 rows, 256 KiB)
+    inside = (ctypes.c_void_p * 1)(out + (128 << 10))
+    assert call(((2048, 2),), kg=inside, vg=arr) == INVALID
+    assert call(((2048, 2),), kg=arr, vg=(ctypes.c_void_p * 1)(out - (128 << 10))) == INVALID
+    # lse (8 KiB) inside the gathered k rows
+    w, r, n = _pats(((2048, 2),))
+    assert lib.dilattn_fwd_seqpar(q, k, v, out, FAKE + (32 << 20) + 4096, 1, L, 2, 64, w, r, n,
+                                  1, 0, 2, arr, (ctypes.c_void_p * 1)(FAKE + (40 << 20)),
+                                  None) == INVALID
 
 
 def test_pack_dilated_rejects_invalid():

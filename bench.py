@@ -426,6 +426,24 @@ TRAIN = "train_b4_32k"                                      # B = 4 training ste
 WIDE = "wide_128k"                                          # d = 128, forward
 
 
+def extra_counts(B, N, H, d, pats, causal, fwd_ms: float, bwd_ms, hbm_gbs: float,
+                 out_res: bool) -> dict:
+    """The forward's algorithmic HBM bytes and rate (against the measured copy
+    bandwidth), and the backward's rate under the 8 d count without the
+    recomputed S (labelled; the headline counts 10 d)."""
+    fb = flops.fwd_bytes(B, N, H, d, pats, out_res)
+    gbs = fb / (fwd_ms * 1e-3) / 1e9
+    ent = {"fwd_algorithmic_bytes": fb, "fwd_hbm_gbs": gbs, "fwd_frac_of_hbm": gbs / hbm_gbs}
+    if bwd_ms is not None:
+        b8 = flops.bwd_flops_no_recompute(B, N, H, d, pats, causal)
+        ent["bwd_tflops_8d_no_recompute"] = b8 / (bwd_ms * 1e-3) / 1e12
+    return ent
+
+
+def hbm_peak() -> float:
+    return float(load_peaks()[0].get("hbm_gbs", PEAK_FALLBACK["hbm_gbs"]))
+
+
 def time_workload(dilattn, dev, name: str, flush_buf, peak: float, steps: int = 3,
                   warmup: int = 2):
     """Whole-call and tile-kernel times of one workload on i.i.d. N(0, 1) bf16 inputs
@@ -487,6 +505,9 @@ def time_workload(dilattn, dev, name: str, flush_buf, peak: float, steps: int = 
                     "step_tflops": (fw + bw) / (fm + bm) / 1e9,
                     "step_frac_of_peak": (fw + bw) / (fm + bm) / 1e9 / peak,
                     "tokens_per_s": B * N / ((fm + bm) * 1e-3)})
+    ent.update(extra_counts(B, N, H, d, pats, wl.causal, fm,
+                            statistics.median(bwhole) if with_bwd else None, hbm_peak(),
+                            with_bwd))
     del q, k, v, do, ws_b
     torch.cuda.empty_cache()
     return ent
@@ -796,6 +817,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "fwd_tile_ms": fwd_tile_ms, "bwd_tile_ms": bwd_tile_ms,
             "fwd_tile_tflops": fwd_tile_tf, "bwd_tile_tflops": bwd_tile_tf,
             "peak_source": peak_src,
+            **extra_counts(B, N, H, d, pats, causal, fwd_ms, bwd_ms, hbm_peak(), True),
         },
         "roofline": {"bound": "tensor", "kernel": dom, "achieved": dom_tf, "peak": peak,
                      "unit": "TFLOP/s", "frac": dom_tf / peak,

@@ -444,8 +444,8 @@ def hbm_peak() -> float:
     return float(load_peaks()[0].get("hbm_gbs", PEAK_FALLBACK["hbm_gbs"]))
 
 
-def time_workload(dilattn, dev, name: str, flush_buf, peak: float, steps: int = 3,
-                  warmup: int = 2):
+def time_workload(dilattn, dev, name: str, flush_buf, peak: float, steps: int = 20,
+                  warmup: int = 5):
     """Whole-call and tile-kernel times of one workload on i.i.d. N(0, 1) bf16 inputs
     drawn on the device (the kernels' cost does not depend on the values), L2
     flushed before every call; medians of `steps` timed calls after `warmup`."""
@@ -513,8 +513,8 @@ def time_workload(dilattn, dev, name: str, flush_buf, peak: float, steps: int = 
     return ent
 
 
-def time_fp8(dilattn, dev, flush_buf, peak: float, name: str = WIDE, steps: int = 3,
-             warmup: int = 2):
+def time_fp8(dilattn, dev, flush_buf, peak: float, name: str = WIDE, steps: int = 20,
+             warmup: int = 5):
     """The FP8 forward (e4m3 q and k, bf16 v) of a d = 128 workload next to the bf16
     forward of the same inputs. Peak: S runs at the FP8 rate (twice bf16, the
     nominal ratio) and PV at the bf16 rate, half of the FLOPs each, so the

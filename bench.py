@@ -230,6 +230,13 @@ class ClockSampler:
         return rec
 
 
+def physical_gpu(local_rank: int) -> str:
+    """The GPU this rank drives, as nvidia-smi and NVML name it: entry local_rank of
+    CUDA_VISIBLE_DEVICES when that lists the node's GPUs, else the local rank."""
+    vis = [x.strip() for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    return vis[local_rank] if local_rank < len(vis) else str(local_rank)
+
+
 def make_clock_sampler(gpu_index: str):
     try:
         import pynvml
@@ -751,8 +758,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if dilattn.device_error() != 0:
         raise RuntimeError("a kernel reported a device-side error during warm-up")
 
-    gpu_index = os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank]
-    sampler = make_clock_sampler(gpu_index)
+    sampler = make_clock_sampler(physical_gpu(local_rank))
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()

@@ -1,8 +1,11 @@
 """Host logic of the benchmark's clock record, with a stand-in for nvidia-smi.
 
 The record must come from samples taken inside the timed region only, report the
-median SM clock of the samples under load, and name every throttle reason seen."""
+median SM clock of the samples under load, and name every throttle reason seen;
+and each rank must sample the GPU it drives."""
 import os
+
+import pytest
 
 import bench
 
@@ -66,3 +69,19 @@ def test_missing_nvidia_smi(monkeypatch):
     rec = s.stop()
     assert rec["samples"] == 0 and rec["reasons"] == ["nvidia-smi unavailable"]
     assert not os.path.exists(s.path)  # no temporary file left behind
+
+
+@pytest.mark.parametrize("env,local_rank,want", [
+    (None, 0, "0"),
+    (None, 3, "3"),                          # nothing set: every rank sees every GPU
+    ("4,5,6,7", 0, "4"),
+    ("4,5,6,7", 2, "6"),
+    ("GPU-aaaa, GPU-bbbb", 1, "GPU-bbbb"),
+    ("", 1, "1"),
+])
+def test_physical_gpu(monkeypatch, env, local_rank, want):
+    if env is None:
+        monkeypatch.delenv("CUDA_VISIBLE_DEVICES", raising=False)
+    else:
+        monkeypatch.setenv("CUDA_VISIBLE_DEVICES", env)
+    assert bench.physical_gpu(local_rank) == want

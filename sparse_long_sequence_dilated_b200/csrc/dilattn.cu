@@ -512,7 +512,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* out, void* out
   mp.out_res = reinterpret_cast<__nv_bfloat16*>(out_res);
   mp.lse = lse;
   const long long total_rows = (long long)B * N * H;
-  constexpr int rows_per_block = 256 / DILATTN_MERGE_TPR;
+  constexpr int rows_per_block = 256 / kMergeTpr;
   const long long blocks = (total_rows + rows_per_block - 1) / rows_per_block;
   merge_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(mp);
   e = cudaGetLastError();

@@ -50,16 +50,14 @@ struct MergeParams {
   float* lse;              // may be null
 };
 
-// DILATTN_MERGE_TPR threads per output row (default 4; 8 and 16 were measured
-// slower at d = 64), each owning D / TPR consecutive columns; 256 / TPR rows
-// per 256-thread block. Single pass with a running max, so every partial load is
+// kMergeTpr threads per output row (8 and 16 were measured slower at d = 64),
+// each owning D / kMergeTpr consecutive columns; 256 / kMergeTpr rows per
+// 256-thread block. Single pass with a running max, so every partial load is
 // independent of the previous pattern's result.
-#ifndef DILATTN_MERGE_TPR
-#define DILATTN_MERGE_TPR 4
-#endif
+constexpr int kMergeTpr = 4;
 template <int D>
 __global__ void __launch_bounds__(256) merge_kernel(const __grid_constant__ MergeParams p) {
-  constexpr int TPR = DILATTN_MERGE_TPR;  // threads per output row
+  constexpr int TPR = kMergeTpr;  // threads per output row
   constexpr int PER = D / TPR;            // floats per thread
   static_assert(PER % 4 == 0, "each thread owns whole float4 groups");
   const long long row = (long long)blockIdx.x * (256 / TPR) + (threadIdx.x / TPR);

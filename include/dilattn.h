@@ -196,9 +196,12 @@ int dilattn_fwd_seqpar(const void* q, const void* k, const void* v, void* out, f
                        const void* const* vg, cudaStream_t stream);
 
 /*
- * The rows a rank sends for a pattern of dilation r that spans ranks:
- * buf[b][m][h][:] = x[b][(h mod r) + m r][h][:] for m < L / r (x and buf
- * bf16, device; buf holds B * (L / r) * H * d elements; L a multiple of r).
+ * The rows a rank sends for a pattern of dilation r that spans ranks (the
+ * dilated rows of LongNet's distributed algorithm, same passages as
+ * dilattn_fwd_seqpar): buf[b][m][h][:] = x[b][(h mod r) + m r][h][:] for
+ * m < L / r (x and buf bf16, device, 16-byte aligned, caller-owned; buf holds
+ * B * (L / r) * H * d elements; L a multiple of r; d in {64, 128}).
+ * Errors: DILATTN_ERR_INVALID_ARG for any of those violated or buf overlapping x.
  */
 int dilattn_pack_dilated(const void* x, void* buf, int B, int L, int H, int d, int r,
                          cudaStream_t stream);

@@ -1,0 +1,176 @@
+"""The forward's unit schedule on the host, exhaustively.
+
+The tile kernel launches one CTA per unit index and maps the index to a
+(pattern, segment, batch, head, query tile) with decode_unit (csrc/common.cuh);
+the host builds the schedule it decodes with make_geoms, pick_merger and
+make_schedule (csrc/dilattn.cu). This test cuts those four functions out of
+the sources as they are (decode_unit renamed, its device qualifiers dropped),
+compiles them with nvcc into a host program and decodes every unit of many
+geometries: fixed ones (the LongNet-base layer, the geometric family at 1M,
+two r = 1 patterns, no r = 1 pattern, ragged and r > w shapes) and random ones.
+Every (pattern, segment, batch, head, tile) must come out exactly once, the
+tile level must never rise within a schedule, the partial-storing patterns'
+units must all precede the merging pattern's, and the unit counts must be the
+sums of nseg * B * H * ntiles. No GPU is touched."""
+import os
+import re
+import shutil
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "sparse_long_sequence_dilated_b200", "csrc")
+
+
+def _cut(text: str, head: str) -> str:
+    """The definition that starts at `head`, through its matching closing brace."""
+    i = text.index(head)
+    j = text.index("{", i)
+    depth = 0
+    for k in range(j, len(text)):
+        if text[k] == "{":
+            depth += 1
+        elif text[k] == "}":
+            depth -= 1
+            if depth == 0:
+                return text[i:k + 1]
+    raise ValueError(head)
+
+
+def _program() -> str:
+    common = open(os.path.join(CSRC, "common.cuh"), encoding="utf-8").read()
+    host = open(os.path.join(CSRC, "dilattn.cu"), encoding="utf-8").read()
+    decode = _cut(common, "__device__ __forceinline__ TileUnit decode_unit(")
+    decode = re.sub(r"^__device__ __forceinline__ TileUnit decode_unit\(",
+                    "static inline TileUnit host_decode_unit(", decode)
+    funcs = "\n\n".join(_cut(host, h) for h in ("long long make_geoms(", "int pick_merger(",
+                                               "long long make_schedule("))
+    return r"""
+#include <algorithm>
+#include <climits>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+#include "common.cuh"
+namespace dil {
+""" + decode + "\n\n" + funcs + r"""
+}  // namespace dil
+using namespace dil;
+
+static uint64_t state = 0x9E3779B97F4A7C15ull;
+static uint64_t next() { state ^= state << 13; state ^= state >> 7; state ^= state << 17; return state; }
+static long long checks = 0;
+
+// Returns the number of violations for one geometry.
+static long long check(int B, int N, int H, int npat, const int* w, const int* r) {
+  PatternGeom geo[kMaxPat];
+  const int merger = pick_merger(w, r, npat);
+  make_geoms(B, N, H, w, r, npat, geo, merger);
+  const unsigned all = (1u << npat) - 1u, mbit = merger >= 0 ? (1u << merger) : 0u;
+  Sched sp, sm;
+  const long long up = make_schedule(geo, npat, B, H, sp, all & ~mbit);
+  const long long um = mbit ? make_schedule(geo, npat, B, H, sm, mbit) : 0;
+  long long base[kMaxPat + 1];
+  base[0] = 0;
+  for (int i = 0; i < npat; ++i)
+    base[i + 1] = base[i] + (long long)geo[i].nseg * B * H * geo[i].ntiles;
+  long long want_p = 0;
+  for (int i = 0; i < npat; ++i)
+    if (i != merger) want_p += base[i + 1] - base[i];
+  std::vector<char> seen((size_t)base[npat], 0);
+  long long bad = 0;
+  if (up != want_p || up + um != base[npat]) ++bad;
+  auto visit = [&](const Sched& sc, long long units, unsigned mask) {
+    int prev_t = INT_MAX;
+    for (long long u = 0; u < units; ++u) {
+      ++checks;
+      const TileUnit t = host_decode_unit(sc, geo, B, H, u);
+      if (t.pat < 0 || t.pat >= npat || !((mask >> t.pat) & 1u) || t.seg < 0 ||
+          t.seg >= geo[t.pat].nseg || t.b < 0 || t.b >= B || t.h < 0 || t.h >= H || t.t < 0 ||
+          t.t >= geo[t.pat].ntiles) {
+        if (bad < 3) printf("N=%d u=%lld out of range: pat %d seg %d b %d h %d t %d\n", N, u,
+                            t.pat, t.seg, t.b, t.h, t.t);
+        ++bad;
+        continue;
+      }
+      if (t.t > prev_t) ++bad;  // longest first: the level never rises
+      prev_t = t.t;
+      const long long idx =
+          base[t.pat] + (((long long)t.seg * B + t.b) * H + t.h) * geo[t.pat].ntiles + t.t;
+      if (seen[(size_t)idx]) ++bad;
+      seen[(size_t)idx] = 1;
+    }
+  };
+  visit(sp, up, all & ~mbit);
+  visit(sm, um, mbit);
+  for (char c : seen)
+    if (!c) ++bad;
+  return bad;
+}
+
+int main() {
+  long long bad = 0;
+  {  // the LongNet-base layer, and at B = 4
+    const int w[] = {2048, 4096, 8192, 16384, 32768}, r[] = {1, 2, 4, 6, 12};
+    bad += check(1, 32768, 12, 5, w, r);
+    bad += check(4, 32768, 12, 5, w, r);
+  }
+  {  // the geometric family at 1M, two batches
+    int w[10], r[10];
+    for (int i = 0; i < 10; ++i) { w[i] = 2048 << i; r[i] = 1 << i; }
+    bad += check(2, 1 << 20, 12, 10, w, r);
+  }
+  {  // two r = 1 patterns; no r = 1 pattern; ragged; r > w; one row
+    const int w1[] = {256, 1024, 512}, r1[] = {1, 1, 2};
+    bad += check(2, 1100, 3, 3, w1, r1);
+    const int w2[] = {500, 1536}, r2[] = {2, 3};
+    bad += check(2, 1536, 4, 2, w2, r2);
+    const int w3[] = {384, 700, 1000, 1100}, r3[] = {1, 3, 6, 12};
+    bad += check(2, 1100, 3, 4, w3, r3);
+    const int w4[] = {64, 96, 1100}, r4[] = {5, 200, 7};
+    bad += check(2, 1100, 3, 3, w4, r4);
+    const int w5[] = {1}, r5[] = {1};
+    bad += check(1, 1, 2, 1, w5, r5);
+  }
+  {  // sixteen patterns
+    int w[16], r[16];
+    for (int i = 0; i < 16; ++i) { w[i] = 64 * (i + 1); r[i] = 1 + i % 5; }
+    bad += check(1, 3000, 2, 16, w, r);
+  }
+  for (int c = 0; c < 3000; ++c) {  // random geometries
+    const int N = 1 + (int)(next() % 5000);
+    const int B = 1 + (int)(next() % 3), H = 1 + (int)(next() % 5);
+    const int npat = 1 + (int)(next() % 6);
+    int w[kMaxPat], r[kMaxPat];
+    for (int i = 0; i < npat; ++i) {
+      w[i] = 1 + (int)(next() % (uint64_t)(N + N / 2 + 1));
+      r[i] = 1 + (int)(next() % 300);
+      if (next() % 4 == 0) r[i] = 1;
+    }
+    bad += check(B, N, H, npat, w, r);
+  }
+  printf("checks %lld bad %lld\n", checks, bad);
+  return bad != 0;
+}
+"""
+
+
+def _nvcc():
+    for cand in (shutil.which("nvcc"), "/usr/local/cuda/bin/nvcc"):
+        if cand and os.path.exists(cand):
+            return cand
+    return None
+
+
+@pytest.mark.skipif(_nvcc() is None, reason="nvcc not found")
+def test_every_unit_decodes_once(tmp_path):
+    src = tmp_path / "sched.cu"
+    src.write_text(_program())
+    exe = tmp_path / "sched"
+    build = subprocess.run([_nvcc(), "-O2", "-std=c++17", "-I", CSRC, "-o", str(exe), str(src)],
+                           capture_output=True, text=True, timeout=600)
+    assert build.returncode == 0, build.stdout + build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=600)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert "bad 0" in run.stdout, run.stdout

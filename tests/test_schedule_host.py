@@ -11,7 +11,12 @@ two r = 1 patterns, no r = 1 pattern, ragged and r > w shapes) and random ones.
 Every (pattern, segment, batch, head, tile) must come out exactly once, the
 tile level must never rise within a schedule, the partial-storing patterns'
 units must all precede the merging pattern's, and the unit counts must be the
-sums of nseg * B * H * ntiles. No GPU is touched."""
+sums of nseg * B * H * ntiles. The backward's schedule gets the same check
+from the decode part of bwd_unit (csrc/bwd_tc.cuh) and the group-order block of
+launch_bwd: every (pattern, segment, batch, head, key tile) once, patterns in
+groups by descending tile count, a unit with rows exactly when its key tile
+holds a kept row, and its query tiles from its own (causal) or the first
+through the segment's last. No GPU is touched."""
 import os
 import re
 import shutil
@@ -168,6 +173,143 @@ def test_every_unit_decodes_once(tmp_path):
     src = tmp_path / "sched.cu"
     src.write_text(_program())
     exe = tmp_path / "sched"
+    build = subprocess.run([_nvcc(), "-O2", "-std=c++17", "-I", CSRC, "-o", str(exe), str(src)],
+                           capture_output=True, text=True, timeout=600)
+    assert build.returncode == 0, build.stdout + build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=600)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert "bad 0" in run.stdout, run.stdout
+
+
+def _bwd_program() -> str:
+    """The backward's unit order (built inline in launch_bwd) and the decode part
+    of bwd_unit, cut from the sources, over a stand-in for the parameter block
+    holding the fields they read."""
+    bwd = open(os.path.join(CSRC, "bwd_tc.cuh"), encoding="utf-8").read()
+    host = open(os.path.join(CSRC, "dilattn.cu"), encoding="utf-8").read()
+    i = bwd.index("__device__ __forceinline__ bool bwd_unit(")
+    j = bwd.index("  // all tiles of a (pattern, segment, head) share one phase", i)
+    decode = bwd[i:j].replace("__device__ __forceinline__ bool bwd_unit(",
+                              "static inline bool host_bwd_unit(") + "  return true;\n}\n"
+    order = _cut(host, "  // group-major unit order:")  # the comment and its block
+    funcs = _cut(host, "long long make_geoms(")
+    return r"""
+#include <algorithm>
+#include <climits>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+#include "common.cuh"
+namespace dil {
+struct BwdParams {
+  PatternGeom pat[kMaxPat];
+  int npat, B, N, H, causal;
+  int gorder[kMaxPat];
+  long long gstart[kMaxPat + 1];
+};
+struct BwdUnit {
+  TileUnit wu;
+  PatternGeom g;
+  SegInfo si;
+  int u, t0, np;
+};
+""" + decode + "\n" + funcs + r"""
+static long long build_order(BwdParams& p, int npat, int B, int H) {
+""" + order + r"""
+  return p.gstart[npat];
+}
+}  // namespace dil
+using namespace dil;
+
+static uint64_t state = 0xD1B54A32D192ED03ull;
+static uint64_t next() { state ^= state << 13; state ^= state >> 7; state ^= state << 17; return state; }
+static long long checks = 0;
+
+static long long check(int B, int N, int H, int npat, const int* w, const int* r, int causal) {
+  BwdParams p;
+  memset(&p, 0, sizeof(p));
+  p.npat = npat; p.B = B; p.N = N; p.H = H; p.causal = causal;
+  make_geoms(B, N, H, w, r, npat, p.pat);
+  const long long units = build_order(p, npat, B, H);
+  long long base[kMaxPat + 1];
+  base[0] = 0;
+  for (int i = 0; i < npat; ++i)
+    base[i + 1] = base[i] + (long long)p.pat[i].nseg * B * H * p.pat[i].ntiles;
+  long long bad = units != base[npat] ? 1 : 0;
+  std::vector<char> seen((size_t)base[npat], 0);
+  int prev_pat = -1, prev_ntiles = INT_MAX;
+  for (long long uu = 0; uu < units; ++uu) {
+    ++checks;
+    BwdUnit U;
+    const bool has = host_bwd_unit(p, uu, U);
+    const TileUnit& t = U.wu;
+    if (t.pat < 0 || t.pat >= npat || t.seg < 0 || t.seg >= p.pat[t.pat].nseg || t.b < 0 ||
+        t.b >= B || t.h < 0 || t.h >= H || U.u < 0 || U.u >= p.pat[t.pat].ntiles) {
+      if (bad < 3) printf("N=%d uu=%lld out of range\n", N, uu);
+      ++bad;
+      continue;
+    }
+    // patterns in groups, by tile count, descending
+    if (t.pat != prev_pat) {
+      if (p.pat[t.pat].ntiles > prev_ntiles) ++bad;
+      prev_ntiles = p.pat[t.pat].ntiles;
+      prev_pat = t.pat;
+    }
+    const long long idx =
+        base[t.pat] + (((long long)t.seg * B + t.b) * H + t.h) * p.pat[t.pat].ntiles + U.u;
+    if (seen[(size_t)idx]) ++bad;
+    seen[(size_t)idx] = 1;
+    // a unit has rows iff its key tile holds a kept row; then it runs the query
+    // tiles from its own (causal) or the first, through the segment's last
+    const SegInfo si = seg_info(p.pat[t.pat], N, t.h, t.seg);
+    const int nq = (si.n + BM - 1) / BM;
+    if (has != (U.u < nq)) ++bad;
+    if (has && (U.t0 != (causal ? U.u : 0) || U.np != nq - U.t0 || U.np < 1)) ++bad;
+  }
+  for (char c : seen)
+    if (!c) ++bad;
+  return bad;
+}
+
+int main() {
+  long long bad = 0;
+  for (int causal = 0; causal < 2; ++causal) {
+    const int w[] = {2048, 4096, 8192, 16384, 32768}, r[] = {1, 2, 4, 6, 12};
+    bad += check(1, 32768, 12, 5, w, r, causal);
+    bad += check(4, 32768, 12, 5, w, r, causal);
+    const int w4[] = {64, 96, 1100}, r4[] = {5, 200, 7};
+    bad += check(2, 1100, 3, 3, w4, r4, causal);
+    const int w5[] = {1}, r5[] = {1};
+    bad += check(1, 1, 2, 1, w5, r5, causal);
+  }
+  {
+    int w[10], r[10];
+    for (int i = 0; i < 10; ++i) { w[i] = 2048 << i; r[i] = 1 << i; }
+    bad += check(1, 1 << 20, 12, 10, w, r, 1);
+  }
+  for (int c = 0; c < 3000; ++c) {
+    const int N = 1 + (int)(next() % 5000);
+    const int B = 1 + (int)(next() % 3), H = 1 + (int)(next() % 5);
+    const int npat = 1 + (int)(next() % 6);
+    int w[kMaxPat], r[kMaxPat];
+    for (int i = 0; i < npat; ++i) {
+      w[i] = 1 + (int)(next() % (uint64_t)(N + N / 2 + 1));
+      r[i] = 1 + (int)(next() % 300);
+      if (next() % 4 == 0) r[i] = 1;
+    }
+    bad += check(B, N, H, npat, w, r, (int)(next() & 1));
+  }
+  printf("checks %lld bad %lld\n", checks, bad);
+  return bad != 0;
+}
+"""
+
+
+@pytest.mark.skipif(_nvcc() is None, reason="nvcc not found")
+def test_every_backward_unit_decodes_once(tmp_path):
+    src = tmp_path / "bsched.cu"
+    src.write_text(_bwd_program())
+    exe = tmp_path / "bsched"
     build = subprocess.run([_nvcc(), "-O2", "-std=c++17", "-I", CSRC, "-o", str(exe), str(src)],
                            capture_output=True, text=True, timeout=600)
     assert build.returncode == 0, build.stdout + build.stderr

@@ -16,7 +16,12 @@ from the decode part of bwd_unit (csrc/bwd_tc.cuh) and the group-order block of
 launch_bwd: every (pattern, segment, batch, head, key tile) once, patterns in
 groups by descending tile count, a unit with rows exactly when its key tile
 holds a kept row, and its query tiles from its own (causal) or the first
-through the segment's last. No GPU is touched."""
+through the segment's last. A third program checks, for every position of
+every (pattern, head), partial_row (csrc/fwd_tc.cuh: where the merging tiles
+look up another pattern's partial result) against the row the storing tile
+wrote, -1 for rows the pattern does not keep, and view_coords
+(csrc/common.cuh) against the position and the bounds of the view the kernel
+picks. No GPU is touched."""
 import os
 import re
 import shutil
@@ -310,6 +315,121 @@ def test_every_backward_unit_decodes_once(tmp_path):
     src = tmp_path / "bsched.cu"
     src.write_text(_bwd_program())
     exe = tmp_path / "bsched"
+    build = subprocess.run([_nvcc(), "-O2", "-std=c++17", "-I", CSRC, "-o", str(exe), str(src)],
+                           capture_output=True, text=True, timeout=600)
+    assert build.returncode == 0, build.stdout + build.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=600)
+    assert run.returncode == 0, run.stdout + run.stderr
+    assert "bad 0" in run.stdout, run.stdout
+
+
+def _rows_program() -> str:
+    """partial_row (csrc/fwd_tc.cuh) and view_coords (csrc/common.cuh), cut from
+    the sources, with make_geoms from csrc/dilattn.cu."""
+    common = open(os.path.join(CSRC, "common.cuh"), encoding="utf-8").read()
+    fwd = open(os.path.join(CSRC, "fwd_tc.cuh"), encoding="utf-8").read()
+    host = open(os.path.join(CSRC, "dilattn.cu"), encoding="utf-8").read()
+    prow = _cut(fwd, "__device__ __forceinline__ int partial_row(").replace(
+        "__device__ __forceinline__ int partial_row(", "static inline int host_partial_row(")
+    view = _cut(common, "__device__ __forceinline__ void view_coords(").replace(
+        "__device__ __forceinline__ void view_coords(", "static inline void host_view_coords(")
+    funcs = _cut(host, "long long make_geoms(")
+    return r"""
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include "common.cuh"
+namespace dil {
+""" + prow + "\n\n" + view + "\n\n" + funcs + r"""
+}  // namespace dil
+using namespace dil;
+
+static uint64_t state = 0x2545F4914F6CDD1Dull;
+static uint64_t next() { state ^= state << 13; state ^= state >> 7; state ^= state << 17; return state; }
+static long long checks = 0;
+
+// Every position of every (pattern, head): the kept rows' view coordinates and
+// partial rows, and -1 for the rows a pattern does not keep.
+static long long check(int B, int N, int H, int npat, const int* w, const int* r) {
+  PatternGeom geo[kMaxPat];
+  make_geoms(B, N, H, w, r, npat, geo);
+  long long bad = 0;
+  for (int i = 0; i < npat; ++i) {
+    const PatternGeom& g = geo[i];
+    const int nfloor = N / g.r, nmod = N % g.r;
+    for (int b = 0; b < B; b += (B > 1 ? B - 1 : 1)) {   // first and last batch
+      for (int h = 0; h < H; ++h) {
+        const int bh = b * H + h;
+        for (int n = 0; n < N; ++n) {
+          ++checks;
+          const int seg = n / g.w;
+          const SegInfo si = seg_info(g, N, h, seg);
+          const long long rel = n - si.start - si.off;
+          const bool kept = rel >= 0 && rel % g.r == 0;
+          const int got = host_partial_row(g, n, si.off, bh);
+          if (!kept) {
+            if (got != -1) ++bad;
+            continue;
+          }
+          const int v = (int)(rel / g.r);
+          if (v >= si.n) ++bad;
+          const long long want =
+              g.part_base + ((long long)bh * g.nseg + seg) * g.pstride + v;
+          if (got != want) {
+            if (bad < 3) printf("N=%d w=%d r=%d h=%d n=%d partial %d want %lld\n", N, g.w, g.r,
+                                h, n, got, want);
+            ++bad;
+          }
+          int ph, m;
+          host_view_coords(g, si, v, ph, m);
+          const int rows = ph < nmod ? nfloor + 1 : nfloor;   // the view the kernel picks
+          if (ph < 0 || ph >= g.r || (long long)ph + (long long)m * g.r != n || m < 0 ||
+              m >= rows)
+            ++bad;
+        }
+      }
+    }
+  }
+  return bad;
+}
+
+int main() {
+  long long bad = 0;
+  {
+    const int w[] = {2048, 4096, 8192, 16384, 32768}, r[] = {1, 2, 4, 6, 12};
+    bad += check(2, 32768, 12, 5, w, r);
+  }
+  {
+    int w[8], r[8];
+    for (int i = 0; i < 8; ++i) { w[i] = 2048 << i; r[i] = 1 << i; }
+    bad += check(1, 262144, 4, 8, w, r);
+  }
+  {
+    const int w[] = {64, 96, 1100, 384, 700}, r[] = {5, 200, 7, 1, 3};
+    bad += check(3, 1100, 3, 5, w, r);
+  }
+  for (int c = 0; c < 600; ++c) {
+    const int N = 1 + (int)(next() % 3000);
+    const int B = 1 + (int)(next() % 3), H = 1 + (int)(next() % 4);
+    const int npat = 1 + (int)(next() % 6);
+    int w[kMaxPat], r[kMaxPat];
+    for (int i = 0; i < npat; ++i) {
+      w[i] = 1 + (int)(next() % (uint64_t)(N + N / 2 + 1));
+      r[i] = 1 + (int)(next() % 300);
+    }
+    bad += check(B, N, H, npat, w, r);
+  }
+  printf("checks %lld bad %lld\n", checks, bad);
+  return bad != 0;
+}
+"""
+
+
+@pytest.mark.skipif(_nvcc() is None, reason="nvcc not found")
+def test_partial_rows_and_view_coordinates(tmp_path):
+    src = tmp_path / "rows.cu"
+    src.write_text(_rows_program())
+    exe = tmp_path / "rows"
     build = subprocess.run([_nvcc(), "-O2", "-std=c++17", "-I", CSRC, "-o", str(exe), str(src)],
                            capture_output=True, text=True, timeout=600)
     assert build.returncode == 0, build.stdout + build.stderr

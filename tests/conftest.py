@@ -10,4 +10,3 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
-    config.addinivalue_line("markers", "slow: long-running full-size parity case")

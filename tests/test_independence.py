@@ -1,9 +1,10 @@
-"""The oracle and the CUDA path share nothing, on the CPU.
+"""The oracle and the CUDA path share nothing, and the product has no other path, on the CPU.
 
 The product (the package and its CUDA sources) never imports, includes or
 names the oracle; the oracle imports nothing of the package; and bench.py
 imports the oracle only inside its CPU-baseline and reference-arm functions,
-never at module level, so its GPU arm cannot reach it."""
+never at module level, so its GPU arm cannot reach it. Without the built
+library the binding raises on the first call that needs it."""
 import ast
 import os
 import re
@@ -74,3 +75,29 @@ def test_bench_imports_the_oracle_only_in_its_cpu_legs():
                 if isinstance(node, ast.ImportFrom) and node.module == "oracle":
                     found.add(fn.name)
     assert found and found <= allowed, found
+
+
+def test_a_missing_library_fails_loudly(tmp_path):
+    """With no built library there is no other path: a copy of the package's
+    Python files without the library raises on the first call that needs it."""
+    import shutil
+    dst = tmp_path / "sparse_long_sequence_dilated_b200"
+    dst.mkdir()
+    for f in os.listdir(PKG):
+        if f.endswith(".py"):
+            shutil.copy(os.path.join(PKG, f), dst / f)
+    code = (
+        "from sparse_long_sequence_dilated_b200 import dilattn\n"
+        "assert not dilattn.LIB_PATH.startswith(" + repr(ROOT) + ")\n"
+        "for call in (lambda: dilattn.load(), lambda: dilattn.status_string(0),\n"
+        "             lambda: dilattn.bwd_workspace_size(1, 64, 1, 64)):\n"
+        "    try:\n"
+        "        call()\n"
+        "        print('no error')\n"
+        "    except RuntimeError as e:\n"
+        "        print('raised', 'is missing' in str(e))\n")
+    env = dict(os.environ, PYTHONPATH=str(tmp_path))
+    res = subprocess.run([sys.executable, "-c", code], cwd=str(tmp_path), env=env,
+                         capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr
+    assert res.stdout.split() == ["raised", "True"] * 3, res.stdout

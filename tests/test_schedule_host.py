@@ -21,7 +21,8 @@ every (pattern, head), partial_row (csrc/fwd_tc.cuh: where the merging tiles
 look up another pattern's partial result) against the row the storing tile
 wrote, -1 for rows the pattern does not keep, and view_coords
 (csrc/common.cuh) against the position and the bounds of the view the kernel
-picks. No GPU is touched."""
+picks, whose rows are exactly the positions below N of that phase. No GPU is
+touched."""
 import os
 import re
 import shutil
@@ -357,6 +358,13 @@ static long long check(int B, int N, int H, int npat, const int* w, const int* r
   for (int i = 0; i < npat; ++i) {
     const PatternGeom& g = geo[i];
     const int nfloor = N / g.r, nmod = N % g.r;
+    // the view a phase selects holds exactly the positions below N of that phase
+    for (int ph = 0; ph < g.r; ++ph) {
+      ++checks;
+      const int rows = ph < nmod ? nfloor + 1 : nfloor;
+      const int want = ph < N ? (N - ph + g.r - 1) / g.r : 0;
+      if (rows != want) ++bad;
+    }
     for (int b = 0; b < B; b += (B > 1 ? B - 1 : 1)) {   // first and last batch
       for (int h = 0; h < H; ++h) {
         const int bh = b * H + h;

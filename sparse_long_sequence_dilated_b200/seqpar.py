@@ -77,11 +77,37 @@ def packed_positions(p: PatternPlan, L: int, rank: int, h: int):
     return [rank * L + (h % p.r) + m * p.r for m in range(L // p.r)]
 
 
+# subgroups of the default group, one set per segment size: ranks -> (the default
+# group they were made from, this rank's subgroup)
+_SEGMENT_GROUPS: dict = {}
+
+
+def segment_group(ranks: int, world: int, group=None):
+    """The process group a segment of `ranks` consecutive blocks gathers over.
+
+    Segments tile the ranks in consecutive runs, so for the default group the
+    gather runs inside this rank's run only (torch.distributed.new_subgroups,
+    created once per segment size; every rank reaches them in the same order
+    because every rank plans the same patterns). A segment over every rank, or
+    a caller's own group, gathers over that group."""
+    if ranks == world or group is not None:
+        return group
+    import torch.distributed as dist
+    made = _SEGMENT_GROUPS.get(ranks)
+    if made is None or made[0] is not dist.group.WORLD:  # none yet, or a new default group
+        made = (dist.group.WORLD, dist.new_subgroups(group_size=ranks)[0])
+        _SEGMENT_GROUPS[ranks] = made
+    return made[1]
+
+
 def forward(q, k, v, patterns, causal: bool = True, group=None, out=None, lse=None, stream=None):
     """This rank's rows of the dilated-attention forward: (out [B, L, H, d], lse [B, H, L]).
 
     q, k, v: this rank's block [B, L, H, d] (bf16, on its GPU). Collective:
-    every rank of the group calls it with the same patterns, in the same order."""
+    every rank of the group calls it with the same patterns, in the same order.
+    Each spanning pattern's rows are gathered among the ranks of the segment
+    (a subgroup of the default group), so a rank receives (ranks - 1) packs per
+    pattern, not (world - 1)."""
     import torch
     import torch.distributed as dist
 
@@ -96,16 +122,20 @@ def forward(q, k, v, patterns, causal: bool = True, group=None, out=None, lse=No
     for p in plans:
         if not p.spans:
             continue
+        sub = segment_group(p.ranks, world, group)
+        n = p.ranks if sub is not group else world  # ranks taking part in the gather
         bufs = []
         for x in (k, v):
             send = dilattn.pack_dilated(x, p.r, stream=stream)
-            # the ranks' packs concatenated along the batch dimension (the form
-            # every backend takes), the same memory as [world, B, L/r, H, d]
-            recv = torch.empty((world * send.shape[0],) + tuple(send.shape[1:]),
+            # the packs concatenated along the batch dimension (the form every
+            # backend takes), the same memory as [n, B, L/r, H, d] in rank order
+            recv = torch.empty((n * send.shape[0],) + tuple(send.shape[1:]),
                                dtype=send.dtype, device=send.device)
-            dist.all_gather_into_tensor(recv, send, group=group)
-            recv = recv.view((world,) + tuple(send.shape))
-            first = p.segment_ranks(rank)[0]
-            bufs.append(recv[first:first + p.ranks])  # contiguous: [ranks, B, L/r, H, d]
+            dist.all_gather_into_tensor(recv, send, group=sub)
+            recv = recv.view((n,) + tuple(send.shape))
+            if n == world and p.ranks < world:
+                first = p.segment_ranks(rank)[0]
+                recv = recv[first:first + p.ranks]
+            bufs.append(recv)  # contiguous: [ranks, B, L/r, H, d]
         kg[p.index], vg[p.index] = bufs
     return dilattn.fwd_seqpar(q, k, v, patterns, rank, world, kg, vg, causal, out, lse, stream)

@@ -35,6 +35,14 @@ CASES = {
 }
 
 
+@pytest.fixture(autouse=True)
+def _one_blas_thread_per_rank(monkeypatch):
+    """The gloo ranks are processes on the same cores: one BLAS thread each
+    (they inherit the environment when spawned)."""
+    for name in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        monkeypatch.setenv(name, "1")
+
+
 def test_plan_local_and_spanning_patterns():
     pl = seqpar.plan(32768, 4, [(2048, 1), (4096, 2), (8192, 4), (16384, 8), (32768, 16)])
     assert [p.spans for p in pl] == [False, False, False, True, True]
@@ -266,7 +274,7 @@ def _rank_forward(rank: int, world: int, port: int, out_dir: str, case: int, cau
     try:
         from sparse_long_sequence_dilated_b200 import dilattn
 
-        N, _, pats = MATH_CASES[case]
+        N, _, pats = FORWARD_CASES[case]
         B, H, d = 2, 3, 8
         L = N // world
         rng = np.random.default_rng(29)
@@ -308,16 +316,23 @@ def _rank_forward(rank: int, world: int, port: int, out_dir: str, case: int, cau
                 for b in range(B)]
         spans = [not p.spans for p in plans]
         ok_calls = seen == [(rank, world, causal, spans, spans)]
+        # segments over fewer ranks than the group gather inside their own subgroup
+        sub = sorted({p.ranks for p in plans if p.spans and p.ranks < world})
+        ok_calls = ok_calls and sorted(seqpar._SEGMENT_GROUPS) == sub
         with open(os.path.join(out_dir, f"r{rank}.txt"), "w") as f:
             f.write(repr((errs, ok_calls)))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("causal", [True, False])
-@pytest.mark.parametrize("case", range(len(MATH_CASES)))
+# the decomposition cases, and 8 ranks whose segments span 2, 4 and 8 of them
+FORWARD_CASES = MATH_CASES + [(8192, 8, [(512, 1), (2048, 2), (4096, 4), (8192, 8)])]
+
+
+@pytest.mark.parametrize("case,causal", [(c, x) for c in range(len(MATH_CASES))
+                                         for x in (True, False)] + [(len(MATH_CASES), True)])
 def test_seqpar_forward_on_gloo_ranks(tmp_path, case, causal):
-    world = MATH_CASES[case][1]
+    world = FORWARD_CASES[case][1]
     port = _free_port()
     mp.start_processes(_rank_forward, args=(world, port, str(tmp_path), case, causal),
                        nprocs=world, join=True, start_method="spawn")

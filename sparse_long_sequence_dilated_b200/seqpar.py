@@ -9,15 +9,16 @@ with world ranks, rank g holds positions [g L, (g + 1) L), L = N / world.
 * A pattern with w > L has segments spanning min(w, N) / L ranks. Inside a
   block, head h keeps the rows (h mod r) + m r (the block start is a
   multiple of r), so every rank sends just those L / r rows of k and v; the
-  ranks all-gather them in rank order and each rank attends its own kept
-  query rows to the gathered dilated sequence, causal with its block's offset
-  in that sequence.
+  ranks of the segment all-gather them in rank order and each rank attends
+  its own kept query rows to the gathered dilated sequence, causal with its
+  block's offset in that sequence.
 
 Every pattern's result for a row ends up on the rank that owns the row, so
-the cross-pattern merge stays local. The all-gather runs over the whole
-group (torch.distributed: NCCL on GPUs, gloo on the CPU) and each rank keeps
-its segment's slice; the kernels are the library's (dilattn_pack_dilated,
-dilattn_fwd_seqpar). This module holds only the bookkeeping.
+the cross-pattern merge stays local. The all-gathers run with
+torch.distributed (NCCL on GPUs, gloo on the CPU) inside each segment's run
+of consecutive ranks (one set of subgroups per segment size); the kernels
+are the library's (dilattn_pack_dilated, dilattn_fwd_seqpar). This module
+holds only the bookkeeping.
 """
 from __future__ import annotations
 

@@ -21,8 +21,9 @@ every (pattern, head), partial_row (csrc/fwd_tc.cuh: where the merging tiles
 look up another pattern's partial result) against the row the storing tile
 wrote, -1 for rows the pattern does not keep, and view_coords
 (csrc/common.cuh) against the position and the bounds of the view the kernel
-picks, whose rows are exactly the positions below N of that phase. No GPU is
-touched."""
+picks, whose rows are exactly the positions below N of that phase, and
+row_pos (csrc/simt.cuh, the fp32 path's inverse of the position map) against
+seg_info. No GPU is touched."""
 import os
 import re
 import shutil
@@ -334,6 +335,10 @@ def _rows_program() -> str:
         "__device__ __forceinline__ int partial_row(", "static inline int host_partial_row(")
     view = _cut(common, "__device__ __forceinline__ void view_coords(").replace(
         "__device__ __forceinline__ void view_coords(", "static inline void host_view_coords(")
+    simt = open(os.path.join(CSRC, "simt.cuh"), encoding="utf-8").read()
+    rowpos = _cut(simt, "struct RowPos {") + ";\n\n" + _cut(
+        simt, "__device__ __forceinline__ RowPos row_pos(").replace(
+        "__device__ __forceinline__ RowPos row_pos(", "static inline RowPos host_row_pos(")
     funcs = _cut(host, "long long make_geoms(")
     return r"""
 #include <algorithm>
@@ -341,7 +346,7 @@ def _rows_program() -> str:
 #include <cstring>
 #include "common.cuh"
 namespace dil {
-""" + prow + "\n\n" + view + "\n\n" + funcs + r"""
+""" + prow + "\n\n" + view + "\n\n" + rowpos + "\n\n" + funcs + r"""
 }  // namespace dil
 using namespace dil;
 
@@ -375,6 +380,12 @@ static long long check(int B, int N, int H, int npat, const int* w, const int* r
           const long long rel = n - si.start - si.off;
           const bool kept = rel >= 0 && rel % g.r == 0;
           const int got = host_partial_row(g, n, si.off, bh);
+          // the fp32 path's inverse of the position map
+          const RowPos rp = host_row_pos(g, N, h, n);
+          if (rp.kept != kept || rp.seg != seg || rp.start != si.start || rp.off != si.off ||
+              rp.end != std::min<long long>(si.start + g.w, N) ||
+              rp.v != (kept ? (int)(rel / g.r) : -1))
+            ++bad;
           if (!kept) {
             if (got != -1) ++bad;
             continue;

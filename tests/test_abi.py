@@ -223,3 +223,21 @@ def test_effective_pairs_matches_oracle(pats, causal):
     assert flops.effective_pairs(2, 30, 5, pats, causal) == oracle.effective_pairs(2, 30, 5, pats, causal)
     want = sum(int(oracle.multiplicity(30, pats, h, causal).sum()) for h in range(5))
     assert flops.effective_pairs(1, 30, 5, pats, causal) == want
+
+
+def test_pattern_limit_agrees_everywhere():
+    # the header's limit, the binding's and the kernels' per-pattern arrays
+    header = open(HEADER, encoding="utf-8").read()
+    common = open(os.path.join(ROOT, "sparse_long_sequence_dilated_b200", "csrc", "common.cuh"),
+                  encoding="utf-8").read()
+    h = int(re.search(r"#define DILATTN_MAX_PATTERNS (\d+)", header).group(1))
+    k = int(re.search(r"constexpr int kMaxPat = (\d+);", common).group(1))
+    assert h == k == dilattn.MAX_PATTERNS
+
+
+def test_bwd_rejects_head_dim_128_as_unsupported():
+    w, r, n = _pats(((128, 1),))
+    base = [FAKE + i * (4096 * 1024) for i in range(10)]
+    lib = dilattn.load()
+    assert lib.dilattn_bwd(*base, 1, 256, 2, 128, w, r, n, 1, FAKE * 64, 1 << 22,
+                           None) == UNSUPPORTED

@@ -61,3 +61,13 @@ def test_reference_arm_other_ranks_print_nothing():
                          capture_output=True, text=True, timeout=120)
     assert res.returncode == 0, res.stderr[-2000:]
     assert not [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_bench_refuses_fewer_than_three_warmup_steps():
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"],
+                         cwd=ROOT, capture_output=True, text=True, timeout=120,
+                         env=dict(os.environ, CUDA_VISIBLE_DEVICES=""))
+    assert res.returncode == 2 and "--warmup must be at least 3" in res.stderr
+    res = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"], cwd=ROOT,
+                         capture_output=True, text=True, timeout=120)
+    assert res.returncode == 0 and "--impl" in res.stdout and "--reference-seconds" in res.stdout
